@@ -1,0 +1,345 @@
+"""Plain fp64 CPU oracle for absorbed Multi-head Latent Attention decode.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import, call or
+link this module: only ``tests/``, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` use it.  It shares no code with the CUDA path.
+
+Everything here is written from the method's definitions, in float64, with
+library primitives (matmul, exp, log, sin, cos) as single steps and no
+blocking, fusion or reordering beyond what the definitions state:
+
+* Day 27 tutorial "Multi-Head Latent Attention: How DeepSeek Compressed the
+  Cache Further" (kgptalkie):
+    - "Learn a Smaller Shared Representation": one latent ``c_t`` per token;
+    - "The Direct Form Explains the Meaning": per-head content key
+      ``k^C_t = U_K c_t``, scored by a dot product with the query;
+    - "Move the Key Projection Into the Query": ``q . (U_K c) = (U_K^T q) . c``;
+    - "Move the Value Expansion After the Weighted Sum":
+      ``sum_t a_t U_V c_t = U_V sum_t a_t c_t``, and the value up-projection
+      may combine with the output projection;
+    - "Position Rotations Complicate the Absorption": score = content term +
+      rotary term, then scaled, masked and softmaxed;
+    - "Count the Cache That Is Actually Stored": L*T*B*(d_c + d_r)*b bytes.
+* "RedKnot-MLA: Multi-Head Offline-Online Reuse for DeepSeek-V4 Long-Context
+  Serving", abstract: documents cached at canonical position zero,
+  query-side RoPE relocation to the request position, Local heads from an
+  offline (MLA-Off) partial plus protected rows recomputed online, Global
+  heads online, merged before one shared output projection.
+
+Readings where the pages are silent (each one is listed with its reason in
+the design notes): softmax scale 1/sqrt(d_n + d_r); RoPE on adjacent pairs
+(2i, 2i+1) with angle pos * base^(-2i/d_r); cached rotary keys stored already
+rotated at their cache position; visibility ``key_pos <= q_pos``; natural-log
+LSE over scaled scores; an empty visible set gives o = 0 and lse = -inf.
+Parity of those readings is unpinned by the pages: they are declared here and
+held fixed, not derived.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+NEG_INF = -np.inf
+
+
+# ---------------------------------------------------------------------------
+# Cache accounting -- tutorial, "Count the Cache That Is Actually Stored"
+# ---------------------------------------------------------------------------
+
+def cache_bytes(L: int, T: int, B: int, d_c: int, d_r: int, b: int) -> int:
+    """Bytes of a uniform-layer MLA cache: one shared latent (no factor of 2
+    around d_c, since it serves both keys and values) plus one rotary key."""
+    return L * T * B * (d_c + d_r) * b
+
+
+def mha_cache_bytes(L: int, T: int, B: int, heads: int, d_k: int, d_v: int, b: int) -> int:
+    """Ordinary multi-head attention cache: a key and a value per head
+    (tutorial, "Start With What Ordinary Attention Saves")."""
+    return L * T * B * heads * (d_k + d_v) * b
+
+
+# ---------------------------------------------------------------------------
+# Content path -- tutorial, "The Direct Form" and "Move the Key Projection"
+# ---------------------------------------------------------------------------
+
+def content_keys(u_k: np.ndarray, c: np.ndarray) -> np.ndarray:
+    """Direct form: expand every latent row into a content key, k^C_t = U_K c_t.
+
+    u_k: [d_n, d_c] (one head's key up-projection); c: [T, d_c] -> [T, d_n].
+    """
+    return np.asarray(c, np.float64) @ np.asarray(u_k, np.float64).T
+
+
+def values(u_v: np.ndarray, c: np.ndarray) -> np.ndarray:
+    """Direct form: expand every latent row into a value, v_t = U_V c_t."""
+    return np.asarray(c, np.float64) @ np.asarray(u_v, np.float64).T
+
+
+def absorb_query(u_k: np.ndarray, q: np.ndarray) -> np.ndarray:
+    """Projection absorption: transform the query once, U_K^T q.
+
+    u_k: [d_n, d_c]; q: [..., d_n] -> [..., d_c].
+    """
+    return np.asarray(q, np.float64) @ np.asarray(u_k, np.float64)
+
+
+def weighted_latent(a: np.ndarray, c: np.ndarray) -> np.ndarray:
+    """sum_t a_t c_t: mix the narrow latents before any expansion."""
+    return np.asarray(a, np.float64) @ np.asarray(c, np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Rotary path -- tutorial, "Position Rotations Complicate the Absorption";
+# RedKnot-MLA abstract, query-side RoPE relocation
+# ---------------------------------------------------------------------------
+
+def rope_inv_freq(d_r: int, base: float) -> np.ndarray:
+    """theta_i = base^(-2i/d_r) for the d_r/2 feature pairs."""
+    i = np.arange(d_r // 2, dtype=np.float64)
+    return np.power(float(base), -2.0 * i / d_r)
+
+
+def rope_rotate(x: np.ndarray, pos, base: float) -> np.ndarray:
+    """Rotate each adjacent feature pair (2i, 2i+1) by the angle pos*theta_i.
+
+    x: [..., d_r]; pos broadcasts against x[..., 0].  Angles are fp64.
+    """
+    x = np.asarray(x, np.float64)
+    ang = np.asarray(pos, np.float64)[..., None] * rope_inv_freq(x.shape[-1], base)
+    cos, sin = np.cos(ang), np.sin(ang)
+    x0, x1 = x[..., 0::2], x[..., 1::2]
+    out = np.empty(np.broadcast_shapes(x.shape, ang.shape[:-1] + (x.shape[-1],)), np.float64)
+    out[..., 0::2] = x0 * cos - x1 * sin
+    out[..., 1::2] = x0 * sin + x1 * cos
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Softmax and log-sum-exp
+# ---------------------------------------------------------------------------
+
+def softmax_lse(s: np.ndarray):
+    """Row softmax and natural-log LSE of scaled, masked scores (-inf = masked).
+
+    Returns (weights, lse).  A row with every entry masked gets weights 0 and
+    lse = -inf.
+    """
+    s = np.asarray(s, np.float64)
+    m = np.max(s, axis=-1, keepdims=True) if s.shape[-1] else np.full(s.shape[:-1] + (1,), NEG_INF)
+    empty = ~np.isfinite(m)
+    m_safe = np.where(empty, 0.0, m)
+    e = np.exp(s - m_safe)
+    tot = np.sum(e, axis=-1, keepdims=True)
+    with np.errstate(divide="ignore"):
+        lse = np.where(empty, NEG_INF, m_safe + np.log(np.where(empty, 1.0, tot)))
+    a = np.where(empty, 0.0, e / np.where(empty, 1.0, tot))
+    return a, lse[..., 0]
+
+
+def merge_lse(o_a, lse_a, o_b, lse_b):
+    """Merge two partial attentions over disjoint key sets.
+
+    (o_x, lse_x) is a normalised output and the LSE of its key set; the
+    result is the attention over the union (RedKnot-MLA abstract: the offline
+    and online paths are merged before the shared output projection).
+    o_*: [..., d]; lse_*: [...].
+    """
+    lse_a = np.asarray(lse_a, np.float64)
+    lse_b = np.asarray(lse_b, np.float64)
+    lse = np.logaddexp(lse_a, lse_b)
+    empty = ~np.isfinite(lse)
+    ref = np.where(empty, 0.0, lse)
+    w_a = np.where(empty, 0.0, np.exp(lse_a - ref))
+    w_b = np.where(empty, 0.0, np.exp(lse_b - ref))
+    o = w_a[..., None] * np.asarray(o_a, np.float64) + w_b[..., None] * np.asarray(o_b, np.float64)
+    return o, lse
+
+
+# ---------------------------------------------------------------------------
+# Paged cache bookkeeping (row -> page, slot; segment -> key position)
+# ---------------------------------------------------------------------------
+
+def sequence_rows(segs_b: np.ndarray, gather_b=None):
+    """Logical rows of one sequence with their key positions and query versions.
+
+    segs_b: [n_seg, 4] of (row_begin, row_end, q_version, key_pos_base).
+    Row r of segment s sits at request position key_pos_base + (r - row_begin)
+    and was cached with its rotary key at that position minus the relocation
+    offset of version q_version.  With ``gather_b`` the row set is that list.
+    Returns (rows, key_pos, version) as int64 arrays.
+    """
+    rows, kpos, ver = [], [], []
+    if gather_b is None:
+        for rb, re, v, kb in segs_b:
+            for r in range(int(rb), int(re)):
+                rows.append(r)
+                kpos.append(int(kb) + r - int(rb))
+                ver.append(int(v))
+    else:
+        for r in gather_b:
+            r = int(r)
+            hit = [s for s in segs_b if int(s[0]) <= r < int(s[1])]
+            if len(hit) != 1:
+                raise ValueError(f"gathered row {r} is in {len(hit)} segments")
+            rb, re, v, kb = (int(x) for x in hit[0])
+            rows.append(r)
+            kpos.append(kb + r - rb)
+            ver.append(v)
+    return (np.array(rows, np.int64), np.array(kpos, np.int64), np.array(ver, np.int64))
+
+
+def gather_cache(pool: np.ndarray, block_table_b: np.ndarray, rows: np.ndarray,
+                 page: int = 64) -> np.ndarray:
+    """Cached rows [T, d_c + d_r] of one sequence, read through its block table."""
+    pages = np.asarray(block_table_b)[rows // page]
+    return np.asarray(pool[pages, rows % page], np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Attention for one sequence, one head
+# ---------------------------------------------------------------------------
+
+def attend_direct(q_nope, q_rope, q_pos, u_k, u_v, c, k_rope, key_pos, key_shift,
+                  scale, base):
+    """Direct (expanded-key) form for one head of one sequence.
+
+    q_nope [S, d_n], q_rope [S, d_r], q_pos [S]; c [T, d_c]; k_rope [T, d_r]
+    as cached (rotated at key_pos - key_shift); key_pos, key_shift [T].
+    The cached rotary key is first restored to its request position by
+    rotating it forward by key_shift (the key-side repair that query-side
+    relocation avoids); the query is rotated at its own position.
+    Returns (o_lat [S, d_c], o [S, d_v], lse [S]).
+    """
+    k_content = content_keys(u_k, c)                        # [T, d_n]
+    v_full = values(u_v, c)                                 # [T, d_v]
+    k_r = rope_rotate(k_rope, key_shift, base)              # [T, d_r]
+    q_r = rope_rotate(q_rope, q_pos, base)                  # [S, d_r]
+    s = scale * (np.asarray(q_nope, np.float64) @ k_content.T + q_r @ k_r.T)
+    visible = np.asarray(key_pos)[None, :] <= np.asarray(q_pos)[:, None]
+    s = np.where(visible, s, NEG_INF)
+    a, lse = softmax_lse(s)
+    return weighted_latent(a, c), a @ v_full, lse
+
+
+def attend_absorbed(q_lat, q_r_by_row, c, k_rope, key_pos, q_pos, scale):
+    """Absorbed form for one head of one sequence.
+
+    q_lat [S, d_c] = U_K^T q_nope; q_r_by_row [S, T, d_r] is, for each key
+    row, the query's rotary part rotated at q_pos - (that row's relocation
+    offset).  Scores are taken directly against the cached c and k_rope.
+    Returns (o_lat [S, d_c], lse [S]).
+    """
+    c = np.asarray(c, np.float64)
+    s = scale * (np.asarray(q_lat, np.float64) @ c.T
+                 + np.einsum("std,td->st", q_r_by_row, np.asarray(k_rope, np.float64)))
+    visible = np.asarray(key_pos)[None, :] <= np.asarray(q_pos)[:, None]
+    s = np.where(visible, s, NEG_INF)
+    a, lse = softmax_lse(s)
+    return weighted_latent(a, c), lse
+
+
+# ---------------------------------------------------------------------------
+# Whole decode over the paged cache
+# ---------------------------------------------------------------------------
+
+def decode(inp, heads=None, rows_override=None, form="direct", seqs=None):
+    """Attention outputs for every (query token, head) of a decode step.
+
+    ``inp`` is a workloads.DecodeInputs (plain arrays).  ``heads`` selects
+    logical head ids (default all).  ``rows_override`` maps a sequence index
+    to an explicit list of logical rows (a key subset, e.g. protected rows or
+    the offline complement); otherwise the sequence's gather list, else all
+    its segment rows.  ``seqs`` restricts the sequences computed.
+    Returns o_lat [n_q, n_h, d_c], lse [n_q, n_h] (and o [n_q, n_h, d_v] for
+    the direct form), NaN where a sequence was skipped.
+    """
+    wl = inp.wl
+    heads = list(range(wl.H)) if heads is None else list(heads)
+    n_h = len(heads)
+    n_q = inp.n_q
+    o_lat = np.full((n_q, n_h, wl.d_c), np.nan)
+    lse = np.full((n_q, n_h), np.nan)
+    o_val = np.full((n_q, n_h, wl.d_v), np.nan)
+    seqs = range(wl.B) if seqs is None else seqs
+    for b in seqs:
+        if rows_override is not None and b in rows_override:
+            rows, kpos, ver = sequence_rows(inp.segs[b], rows_override[b])
+        elif inp.gather_rows is not None:
+            g = inp.gather_rows[b, :int(inp.n_gather[b])]
+            rows, kpos, ver = sequence_rows(inp.segs[b], g)
+        else:
+            rows, kpos, ver = sequence_rows(inp.segs[b])
+        cache = gather_cache(inp.pool, inp.block_table[b], rows)
+        c, k_rope = cache[:, :wl.d_c], cache[:, wl.d_c:]
+        shift = np.asarray(inp.deltas, np.int64)[ver]
+        qs = slice(b * wl.s_q, (b + 1) * wl.s_q)
+        q_pos = np.asarray(inp.q_pos[qs], np.int64)
+        for i, h in enumerate(heads):
+            if form == "direct":
+                ol, ov, ls = attend_direct(inp.q_nope[qs, h], inp.q_rope[qs, h], q_pos,
+                                           inp.w_uk[h], inp.w_uv[h], c, k_rope, kpos,
+                                           shift, wl.scale, wl.rope_base)
+                o_val[qs, i] = ov
+            else:
+                q_lat = absorb_query(inp.w_uk[h], inp.q_nope[qs, h])
+                rel = q_pos[:, None] - shift[None, :]              # [S, T]
+                q_r = rope_rotate(np.asarray(inp.q_rope[qs, h], np.float64)[:, None, :],
+                                  rel, wl.rope_base)               # [S, T, d_r]
+                ol, ls = attend_absorbed(q_lat, q_r, c, k_rope, kpos, q_pos, wl.scale)
+            o_lat[qs, i] = ol
+            lse[qs, i] = ls
+    if form == "direct":
+        return o_lat, lse, o_val
+    return o_lat, lse
+
+
+def decode_absorbed_fast(inp, heads=None, seqs=None):
+    """Absorbed form, vectorised over heads (same definition as ``decode``
+    with form="absorbed", grouped by relocation version so the rotary query
+    is formed once per version rather than once per key row).  Used where the
+    per-row form is too slow (long contexts) and as the timed CPU baseline.
+    Returns o_lat [n_q, n_h, d_c], lse [n_q, n_h].
+    """
+    wl = inp.wl
+    heads = np.arange(wl.H) if heads is None else np.asarray(list(heads))
+    n_q = inp.n_q
+    o_lat = np.full((n_q, len(heads), wl.d_c), np.nan)
+    lse = np.full((n_q, len(heads)), np.nan)
+    seqs = range(wl.B) if seqs is None else seqs
+    w_uk = np.asarray(inp.w_uk[heads], np.float64)                    # [n_h, d_n, d_c]
+    for b in seqs:
+        if inp.gather_rows is not None:
+            rows, kpos, ver = sequence_rows(inp.segs[b], inp.gather_rows[b, :int(inp.n_gather[b])])
+        else:
+            rows, kpos, ver = sequence_rows(inp.segs[b])
+        cache = gather_cache(inp.pool, inp.block_table[b], rows)
+        c, k_rope = cache[:, :wl.d_c], cache[:, wl.d_c:]
+        for j in range(wl.s_q):
+            qi = b * wl.s_q + j
+            p = int(inp.q_pos[qi])
+            qn = np.asarray(inp.q_nope[qi, heads], np.float64)            # [n_h, d_n]
+            q_lat = np.einsum("hn,hnc->hc", qn, w_uk)                    # U_K^T q per head
+            s = q_lat @ c.T                                              # content term
+            for v in np.unique(ver):
+                sel = ver == v
+                q_r = rope_rotate(np.asarray(inp.q_rope[qi, heads], np.float64),
+                                  p - int(inp.deltas[v]), wl.rope_base)    # [n_h, d_r]
+                s[:, sel] += q_r @ k_rope[sel].T                         # rotary term
+            s = np.where((kpos <= p)[None, :], wl.scale * s, NEG_INF)
+            a, ls = softmax_lse(s)
+            o_lat[qi] = a @ c
+            lse[qi] = ls
+    return o_lat, lse
+
+
+def out_proj(o_lat, w_uv, w_o):
+    """Value up-projection per head, then the shared output projection.
+
+    o_lat [n_q, H, d_c]; w_uv [H, d_v, d_c]; w_o [d_model, H*d_v].
+    Returns v [n_q, H, d_v] and out [n_q, d_model] (tutorial, "Move the Value
+    Expansion After the Weighted Sum": expand the one mixed latent, then the
+    head's contribution joins the final output projection).
+    """
+    o_lat = np.asarray(o_lat, np.float64)
+    v = np.einsum("hdc,qhc->qhd", np.asarray(w_uv, np.float64), o_lat)
+    out = v.reshape(v.shape[0], -1) @ np.asarray(w_o, np.float64).T
+    return v, out

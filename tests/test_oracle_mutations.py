@@ -1,0 +1,131 @@
+"""Planted mistakes in the oracle must fail at least one pin.
+
+Each mutant replaces one oracle function (on the CPU, for the duration of
+one test) with a plausible wrong variant: a sign, a dropped term, a
+transposed operand, a wrong index or comparison.  The pins of
+``test_oracle_pins`` are then re-run and at least one must fail.
+"""
+import numpy as np
+import pytest
+
+from oracle import mla_oracle as O
+import tests.test_oracle_pins as P
+
+PINS = [
+    P.test_worked_absorption_example,
+    P.test_worked_value_example,
+    lambda: P.test_rope_matches_complex_rotation(4095),
+    lambda: P.test_rope_relative_position_invariance(1000),
+    P.test_relocation_offset_invariance,
+    P.test_matches_torch_sdpa_with_expanded_keys,
+    P.test_softmax_rows_sum_to_one_and_lse_closed_form,
+    P.test_zero_query_gives_mean_of_visible_rows,
+    P.test_merge_of_any_split_equals_unsplit,
+    P.test_merge_with_empty_is_identity,
+    P.test_out_proj_fold_identity,
+]
+
+
+def _rope_sign(x, pos, base):
+    x = np.asarray(x, np.float64)
+    ang = np.asarray(pos, np.float64)[..., None] * O.rope_inv_freq(x.shape[-1], base)
+    out = np.empty(np.broadcast_shapes(x.shape, ang.shape[:-1] + (x.shape[-1],)))
+    out[..., 0::2] = x[..., 0::2] * np.cos(ang) + x[..., 1::2] * np.sin(ang)
+    out[..., 1::2] = -x[..., 0::2] * np.sin(ang) + x[..., 1::2] * np.cos(ang)
+    return out
+
+
+def _rope_half(x, pos, base):
+    x = np.asarray(x, np.float64)
+    d = x.shape[-1]
+    ang = np.asarray(pos, np.float64)[..., None] * O.rope_inv_freq(d, base)
+    a, b = x[..., :d // 2], x[..., d // 2:]
+    return np.concatenate([a * np.cos(ang) - b * np.sin(ang), a * np.sin(ang) + b * np.cos(ang)], -1)
+
+
+def _freq_off_by_one(d_r, base):
+    i = np.arange(1, d_r // 2 + 1, dtype=np.float64)
+    return np.power(float(base), -2.0 * i / d_r)
+
+
+def _direct_no_rope(q_nope, q_rope, q_pos, u_k, u_v, c, k_rope, key_pos, key_shift, scale, base):
+    return _ORIG["attend_direct"](q_nope, np.zeros_like(q_rope), q_pos, u_k, u_v, c,
+                                  k_rope, key_pos, key_shift, scale, base)
+
+
+def _direct_shift_sign(q_nope, q_rope, q_pos, u_k, u_v, c, k_rope, key_pos, key_shift, scale, base):
+    return _ORIG["attend_direct"](q_nope, q_rope, q_pos, u_k, u_v, c, k_rope, key_pos,
+                                  -np.asarray(key_shift), scale, base)
+
+
+def _direct_strict_mask(q_nope, q_rope, q_pos, u_k, u_v, c, k_rope, key_pos, key_shift, scale, base):
+    return _ORIG["attend_direct"](q_nope, q_rope, q_pos, u_k, u_v, c, k_rope,
+                                  np.asarray(key_pos) + 1, key_shift, scale, base)
+
+
+def _direct_no_scale(q_nope, q_rope, q_pos, u_k, u_v, c, k_rope, key_pos, key_shift, scale, base):
+    return _ORIG["attend_direct"](q_nope, q_rope, q_pos, u_k, u_v, c, k_rope, key_pos,
+                                  key_shift, 1.0, base)
+
+
+def _content_keys_T(u_k, c):
+    return np.asarray(c, np.float64) @ np.asarray(u_k, np.float64).T[::-1]
+
+
+def _absorb_T(u_k, q):
+    return np.asarray(q, np.float64) @ np.asarray(u_k, np.float64)[::-1]
+
+
+def _values_T(u_v, c):
+    return np.asarray(c, np.float64)[:, ::-1] @ np.asarray(u_v, np.float64).T
+
+
+def _merge_swapped(o_a, lse_a, o_b, lse_b):
+    o, l = _ORIG["merge_lse"](o_a, lse_a, o_b, lse_b)
+    la, lb = np.asarray(lse_a), np.asarray(lse_b)
+    wa = np.exp(la - l)
+    wb = np.exp(lb - l)
+    return wb[..., None] * np.asarray(o_a) + wa[..., None] * np.asarray(o_b), l
+
+
+def _softmax_no_max(s):
+    a, lse = _ORIG["softmax_lse"](s)
+    m = np.max(np.where(np.isfinite(s), s, -1e300), axis=-1)
+    return a, lse - np.where(np.isfinite(m), m, 0.0)
+
+
+def _out_proj_T(o_lat, w_uv, w_o):
+    v = np.einsum("hdc,qhc->qdh", np.asarray(w_uv, np.float64), np.asarray(o_lat, np.float64))
+    return v, v.reshape(v.shape[0], -1) @ np.asarray(w_o, np.float64).T
+
+
+_ORIG = {k: getattr(O, k) for k in ("attend_direct", "merge_lse", "softmax_lse")}
+
+MUTANTS = {
+    "rope_sign": ("rope_rotate", _rope_sign),
+    "rope_rotate_half": ("rope_rotate", _rope_half),
+    "rope_freq_index": ("rope_inv_freq", _freq_off_by_one),
+    "drop_rotary_term": ("attend_direct", _direct_no_rope),
+    "relocation_sign": ("attend_direct", _direct_shift_sign),
+    "strict_mask": ("attend_direct", _direct_strict_mask),
+    "scale_dropped": ("attend_direct", _direct_no_scale),
+    "content_key_rows": ("content_keys", _content_keys_T),
+    "absorb_rows": ("absorb_query", _absorb_T),
+    "value_cols": ("values", _values_T),
+    "merge_weights_swapped": ("merge_lse", _merge_swapped),
+    "lse_without_max": ("softmax_lse", _softmax_no_max),
+    "out_proj_transposed": ("out_proj", _out_proj_T),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(O, attr, fn)
+    failed = []
+    for pin in PINS:
+        try:
+            pin()
+        except Exception:            # an assertion or a shape error both count
+            failed.append(pin)
+    assert failed, f"mutant {name} passed every pin"

@@ -1,0 +1,283 @@
+"""Pins of the fp64 oracle to facts fixed outside the oracle itself.
+
+Each test ties a part of the oracle to a value the pages print, a closed
+form, an invariant, or a special case that reduces to a library routine
+(torch's scaled_dot_product_attention, Python's complex exponential), so
+that a dropped term, a wrong sign or index, or a transposed operand fails.
+CPU only.
+"""
+import cmath
+import copy
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import mla_oracle as O
+from head_latent_attention_02_b200.workloads import Workload, make_inputs
+
+GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")))
+
+
+# --------------------------------------------------------------- worked examples
+
+def test_worked_absorption_example():
+    g = GOLD["absorption"]
+    u_k, c, q = np.array(g["u_k"]), np.array(g["c"]), np.array(g["q"])
+    k = O.content_keys(u_k, c[None, :])[0]
+    assert np.array_equal(k, g["content_key"])
+    assert float(q @ k) == g["direct_score"]
+    qa = O.absorb_query(u_k, q)
+    assert np.array_equal(qa, g["absorbed_query"])
+    assert float(qa @ c) == g["absorbed_score"]
+
+
+def test_worked_value_example():
+    g = GOLD["value"]
+    c, a, u_v = np.array(g["c"]), np.array(g["weights"]), np.array(g["u_v"])
+    lat = O.weighted_latent(a, c)
+    assert np.allclose(lat, g["weighted_latent"], rtol=0, atol=1e-15)
+    out = O.values(u_v, lat[None, :])[0]
+    assert np.allclose(out, g["value_out"], rtol=0, atol=1e-15)
+    # linearity: expanding each latent then mixing gives the same output
+    per_row = O.values(u_v, c)
+    assert np.allclose(a @ per_row, g["value_out"], rtol=0, atol=1e-15)
+
+
+def test_cache_count_example():
+    g = GOLD["cache_count"]
+    assert O.cache_bytes(1, 1, 1, g["d_c"], g["d_r"], g["bytes_per_number"]) == g["mla_bytes_per_layer_token"]
+    assert O.mha_cache_bytes(1, 1, 1, g["mha_heads"], g["mha_key"], g["mha_value"],
+                             g["bytes_per_number"]) == g["mha_bytes_per_layer_token"]
+    assert O.mha_cache_bytes(1, 1, 1, 2, 4, 4, 1) == g["mha_numbers_per_layer_token"]
+    # the headline layout: 576 bf16 numbers = 1152 bytes per layer-token
+    assert O.cache_bytes(1, 1, 1, 512, 64, 2) == 1152
+
+
+# --------------------------------------------------------------------- RoPE
+
+def _rope_complex(x, pos, base):
+    """Pairs (2i, 2i+1) as complex numbers times exp(i*pos*theta_i)."""
+    d = len(x)
+    out = []
+    for i in range(d // 2):
+        th = base ** (-2.0 * i / d)
+        z = complex(x[2 * i], x[2 * i + 1]) * cmath.exp(1j * pos * th)
+        out += [z.real, z.imag]
+    return np.array(out)
+
+
+@pytest.mark.parametrize("pos", [0, 1, 7, 4095, 24575, 262143])
+def test_rope_matches_complex_rotation(pos):
+    rng = np.random.default_rng(pos)
+    x = rng.standard_normal(64)
+    got = O.rope_rotate(x, pos, 10000.0)
+    ref = _rope_complex(x, pos, 10000.0)
+    assert np.allclose(got, ref, rtol=0, atol=1e-9)
+    assert math.isclose(np.linalg.norm(got), np.linalg.norm(x), rel_tol=1e-12)
+
+
+def test_rope_position_zero_is_identity_and_composes():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((5, 16))
+    assert np.array_equal(O.rope_rotate(x, 0, 10000.0), x)
+    a, b = 1234, 56789
+    two = O.rope_rotate(O.rope_rotate(x, a, 10000.0), b, 10000.0)
+    assert np.allclose(two, O.rope_rotate(x, a + b, 10000.0), rtol=0, atol=1e-9)
+
+
+def _tiny(B=2, H=3, d_c=8, d_r=4, d_n=5, d_v=6, s_q=1, lengths=(13, 70), **kw):
+    wl = Workload("t", "f32", B=B, H=H, d_c=d_c, d_r=d_r, d_n=d_n, d_v=d_v,
+                  d_model=H * d_v, s_q=s_q, lengths=None if lengths is None else list(lengths), **kw)
+    return make_inputs(wl, seed=3)
+
+
+def _shift_positions(inp, delta_pos):
+    """Every request position (queries and keys) moves by delta_pos; the cache
+    rows, rotated at their cache positions, move with them."""
+    out = copy.deepcopy(inp)
+    wl = inp.wl
+    out.q_pos = inp.q_pos + delta_pos
+    out.segs = inp.segs.copy()
+    out.segs[:, :, 3] += delta_pos
+    used = ~np.isnan(inp.pool[:, :, 0])
+    kr = inp.pool[:, :, wl.d_c:].astype(np.float64)
+    rot = O.rope_rotate(kr, delta_pos, wl.rope_base)
+    out.pool = inp.pool.astype(np.float64)
+    out.pool[:, :, wl.d_c:] = np.where(used[..., None], rot, np.nan)
+    return out
+
+
+@pytest.mark.parametrize("dpos", [5, 1000, 250000])
+def test_rope_relative_position_invariance(dpos):
+    inp = _tiny()
+    o1, l1, v1 = O.decode(inp)
+    o2, l2, v2 = O.decode(_shift_positions(inp, dpos))
+    assert np.allclose(o1, o2, rtol=0, atol=1e-9)
+    assert np.allclose(l1, l2, rtol=0, atol=1e-9)
+
+
+def test_relocation_offset_invariance():
+    """A document whose rotary keys were cached at canonical positions gives the
+    same result as the same document cached at its request positions with no
+    relocation (query-side repair equals key-side repair)."""
+    wl = Workload("t", "f32", B=1, H=2, d_c=8, d_r=4, d_n=5, d_v=6, d_model=12,
+                  prefix=64, doc=128)
+    inp = make_inputs(wl, seed=5)
+    o_rel, l_rel, _ = O.decode(inp)
+    flat = copy.deepcopy(inp)
+    # rotate the document rows forward by the offset and drop the relocation
+    doc_pages = inp.block_table[0, 1:3]
+    flat.pool = inp.pool.astype(np.float64)
+    flat.pool[doc_pages, :, wl.d_c:] = O.rope_rotate(inp.pool[doc_pages, :, wl.d_c:], 64, wl.rope_base)
+    flat.deltas = np.array([0, 0], np.int32)
+    o_flat, l_flat, _ = O.decode(flat)
+    assert np.allclose(o_rel, o_flat, rtol=0, atol=1e-10)
+    assert np.allclose(l_rel, l_flat, rtol=0, atol=1e-10)
+
+
+# ------------------------------------------------ special case: library attention
+
+def test_matches_torch_sdpa_with_expanded_keys():
+    """With keys and values expanded explicitly and the rotation done by complex
+    multiplication, the oracle equals torch's scaled_dot_product_attention."""
+    inp = _tiny(s_q=2, lengths=(13, 70))
+    wl = inp.wl
+    o_lat, lse, o_val = O.decode(inp)
+    for b in range(wl.B):
+        rows = int(inp.n_rows[b])
+        r = np.arange(rows)
+        cache = inp.pool[inp.block_table[b, r // 64], r % 64].astype(np.float64)
+        c, kr = cache[:, :wl.d_c], cache[:, wl.d_c:]
+        qs = slice(b * wl.s_q, (b + 1) * wl.s_q)
+        qp = inp.q_pos[qs]
+        mask = torch.tensor(r[None, :] <= qp[:, None])
+        for h in range(wl.H):
+            k = np.concatenate([c @ inp.w_uk[h].astype(np.float64).T,
+                                np.stack([_rope_complex(kr[t], 0, wl.rope_base) for t in r])], 1)
+            q = np.concatenate([inp.q_nope[qs, h].astype(np.float64),
+                                np.stack([_rope_complex(inp.q_rope[qs][j, h], qp[j], wl.rope_base)
+                                          for j in range(wl.s_q)])], 1)
+            v = c @ inp.w_uv[h].astype(np.float64).T
+            T = torch.from_numpy
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                T(q)[None], T(k)[None], T(v)[None], attn_mask=mask[None], scale=wl.scale)[0]
+            ref_lat = torch.nn.functional.scaled_dot_product_attention(
+                T(q)[None], T(k)[None], T(c)[None], attn_mask=mask[None], scale=wl.scale)[0]
+            assert np.allclose(o_val[qs, h], ref.numpy(), rtol=0, atol=1e-12)
+            assert np.allclose(o_lat[qs, h], ref_lat.numpy(), rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------- softmax closed forms
+
+def test_softmax_rows_sum_to_one_and_lse_closed_form():
+    rng = np.random.default_rng(0)
+    s = rng.standard_normal((4, 37)) * 5
+    a, lse = O.softmax_lse(s)
+    assert np.allclose(a.sum(-1), 1.0, rtol=0, atol=1e-14)
+    same = np.full((2, 9), 0.7)
+    a2, l2 = O.softmax_lse(same)
+    assert np.allclose(a2, 1 / 9, rtol=0, atol=1e-15)
+    assert np.allclose(l2, 0.7 + math.log(9), rtol=0, atol=1e-14)
+    a3, l3 = O.softmax_lse(np.full((1, 3), -np.inf))
+    assert np.all(a3 == 0) and np.all(l3 == -np.inf)
+
+
+def test_single_row_returns_its_latent():
+    inp = _tiny(lengths=(1, 1))
+    o_lat, lse, _ = O.decode(inp)
+    for b in range(2):
+        c = inp.pool[inp.block_table[b, 0], 0, :inp.wl.d_c]
+        assert np.array_equal(o_lat[b, :, :], np.broadcast_to(c, o_lat[b].shape))
+
+
+def test_zero_query_gives_mean_of_visible_rows():
+    inp = _tiny(s_q=2, lengths=(13, 70))
+    inp.q_nope[:] = 0
+    inp.q_rope[:] = 0
+    o_lat, lse, _ = O.decode(inp)
+    wl = inp.wl
+    for b in range(wl.B):
+        rows = int(inp.n_rows[b])
+        for j in range(wl.s_q):
+            qi = b * wl.s_q + j
+            vis = np.arange(int(inp.q_pos[qi]) + 1)      # key_pos <= q_pos
+            vis = vis[vis < rows]
+            c = inp.pool[inp.block_table[b, vis // 64], vis % 64, :wl.d_c].astype(np.float64)
+            assert np.allclose(o_lat[qi], c.mean(0), rtol=0, atol=1e-13)
+            assert np.allclose(lse[qi], math.log(len(vis)), rtol=0, atol=1e-13)
+    # the last query of a sequence sees one more row than the one before it
+    assert int(inp.q_pos[1]) == int(inp.n_rows[0]) - 1
+
+
+# -------------------------------------------------------------- merge and forms
+
+def test_merge_of_any_split_equals_unsplit():
+    inp = _tiny(lengths=(13, 70))
+    full_lat, full_lse, _ = O.decode(inp)
+    rng = np.random.default_rng(7)
+    for b in range(2):
+        rows = np.arange(int(inp.n_rows[b]))
+        mask = rng.random(len(rows)) < 0.4
+        mask[0], mask[-1] = True, False
+        a_lat, a_lse, _ = O.decode(inp, rows_override={b: rows[mask]}, seqs=[b])
+        b_lat, b_lse, _ = O.decode(inp, rows_override={b: rows[~mask]}, seqs=[b])
+        m_lat, m_lse = O.merge_lse(a_lat[b], a_lse[b], b_lat[b], b_lse[b])
+        assert np.allclose(m_lat, full_lat[b], rtol=0, atol=1e-12)
+        assert np.allclose(m_lse, full_lse[b], rtol=0, atol=1e-12)
+
+
+def test_merge_with_empty_is_identity():
+    rng = np.random.default_rng(2)
+    o, l = rng.standard_normal((3, 5)), rng.standard_normal(3)
+    ninf = np.full(3, -np.inf)
+    m, ml = O.merge_lse(o, l, np.zeros((3, 5)), ninf)
+    assert np.array_equal(ml, l) and np.allclose(m, o, rtol=0, atol=0)
+    m2, ml2 = O.merge_lse(np.zeros((3, 5)), ninf, np.zeros((3, 5)), ninf)
+    assert np.all(ml2 == -np.inf) and np.all(m2 == 0)
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(s_q=2, lengths=(64, 129)),
+                                dict(prefix=64, doc=128, B=1, lengths=None)])
+def test_absorbed_equals_direct(kw):
+    inp = _tiny(**kw)
+    d_lat, d_lse, _ = O.decode(inp)
+    a_lat, a_lse = O.decode(inp, form="absorbed")
+    f_lat, f_lse = O.decode_absorbed_fast(inp)
+    for lat, lse in ((a_lat, a_lse), (f_lat, f_lse)):
+        assert np.allclose(lat, d_lat, rtol=1e-10, atol=1e-12)
+        assert np.allclose(lse, d_lse, rtol=1e-10, atol=1e-12)
+
+
+# ---------------------------------------------------------------- bookkeeping
+
+def test_page_placement_and_poison_do_not_matter():
+    a = _tiny(lengths=(13, 200))
+    b = copy.deepcopy(a)
+    perm = np.random.default_rng(9).permutation(a.pool.shape[0])
+    inv = np.argsort(perm)
+    b.pool = a.pool[perm]                       # page p moves to slot inv[p]
+    b.block_table = inv[a.block_table].astype(np.int32)
+    oa, la, _ = O.decode(a)
+    ob, lb, _ = O.decode(b)
+    assert np.isfinite(oa).all() and np.array_equal(oa, ob) and np.array_equal(la, lb)
+
+
+def test_out_proj_fold_identity():
+    """The value up-projection folds into the shared output projection:
+    W_O . concat_h(W_UV[h] o_h) == sum_h (W_O[:, h] W_UV[h]) o_h."""
+    rng = np.random.default_rng(4)
+    H, d_v, d_c, d_model, n = 3, 4, 6, 5, 2
+    w_uv = rng.standard_normal((H, d_v, d_c))
+    w_o = rng.standard_normal((d_model, H * d_v))
+    o = rng.standard_normal((n, H, d_c))
+    v, out = O.out_proj(o, w_uv, w_o)
+    folded = sum(o[:, h] @ (w_o[:, h * d_v:(h + 1) * d_v] @ w_uv[h]).T for h in range(H))
+    assert np.allclose(out, folded, rtol=0, atol=1e-12)
+    g = GOLD["value"]
+    v1, _ = O.out_proj(np.array(g["weighted_latent"])[None, None, :],
+                       np.array(g["u_v"])[None], np.eye(4))
+    assert np.allclose(v1[0, 0], g["value_out"], rtol=0, atol=1e-15)
