@@ -1,0 +1,332 @@
+// mla_lib.cu -- the C ABI of libmla (include/mla.h): argument validation,
+// TMA descriptor set-up and kernel launches.  Single translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "mla.h"
+#include "common.cuh"
+#include "ptx.cuh"
+#include "kernels_simt.cuh"
+#include "decode_tc.cuh"
+
+using namespace mla;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+  bool tc_attr_set = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+mla_status_t device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    d.ready = true;
+  }
+  *out = &d;
+  return MLA_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool dims_ok(const mla_dims_t* d) {
+  return d && d->H > 0 && d->d_c > 0 && d->d_r >= 0 && d->d_r % 2 == 0 && d->d_n > 0 &&
+         d->d_v > 0 && d->d_model >= 0 && (d->dtype == MLA_F32 || d->dtype == MLA_BF16) &&
+         std::isfinite(d->scale) && d->rope_base > 0.0;
+}
+
+size_t elem_size(const mla_dims_t* d) { return d->dtype == MLA_BF16 ? 2 : 4; }
+
+bool tc_eligible(const mla_dims_t* d) {
+  return d->dtype == MLA_BF16 && d->d_c == tc::kDc && d->d_r == tc::kDr;
+}
+
+// cuTensorMapEncodeTiled, fetched from the driver at run time so that the
+// library loads on machines without a driver.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 map over a [rows, 576] matrix, box {64 columns, box_rows}, 128-byte swizzle.
+bool make_map_576(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)tc::kRow, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)tc::kRow * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct WsLayout {
+  size_t off_plan, off_streams, off_bad, off_partial, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+WsLayout ws_layout(int n_streams, int G) {
+  WsLayout w;
+  w.off_plan = 0;
+  w.off_streams = align256(sizeof(tc::PlanHeader));
+  w.off_bad = w.off_streams + align256(sizeof(int) * (size_t)(n_streams + 1));
+  w.off_partial = w.off_bad + align256(sizeof(int) * (size_t)n_streams);
+  w.total = w.off_partial + sizeof(float) * tc::kSlotFloats * 2 * (size_t)G;
+  return w;
+}
+
+mla_status_t launch_ok() {
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t mla_abi_version(void) { return MLA_ABI_VERSION; }
+
+const char* mla_status_str(mla_status_t s) {
+  switch (s) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+    case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT";
+    case MLA_ERR_BAD_INDEX: return "MLA_ERR_BAD_INDEX";
+  }
+  return "MLA_ERR_UNKNOWN";
+}
+
+mla_status_t mla_get_status(mla_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+  return static_cast<mla_status_t>(v);
+}
+
+mla_status_t mla_absorb_q(const mla_dims_t* dims, int32_t n_q, const void* q_nope,
+                          const void* q_rope, const int32_t* q_pos, const int32_t* delta,
+                          int32_t n_ver, const void* w_uk, void* q_abs, mla_stream_t stream) {
+  if (!dims_ok(dims) || n_q < 0 || n_ver < 1 || n_ver > kMaxVersions || !delta)
+    return MLA_ERR_INVALID_ARG;
+  if (n_q == 0) return MLA_OK;
+  if (!q_nope || !q_rope || !q_pos || !w_uk || !q_abs) return MLA_ERR_INVALID_ARG;
+  AbsorbArgs a;
+  a.n_q = n_q;
+  a.H = dims->H;
+  a.d_c = dims->d_c;
+  a.d_r = dims->d_r;
+  a.d_n = dims->d_n;
+  a.n_ver = n_ver;
+  a.rope_base = dims->rope_base;
+  for (int i = 0; i < kMaxVersions; ++i) a.delta[i] = i < n_ver ? delta[i] : 0;
+  a.q_nope = q_nope;
+  a.q_rope = q_rope;
+  a.q_pos = q_pos;
+  a.w_uk = w_uk;
+  a.q_abs = q_abs;
+  dim3 grid(dims->H, (n_q + kAbsQ - 1) / kAbsQ);
+  const size_t smem = sizeof(float) * kAbsQ * dims->d_n;
+  if (smem > 48 * 1024) return MLA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dims->dtype == MLA_BF16)
+    absorb_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(a);
+  else
+    absorb_kernel<float><<<grid, 256, smem, st>>>(a);
+  return launch_ok();
+}
+
+size_t mla_decode_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t n_h) {
+  if (!dims_ok(dims) || B < 0 || s_q < 1 || n_h < 1) return 0;
+  if (!tc_eligible(dims)) return 256;   // the generic kernel needs no scratch
+  DeviceInfo* d = nullptr;
+  if (device_info(&d) != MLA_OK) return 0;
+  const int n_hb = (n_h + tc::kM - 1) / tc::kM;
+  return ws_layout(B * s_q * n_hb, d->num_sms / 2).total;
+}
+
+mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const void* q_abs,
+                        int32_t n_ver, int32_t h0, int32_t n_h, const void* cache,
+                        int64_t n_pages, const int32_t* block_table, int32_t max_pages,
+                        const mla_seg_t* segs, int32_t max_segs, const int32_t* gather_rows,
+                        const int32_t* n_gather, int32_t max_gather, const int32_t* q_pos,
+                        float* o_lat, float* lse, void* workspace, size_t ws_bytes,
+                        mla_stream_t stream) {
+  if (!dims_ok(dims) || B < 0 || s_q < 1 || n_ver < 1 || h0 < 0 || n_h < 1 ||
+      h0 + n_h > dims->H || n_pages < 1 || max_pages < 1 || max_segs < 1)
+    return MLA_ERR_INVALID_ARG;
+  if (dims->page_size != kPage || n_ver > kMaxVersions) return MLA_ERR_UNSUPPORTED;
+  if (gather_rows && (!n_gather || max_gather < 1)) return MLA_ERR_INVALID_ARG;
+  if (B == 0) return MLA_OK;
+  if (!q_abs || !cache || !block_table || !segs || !q_pos || !o_lat || !lse)
+    return MLA_ERR_INVALID_ARG;
+  if (n_pages * kPage > INT32_MAX) return MLA_ERR_UNSUPPORTED;
+  const size_t es = elem_size(dims);
+  if (!aligned(cache, 256) || !aligned(q_abs, 16) || !aligned(o_lat, 16) || !aligned(lse, 4))
+    return MLA_ERR_INVALID_ARG;
+
+  DecodeArgs a;
+  a.B = B;
+  a.s_q = s_q;
+  a.n_q = B * s_q;
+  a.H = dims->H;
+  a.h0 = h0;
+  a.n_h = n_h;
+  a.d_c = dims->d_c;
+  a.d_r = dims->d_r;
+  a.n_ver = n_ver;
+  a.max_pages = max_pages;
+  a.max_segs = max_segs;
+  a.max_gather = gather_rows ? max_gather : 0;
+  a.n_pages = n_pages;
+  a.scale = dims->scale;
+  a.q_abs = q_abs;
+  a.cache = cache;
+  a.block_table = block_table;
+  a.segs = segs;
+  a.gather_rows = gather_rows;
+  a.n_gather = gather_rows ? n_gather : nullptr;
+  a.q_pos = q_pos;
+  a.o_lat = o_lat;
+  a.lse = lse;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+  if (!tc_eligible(dims)) {
+    const int row = dims->d_c + dims->d_r;
+    const size_t smem = sizeof(float) * ((size_t)n_ver * row + dims->d_c + 128 + 4) +
+                        sizeof(long long) * 128 + 64;
+    if (smem > 48 * 1024) return MLA_ERR_UNSUPPORTED;
+    dim3 grid(n_h, B * s_q);
+    if (dims->dtype == MLA_BF16)
+      decode_simt_kernel<__nv_bfloat16><<<grid, 128, smem, st>>>(a);
+    else
+      decode_simt_kernel<float><<<grid, 128, smem, st>>>(a);
+    (void)es;
+    return launch_ok();
+  }
+
+  DeviceInfo* dev = nullptr;
+  if (device_info(&dev) != MLA_OK) return MLA_ERR_CUDA;
+  const int G = dev->num_sms / 2;
+  const int n_hb = (n_h + tc::kM - 1) / tc::kM;
+  const int n_streams = B * s_q * n_hb;
+  const WsLayout wl = ws_layout(n_streams, G);
+  if (!workspace || ws_bytes < wl.total) return MLA_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return MLA_ERR_INVALID_ARG;
+
+  CUtensorMap tm_q, tm_kv[tc::kNumBoxHeights];
+  if (!make_map_576(&tm_q, q_abs, (uint64_t)n_ver * B * s_q * dims->H, tc::kM))
+    return MLA_ERR_CUDA;
+  for (int i = 0; i < tc::kNumBoxHeights; ++i)
+    if (!make_map_576(&tm_kv[i], cache, (uint64_t)n_pages * kPage, (uint32_t)(tc::kN >> i)))
+      return MLA_ERR_CUDA;
+
+  if (!dev->tc_attr_set) {
+    if (cudaFuncSetAttribute(tc::decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             tc::kSmemBytes) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    dev->tc_attr_set = true;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  tc::PlanHeader* plan = reinterpret_cast<tc::PlanHeader*>(ws + wl.off_plan);
+  int* stream_off = reinterpret_cast<int*>(ws + wl.off_streams);
+  int* stream_bad = reinterpret_cast<int*>(ws + wl.off_bad);
+  float* partial = reinterpret_cast<float*>(ws + wl.off_partial);
+
+  tc::plan_kernel<<<1, 256, 0, st>>>(a, n_hb, G, plan, stream_off, stream_bad);
+  if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+
+  tc::Params p;
+  p.a = a;
+  p.n_hb = n_hb;
+  p.G = G;
+  p.plan = plan;
+  p.stream_off = stream_off;
+  p.partial = partial;
+  p.scale_log2 = dims->scale * tc::kLog2e;
+  tc::decode_tc_kernel<<<2 * G, tc::kThreads, tc::kSmemBytes, st>>>(
+      p, tm_q, tm_kv[0], tm_kv[1], tm_kv[2], tm_kv[3], tm_kv[4], tm_kv[5], tm_kv[6]);
+  if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+
+  tc::combine_kernel<<<n_streams, 256, 0, st>>>(a, n_hb, plan, stream_off, stream_bad, partial);
+  return launch_ok();
+}
+
+mla_status_t mla_merge_lse(int32_t n_q, int32_t H, int32_t h0, int32_t n_h, int32_t d,
+                           const float* o_a, const float* lse_a, const float* o_b,
+                           const float* lse_b, float* o, float* lse, mla_stream_t stream) {
+  if (n_q < 0 || H < 1 || h0 < 0 || n_h < 1 || h0 + n_h > H || d < 1) return MLA_ERR_INVALID_ARG;
+  if (n_q == 0) return MLA_OK;
+  if (!o_a || !lse_a || !o_b || !lse_b || !o || !lse) return MLA_ERR_INVALID_ARG;
+  const long long rows = (long long)n_q * n_h;
+  const long long blocks = (rows + 7) / 8;
+  if (blocks > INT32_MAX) return MLA_ERR_INVALID_ARG;
+  merge_lse_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      n_q, H, h0, n_h, d, o_a, lse_a, o_b, lse_b, o, lse);
+  return launch_ok();
+}
+
+mla_status_t mla_out_proj(const mla_dims_t* dims, int32_t n_q, const float* o_lat,
+                          const void* w_uv, const void* w_o, float* v, float* out,
+                          mla_stream_t stream) {
+  if (!dims_ok(dims) || n_q < 0) return MLA_ERR_INVALID_ARG;
+  if (n_q == 0) return MLA_OK;
+  if (!o_lat || !w_uv || !v || (w_o && (!out || dims->d_model < 1))) return MLA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int H = dims->H, d_c = dims->d_c, d_v = dims->d_v;
+  dim3 g1(H, (d_v + 7) / 8);
+  if (dims->dtype == MLA_BF16)
+    vproj_simt_kernel<__nv_bfloat16><<<g1, 256, 0, st>>>(
+        n_q, H, d_c, d_v, o_lat, static_cast<const __nv_bfloat16*>(w_uv), v);
+  else
+    vproj_simt_kernel<float><<<g1, 256, 0, st>>>(n_q, H, d_c, d_v, o_lat,
+                                                 static_cast<const float*>(w_uv), v);
+  if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  if (!w_o) return MLA_OK;
+  const int K = H * d_v;
+  dim3 g2((dims->d_model + 7) / 8);
+  if (dims->dtype == MLA_BF16)
+    oproj_simt_kernel<__nv_bfloat16><<<g2, 256, 0, st>>>(
+        n_q, K, dims->d_model, v, static_cast<const __nv_bfloat16*>(w_o), out);
+  else
+    oproj_simt_kernel<float><<<g2, 256, 0, st>>>(n_q, K, dims->d_model, v,
+                                                 static_cast<const float*>(w_o), out);
+  return launch_ok();
+}
+
+}  // extern "C"

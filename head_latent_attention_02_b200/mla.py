@@ -1,0 +1,145 @@
+"""Python binding of libmla (include/mla.h): argument marshalling only.
+
+Every step runs in the library's CUDA kernels; this module turns torch
+tensors into pointers and sizes, calls the C ABI and raises on a non-OK
+status.  It fails loudly when libmla.so is missing -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmla.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "mla.h")
+
+MLA_F32, MLA_BF16 = 0, 1
+STATUS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED", 3: "MLA_ERR_WORKSPACE",
+          4: "MLA_ERR_CUDA", 5: "MLA_ERR_TIMEOUT", 6: "MLA_ERR_BAD_INDEX"}
+
+
+class MLAError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {STATUS.get(code, code)}")
+        self.code = code
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("H", ctypes.c_int32), ("d_c", ctypes.c_int32), ("d_r", ctypes.c_int32),
+                ("d_n", ctypes.c_int32), ("d_v", ctypes.c_int32), ("d_model", ctypes.c_int32),
+                ("page_size", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("scale", ctypes.c_float), ("rope_base", ctypes.c_double)]
+
+
+_lib = None
+_vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+_SIGS = {
+    "mla_abi_version": ([], _i32),
+    "mla_status_str": ([_i32], ctypes.c_char_p),
+    "mla_get_status": ([_vp], _i32),
+    "mla_absorb_q": ([ctypes.POINTER(Dims), _i32, _vp, _vp, _vp, ctypes.POINTER(_i32), _i32, _vp,
+                      _vp, _vp], _i32),
+    "mla_decode": ([ctypes.POINTER(Dims), _i32, _i32, _vp, _i32, _i32, _i32, _vp, _i64, _vp, _i32,
+                    _vp, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
+    "mla_decode_workspace_size": ([ctypes.POINTER(Dims), _i32, _i32, _i32], _sz),
+    "mla_merge_lse": ([_i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
+    "mla_out_proj": ([ctypes.POINTER(Dims), _i32, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmla.so (built in-tree); raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libmla.so not built at {LIB_PATH}: run "
+                               "`python -m head_latent_attention_02_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def header_symbols() -> list:
+    """Entry points declared in include/mla.h."""
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\*]+\s+\*?(mla_\w+)\s*\(", txt, re.M)))
+
+
+def make_dims(wl, dtype: Optional[int] = None) -> Dims:
+    return Dims(wl.H, wl.d_c, wl.d_r, wl.d_n, wl.d_v, wl.d_model, 64,
+                (MLA_BF16 if wl.dtype == "bf16" else MLA_F32) if dtype is None else dtype,
+                wl.scale, wl.rope_base)
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def _s(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise MLAError(fn, code)
+
+
+def status_str(code: int) -> str:
+    return lib().mla_status_str(code).decode()
+
+
+def get_status(stream=None) -> int:
+    """Waits for the stream and returns (and clears) the device status word."""
+    return int(lib().mla_get_status(_s(stream)))
+
+
+def absorb_q(dims: Dims, q_nope, q_rope, q_pos, deltas: Sequence[int], w_uk, q_abs, stream=None):
+    n_q = q_nope.shape[0]
+    arr = (_i32 * len(deltas))(*[int(d) for d in deltas])
+    _check("mla_absorb_q", lib().mla_absorb_q(ctypes.byref(dims), n_q, _p(q_nope), _p(q_rope),
+                                              _p(q_pos), arr, len(deltas), _p(w_uk), _p(q_abs),
+                                              _s(stream)))
+
+
+def workspace_size(dims: Dims, B: int, s_q: int, n_h: int) -> int:
+    return int(lib().mla_decode_workspace_size(ctypes.byref(dims), B, s_q, n_h))
+
+
+def decode(dims: Dims, B: int, s_q: int, q_abs, n_ver: int, h0: int, n_h: int, cache,
+           block_table, segs, q_pos, o_lat, lse, workspace, gather_rows=None, n_gather=None,
+           stream=None):
+    n_pages = cache.shape[0]
+    max_pages = block_table.shape[1]
+    max_segs = segs.shape[1]
+    max_gather = gather_rows.shape[1] if gather_rows is not None else 0
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("mla_decode", lib().mla_decode(
+        ctypes.byref(dims), B, s_q, _p(q_abs), n_ver, h0, n_h, _p(cache), n_pages,
+        _p(block_table), max_pages, _p(segs), max_segs, _p(gather_rows), _p(n_gather),
+        max_gather, _p(q_pos), _p(o_lat), _p(lse), _p(workspace), ws_bytes, _s(stream)))
+
+
+def merge_lse(n_q: int, H: int, h0: int, n_h: int, d: int, o_a, lse_a, o_b, lse_b, o, lse,
+              stream=None):
+    _check("mla_merge_lse", lib().mla_merge_lse(n_q, H, h0, n_h, d, _p(o_a), _p(lse_a), _p(o_b),
+                                                _p(lse_b), _p(o), _p(lse), _s(stream)))
+
+
+def out_proj(dims: Dims, o_lat, w_uv, w_o, v, out, stream=None):
+    n_q = o_lat.shape[0]
+    _check("mla_out_proj", lib().mla_out_proj(ctypes.byref(dims), n_q, _p(o_lat), _p(w_uv),
+                                              _p(w_o), _p(v), _p(out), _s(stream)))

@@ -1,0 +1,211 @@
+/*
+ * mla.h -- C ABI of libmla: absorbed Multi-head Latent Attention decode over a
+ * paged latent KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * Sources of the operations:
+ *   [T27] Day 27 tutorial "Multi-Head Latent Attention: How DeepSeek Compressed
+ *         the Cache Further" (kgptalkie), sections named per call below.
+ *   [RK]  "RedKnot-MLA: Multi-Head Offline-Online Reuse for DeepSeek-V4
+ *         Long-Context Serving", abstract.
+ *
+ * Conventions shared by every call
+ *   - Every pointer is a DEVICE pointer owned by the caller unless a comment
+ *     says "host".  The library never allocates device memory and keeps no
+ *     state between calls except cached per-device properties and TMA
+ *     descriptors.  Buffers must not alias unless a call says so.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream) and returns an mla_status_t synchronously.
+ *     Argument errors are reported before anything is launched and leave the
+ *     outputs untouched.  MLA_ERR_CUDA reports a failed launch.
+ *   - Errors found by a kernel while it runs (a page id out of range, a row
+ *     outside every segment) are written to a device status word; the
+ *     offending work item is skipped (its outputs are set to NaN), the kernel
+ *     never traps.  mla_get_status() reads and clears that word.
+ *   - Storage types: dims.dtype == MLA_BF16 means q_nope, q_rope, q_abs, the
+ *     cache, W_UK, W_UV and W_O hold bfloat16; MLA_F32 means they hold float.
+ *     Accumulation is always fp32; o_lat, lse, v and out are always float.
+ *   - Layouts are dense row-major in the index order written in brackets.
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLA_ABI_VERSION 1
+
+/* A cudaStream_t, declared without including the CUDA headers. */
+typedef struct CUstream_st* mla_stream_t;
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned buffer       */
+  MLA_ERR_UNSUPPORTED = 2,  /* valid arguments with no kernel for them          */
+  MLA_ERR_WORKSPACE = 3,    /* workspace smaller than mla_decode_workspace_size */
+  MLA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed             */
+  MLA_ERR_TIMEOUT = 5,      /* a bounded device-side wait gave up               */
+  MLA_ERR_BAD_INDEX = 6     /* a kernel met a page id / row / segment out of range */
+} mla_status_t;
+
+typedef enum { MLA_F32 = 0, MLA_BF16 = 1 } mla_dtype_t;
+
+/* Model dimensions of one attention layer.
+ *   H          query heads
+ *   d_c        width of the shared content latent c_KV ([T27] "Learn a Smaller
+ *              Shared Representation")
+ *   d_r        width of the decoupled rotary key ([T27] "Position Rotations
+ *              Complicate the Absorption"); even
+ *   d_n, d_v   per-head no-position key width and value width
+ *   d_model    output width of the shared output projection W_O
+ *   page_size  cache rows per page; must be 64
+ *   dtype      MLA_F32 or MLA_BF16 (storage type, see above)
+ *   scale      softmax scale applied to every score (1/sqrt(d_n + d_r) is the
+ *              scale of the expanded query/key width)
+ *   rope_base  RoPE base: feature pair i of a vector at position p is rotated
+ *              by p * rope_base^(-2i/d_r); pairs are adjacent (2i, 2i+1). */
+typedef struct {
+  int32_t H, d_c, d_r, d_n, d_v, d_model, page_size;
+  int32_t dtype;
+  float scale;
+  double rope_base;
+} mla_dims_t;
+
+/* One segment of a sequence's logical row space.  Rows [row_begin, row_end)
+ * hold cache rows whose request positions are key_pos_base + (r - row_begin);
+ * their rotary keys were cached at (request position - delta[q_version]),
+ * where delta[] are the relocation offsets given to mla_absorb_q.  A document
+ * cached offline at canonical position 0 and placed at request offset P is
+ * the segment {P, P + len, v, P} with delta[v] = P ([RK]: query-side RoPE
+ * relocation restores the document's request position).  row_begin must be
+ * a multiple of page_size; row_begin == row_end marks an unused slot. */
+typedef struct {
+  int32_t row_begin, row_end, q_version, key_pos_base;
+} mla_seg_t;
+
+/* ABI version of the loaded library (MLA_ABI_VERSION). */
+int32_t mla_abi_version(void);
+
+/* Static string naming a status code. */
+const char* mla_status_str(mla_status_t status);
+
+/* Waits for `stream`, then returns and clears the device status word that
+ * kernels set when they skip bad work items (MLA_OK if none). */
+mla_status_t mla_get_status(mla_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * mla_absorb_q -- projection absorption plus query-side RoPE relocation.
+ * [T27] "Move the Key Projection Into the Query": q . (U_K c) = (U_K^T q) . c,
+ * so the newest query is transformed once per step instead of expanding every
+ * cached latent.  [T27] "Position Rotations Complicate the Absorption": the
+ * rotary part stays a separate term.  [RK]: the rotary query is rotated at
+ * (q_pos - delta[v]) so that keys cached at shifted positions need no rewrite.
+ *
+ *   q_nope [n_q, H, d_n]   no-position query per head            (dtype)
+ *   q_rope [n_q, H, d_r]   rotary query per head, unrotated       (dtype)
+ *   q_pos  [n_q]           request position of each query token   (int32)
+ *   delta  [n_ver]  HOST   relocation offsets; version v rotates the rotary
+ *                          query at q_pos - delta[v]; 1 <= n_ver <= 8
+ *   w_uk   [H, d_n, d_c]   W_UK[h]: c -> content key              (dtype)
+ *   q_abs  [n_ver, n_q, H, d_c + d_r]  out: [W_UK[h]^T q_nope | R(q_pos -
+ *                          delta[v]) q_rope], rounded to dtype
+ * Angles are computed in double precision.  Errors: INVALID_ARG for null
+ * pointers, n_q < 0, n_ver outside [1, 8], odd d_r. */
+mla_status_t mla_absorb_q(const mla_dims_t* dims, int32_t n_q, const void* q_nope,
+                          const void* q_rope, const int32_t* q_pos, const int32_t* delta,
+                          int32_t n_ver, const void* w_uk, void* q_abs,
+                          mla_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * mla_decode -- absorbed attention of every query token over its sequence's
+ * packed latent cache, for the head range [h0, h0 + n_h).
+ * [T27] "Move the Key Projection Into the Query" and "Position Rotations
+ * Complicate the Absorption": score(t) = scale * (q_abs_content . c_t +
+ * q_abs_rope . k_rope_t), masked where key_pos(t) > q_pos, softmaxed.
+ * [T27] "Move the Value Expansion After the Weighted Sum": the output is the
+ * weighted latent o_lat = sum_t a_t c_t; the value expansion happens later
+ * (mla_out_proj).  Long sequences are split across SMs and the splits are
+ * merged by log-sum-exp inside this call.
+ *
+ *   B, s_q        sequences and query tokens per sequence; query row i =
+ *                 b * s_q + j
+ *   q_abs         [n_ver, B*s_q, H, d_c + d_r] from mla_absorb_q (dtype)
+ *   h0, n_h       head range; 0 <= h0, n_h >= 1, h0 + n_h <= H
+ *   cache         [n_pages, page_size, d_c + d_r]: row = [c_KV | k_rope],
+ *                 k_rope already rotated at its cache position (dtype);
+ *                 256-byte aligned
+ *   block_table   [B, max_pages]: page id of each page_size-row block of a
+ *                 sequence's logical row space (int32)
+ *   segs          [B, max_segs] (mla_seg_t): a sequence's segments, sorted,
+ *                 disjoint; its rows are the union of its segments
+ *   gather_rows   NULL, or [B, max_gather] logical rows to attend instead of
+ *                 all segment rows ([RK]: protected token rows recomputed
+ *                 online); n_gather [B] gives how many entries are used.
+ *                 Every gathered row must lie in a segment.
+ *   q_pos         [B*s_q] request positions (int32)
+ *   o_lat         [B*s_q, H, d_c] out (float): heads outside [h0, h0+n_h)
+ *                 are not written
+ *   lse           [B*s_q, H] out (float): natural-log sum of exp of the
+ *                 scaled visible scores; a query that sees no row gets
+ *                 o_lat = 0 and lse = -inf
+ *   workspace     scratch of ws_bytes >= mla_decode_workspace_size(...),
+ *                 256-byte aligned; contents need not be initialised
+ * Rows past the end of a segment in its last page, and pages no table
+ * references, may hold anything (NaN included) without affecting results.
+ * Errors: INVALID_ARG (null/size/alignment), UNSUPPORTED (page_size != 64,
+ * n_ver > 8), WORKSPACE (ws_bytes too small). */
+mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const void* q_abs,
+                        int32_t n_ver, int32_t h0, int32_t n_h, const void* cache,
+                        int64_t n_pages, const int32_t* block_table, int32_t max_pages,
+                        const mla_seg_t* segs, int32_t max_segs, const int32_t* gather_rows,
+                        const int32_t* n_gather, int32_t max_gather, const int32_t* q_pos,
+                        float* o_lat, float* lse, void* workspace, size_t ws_bytes,
+                        mla_stream_t stream);
+
+/* Bytes of workspace mla_decode needs for these sizes on the current device
+ * (0 if the arguments are invalid or the device cannot be queried). */
+size_t mla_decode_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q,
+                                 int32_t n_h);
+
+/* ---------------------------------------------------------------------------
+ * mla_merge_lse -- merge two partial attentions over disjoint key sets.
+ * [RK]: certified Local-head contributions kept offline (MLA-Off) and the
+ * rows recomputed online (MLA-Online) are merged before the single shared
+ * output projection.  For each query row q and head h in [h0, h0 + n_h):
+ *   lse = log(exp(lse_a) + exp(lse_b))
+ *   o   = exp(lse_a - lse) * o_a + exp(lse_b - lse) * o_b
+ * with lse = -inf and o = 0 when both sides are empty.
+ *   o_a, o_b, o     [n_q, H, d]   (float)
+ *   lse_a, lse_b, lse [n_q, H]    (float)
+ * o may equal o_a or o_b and lse may equal lse_a or lse_b (in place); no
+ * other aliasing.  Errors: INVALID_ARG. */
+mla_status_t mla_merge_lse(int32_t n_q, int32_t H, int32_t h0, int32_t n_h, int32_t d,
+                           const float* o_a, const float* lse_a, const float* o_b,
+                           const float* lse_b, float* o, float* lse, mla_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * mla_out_proj -- value up-projection per head, then the shared output
+ * projection.  [T27] "Move the Value Expansion After the Weighted Sum": the
+ * one mixed latent is expanded once, v_h = W_UV[h] o_lat_h, and each head's
+ * value joins the final output projection, out = W_O [v_0; ...; v_{H-1}].
+ *   o_lat [n_q, H, d_c]     (float)
+ *   w_uv  [H, d_v, d_c]     (dtype)
+ *   w_o   [d_model, H*d_v]  (dtype) or NULL to stop after v
+ *   v     [n_q, H, d_v]     out (float)
+ *   out   [n_q, d_model]    out (float); ignored when w_o is NULL
+ * For dtype MLA_BF16 the float operands o_lat and v are rounded to bfloat16
+ * on their way into the tensor-core products (accumulation stays fp32).
+ * Errors: INVALID_ARG. */
+mla_status_t mla_out_proj(const mla_dims_t* dims, int32_t n_q, const float* o_lat,
+                          const void* w_uv, const void* w_o, float* v, float* out,
+                          mla_stream_t stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* MLA_H_ */

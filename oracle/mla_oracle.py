@@ -292,11 +292,12 @@ def decode(inp, heads=None, rows_override=None, form="direct", seqs=None):
     return o_lat, lse
 
 
-def decode_absorbed_fast(inp, heads=None, seqs=None):
+def decode_absorbed_fast(inp, heads=None, seqs=None, rows_override=None):
     """Absorbed form, vectorised over heads (same definition as ``decode``
     with form="absorbed", grouped by relocation version so the rotary query
     is formed once per version rather than once per key row).  Used where the
     per-row form is too slow (long contexts) and as the timed CPU baseline.
+    ``rows_override`` maps a sequence to an explicit row list, as in ``decode``.
     Returns o_lat [n_q, n_h, d_c], lse [n_q, n_h].
     """
     wl = inp.wl
@@ -307,7 +308,9 @@ def decode_absorbed_fast(inp, heads=None, seqs=None):
     seqs = range(wl.B) if seqs is None else seqs
     w_uk = np.asarray(inp.w_uk[heads], np.float64)                    # [n_h, d_n, d_c]
     for b in seqs:
-        if inp.gather_rows is not None:
+        if rows_override is not None and b in rows_override:
+            rows, kpos, ver = sequence_rows(inp.segs[b], rows_override[b])
+        elif inp.gather_rows is not None:
             rows, kpos, ver = sequence_rows(inp.segs[b], inp.gather_rows[b, :int(inp.n_gather[b])])
         else:
             rows, kpos, ver = sequence_rows(inp.segs[b])

@@ -1,0 +1,101 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports
+every entry point include/mla.h declares, and rejects bad arguments before
+touching the device."""
+import ctypes
+
+import pytest
+
+from head_latent_attention_02_b200 import build as B
+from head_latent_attention_02_b200 import mla
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return mla.lib()
+
+
+def test_exports_every_header_symbol(L):
+    names = mla.header_symbols()
+    assert {"mla_absorb_q", "mla_decode", "mla_merge_lse", "mla_out_proj"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(mla._SIGS) >= set(names)
+
+
+def test_version_and_status_strings(L):
+    assert L.mla_abi_version() == 1
+    for code, name in mla.STATUS.items():
+        assert mla.status_str(code) == name
+    assert mla.status_str(99) == "MLA_ERR_UNKNOWN"
+
+
+def _dims(**kw):
+    d = dict(H=128, d_c=512, d_r=64, d_n=128, d_v=128, d_model=7168, page_size=64,
+             dtype=mla.MLA_BF16, scale=1 / 192 ** 0.5, rope_base=10000.0)
+    d.update(kw)
+    return mla.Dims(**d)
+
+
+NULL = None
+FAKE = 0x1000   # never dereferenced: every case below fails validation first
+
+
+def _decode(d, B=1, s_q=1, n_ver=1, h0=0, n_h=None, n_pages=4, max_pages=4, max_segs=1,
+            gather=NULL, n_gather=NULL, max_gather=0, ws_bytes=0):
+    n_h = (d.H if d is not None else 8) if n_h is None else n_h
+    return mla.lib().mla_decode(ctypes.byref(d) if d is not None else None, B, s_q, FAKE, n_ver,
+                                h0, n_h, FAKE, n_pages, FAKE, max_pages, FAKE, max_segs, gather,
+                                n_gather, max_gather, FAKE, FAKE, FAKE, FAKE, ws_bytes, None)
+
+
+@pytest.mark.parametrize("case", [
+    dict(d=None), dict(B=-1), dict(s_q=0), dict(n_ver=0), dict(h0=-1), dict(n_h=0),
+    dict(h0=100, n_h=29), dict(n_pages=0), dict(max_pages=0), dict(max_segs=0),
+    dict(gather=FAKE, n_gather=NULL, max_gather=4), dict(gather=FAKE, n_gather=FAKE, max_gather=0),
+])
+def test_decode_rejects_bad_arguments(L, case):
+    d = case.pop("d", _dims())
+    assert _decode(d, **case) == 1   # MLA_ERR_INVALID_ARG
+
+
+def test_decode_rejects_bad_dims(L):
+    assert _decode(_dims(d_r=63)) == 1
+    assert _decode(_dims(dtype=7)) == 1
+    assert _decode(_dims(H=0), n_h=1) == 1
+    assert _decode(_dims(page_size=32)) == 2          # MLA_ERR_UNSUPPORTED
+    assert _decode(_dims(), n_ver=9) == 2
+
+
+def test_decode_rejects_misaligned_cache(L):
+    d = _dims()
+    rc = mla.lib().mla_decode(ctypes.byref(d), 1, 1, FAKE, 1, 0, 128, FAKE + 16, 4, FAKE, 4,
+                              FAKE, 1, None, None, 0, FAKE, FAKE, FAKE, FAKE, 0, None)
+    assert rc == 1
+
+
+def test_absorb_merge_outproj_reject_bad_arguments(L):
+    d = _dims()
+    f = mla.lib()
+    arr = (ctypes.c_int32 * 1)(0)
+    assert f.mla_absorb_q(ctypes.byref(d), 4, FAKE, FAKE, FAKE, arr, 0, FAKE, FAKE, None) == 1
+    assert f.mla_absorb_q(ctypes.byref(d), 4, FAKE, FAKE, FAKE, arr, 9, FAKE, FAKE, None) == 1
+    assert f.mla_absorb_q(ctypes.byref(d), 4, FAKE, FAKE, FAKE, None, 1, FAKE, FAKE, None) == 1
+    assert f.mla_absorb_q(ctypes.byref(d), -1, FAKE, FAKE, FAKE, arr, 1, FAKE, FAKE, None) == 1
+    assert f.mla_absorb_q(ctypes.byref(d), 4, None, FAKE, FAKE, arr, 1, FAKE, FAKE, None) == 1
+    assert f.mla_absorb_q(ctypes.byref(d), 0, None, None, None, arr, 1, None, None, None) == 0
+    assert f.mla_merge_lse(2, 64, 60, 8, 512, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert f.mla_merge_lse(2, 64, 0, 8, 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert f.mla_merge_lse(2, 64, 0, 8, 512, None, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert f.mla_merge_lse(0, 64, 0, 8, 512, None, None, None, None, None, None, None) == 0
+    assert f.mla_out_proj(ctypes.byref(d), 2, None, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert f.mla_out_proj(ctypes.byref(d), 2, FAKE, FAKE, FAKE, FAKE, None, None) == 1
+    assert f.mla_out_proj(ctypes.byref(d), -1, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+
+
+def test_workspace_size_rejects_bad_arguments(L):
+    d = _dims()
+    assert mla.lib().mla_decode_workspace_size(None, 1, 1, 128) == 0
+    assert mla.lib().mla_decode_workspace_size(ctypes.byref(d), 1, 0, 128) == 0
+    # the generic (non-576-wide) kernel needs only a token workspace
+    assert mla.lib().mla_decode_workspace_size(ctypes.byref(_dims(dtype=mla.MLA_F32)), 1, 1, 8) == 256
