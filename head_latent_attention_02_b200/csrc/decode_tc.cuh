@@ -1,30 +1,32 @@
-// decode_tc.cuh -- absorbed MLA decode on sm_100a tensor cores.
+// decode_tc.cuh -- absorbed MLA decode on sm_100a tensor cores (CTA pairs).
 //
 // What it computes (Day 27 tutorial "Multi-Head Latent Attention", sections
 // "Move the Key Projection Into the Query", "Position Rotations Complicate
-// the Absorption", "Move the Value Expansion After the Weighted Sum"): for a
-// tile of up to 128 query rows (one query token x up to 128 heads) and every
-// cached row t of the sequence,
+// the Absorption", "Move the Value Expansion After the Weighted Sum"): for
+// 128 query rows (one query token x up to 128 heads) and every cached row t,
 //     S[m, t] = scale * (q_abs[m, :512] . c_t + q_abs[m, 512:] . k_rope_t)
 //     P = online-softmax(S masked by key_pos(t) <= q_pos),  O[m, :] = sum_t P[m,t] c_t
-// with the latent row [c_t | k_rope_t] (576 bf16) read once from HBM.
+// reading each 576-element latent row [c_t | k_rope_t] from HBM once.
 //
-// Decomposition.  A 128-row fp32 accumulator over d_c = 512 fills all 512
-// TMEM columns of an SM, so the work of one tile is split across a cluster of
-// two CTAs along d_c: CTA 0 owns latent columns [0, 256) plus the 64 rotary
-// columns, CTA 1 owns latent columns [256, 512).  Each CTA streams only its
-// columns of every 64-row page (TMA, 128-byte swizzle), so every cache byte
-// crosses HBM once.  Each CTA computes a partial score over its columns
-// (tcgen05.mma, M=128 N=64, fp32 in TMEM), the two partials are exchanged
-// through distributed shared memory and added in the same order on both
-// sides, both CTAs run the identical online softmax, and each accumulates its
-// half of O = P . c (tcgen05.mma, M=128 N=256, fp32 in TMEM columns 0-255).
+// Decomposition.  A cluster of two CTAs on two SMs shares one tcgen05 MMA
+// (cta_group::2): CTA r holds the query rows of heads [64r, 64r + 64) and the
+// cache rows of page 2k + r of a 128-row tile; the pair computes the full
+// 128 x 128 score tile, each CTA receiving its 64 head rows in TMEM (tokens
+// 0-63 in lanes 0-63, tokens 64-127 in lanes 64-127 of the same columns).
+// The softmax of a head row is shared by lanes t and t + 64 (the row max is
+// combined through shared memory).  P . c runs as two M=128 x N=256 pair
+// MMAs (latent halves); each CTA supplies the c columns of its N half for all
+// 128 rows, re-read through L2 in 8 KB stages, and accumulates O for its 64
+// heads in 256 TMEM columns (lanes 0-63: latent [0,128) and [256,384);
+// lanes 64-127: [128,256) and [384,512)).  No scores or probabilities cross
+// between the SMs: only the MMA operands do, inside the pair instruction.
 //
-// Roles per CTA (192 threads): warp 0 loads (TMA), warp 1 issues tcgen05.mma,
-// warps 2-5 hold one query row per thread for softmax and the epilogue.
-// Long sequences are split over CTA pairs; each pair gets a contiguous run of
-// (sequence, row tile, page) units and writes either the final output or a
-// normalised partial (o, lse) that the combine kernel merges.
+// Roles per CTA (192 threads): warp 0 streams Q, cache and value stages
+// (TMA), warp 1 of CTA 0 issues every MMA of the pair, warps 2-5 own one
+// TMEM lane each for softmax and the epilogue.  Work is split over CTA pairs
+// as contiguous runs of (sequence, head block, tile) units; a pair writes
+// the final result of a sequence it covers entirely, else a normalised
+// partial (o, lse) that the combine kernel merges.
 #pragma once
 #include <cuda.h>
 
@@ -35,76 +37,81 @@ namespace mla {
 namespace tc {
 
 constexpr int kDc = 512, kDr = 64, kRow = kDc + kDr;
-constexpr int kM = 128;                       // query rows per tile
-constexpr int kN = 64;                        // cache rows per tile (one page)
-constexpr int kPanelKV = kN * 128;            // one 64-column panel of a page: 8 KB
-constexpr int kPanelQ = kM * 128;             // one 64-column panel of Q: 16 KB
-constexpr int kMaxPanels = 5;                 // CTA 0: 4 latent + 1 rotary panel
-constexpr int kStages = 2;
-constexpr int kStageBytes = kMaxPanels * kPanelKV;   // 40 KB
-constexpr int kQBytes = kMaxPanels * kPanelQ;        // 80 KB
-constexpr int kPBytes = kM * 128;                    // 16 KB (128 x 64 bf16)
-constexpr int kXBytes = kM * kN * 4;                 // 32 KB partial scores
+constexpr int kM = 128;                  // query rows of the pair
+constexpr int kMh = 64;                  // query rows per CTA
+constexpr int kT = 128;                  // cache rows per tile (two pages)
+constexpr int kPg = 64;                  // rows per page
+constexpr int kPanel = 8192;             // 64 rows x 128 B, 128-byte swizzle
+constexpr int kQPanels = 9;              // 8 latent + 1 rotary 64-column panels
+constexpr int kStages = 14;              // 8 KB ring stages (K panels and V halves)
 constexpr int kOffQ = 0;
-constexpr int kOffKV = kOffQ + kQBytes;
-constexpr int kOffP = kOffKV + kStages * kStageBytes;
-constexpr int kOffX = kOffP + 2 * kPBytes;
-constexpr int kOffBar = kOffX + kXBytes;
-constexpr int kBarBytes = 256;
+constexpr int kOffRing = kOffQ + kQPanels * kPanel;
+constexpr int kOffP = kOffRing + kStages * kPanel;
+constexpr int kPBuf = 2 * kPanel;        // 64 rows x 128 tokens bf16
+constexpr int kOffMisc = kOffP + 2 * kPBuf;
+constexpr int kMiscBytes = 2048;
+constexpr int kOffBar = kOffMisc + kMiscBytes;
+constexpr int kBarBytes = 512;
 constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;   // + alignment slack
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
 constexpr int kColO = 0, kColS = 256;
-constexpr int kMinChunk = 4;
-constexpr int kNumBoxHeights = 7;             // 64, 32, 16, 8, 4, 2, 1 rows
+constexpr int kMinChunk = 2;
+constexpr int kNumBoxHeights = 7;        // 64, 32, 16, 8, 4, 2, 1 rows
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRescaleThreshold = 8.0f;     // log2 units: lazy rescale margin
-
-// Partial slot: 128 rows x 512 fp32 + 128 lse.
-constexpr size_t kSlotFloats = (size_t)kM * kDc + kM;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: lazy rescale margin
+constexpr size_t kSlotFloats = (size_t)kM * kDc + kM;   // partial: o rows + lse
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct PlanHeader {
-  int U;          // total (sequence, row tile, page) units
-  int C;          // units per worker
-  int G;          // workers (CTA pairs)
-  int n_streams;  // (sequence, row tile) streams
+  int U, C, G, n_streams;
 };
 
 struct Params {
   DecodeArgs a;
-  int n_hb;                 // head blocks of <= 128 heads
+  int n_hb;
   int G;
   const PlanHeader* plan;
-  const int* stream_off;    // [n_streams + 1]
-  float* partial;           // [2G][kSlotFloats]
+  const int* stream_off;
+  float* partial;
   float scale_log2;
 };
 
 // ----------------------------------------------------------------- tiles
 struct Tile {
-  int n_valid;        // rows of the tile that exist (0..64)
-  int ver;            // query version of the tile (gather: of its first row)
-  long long phys0;    // physical row of row 0 (page mode)
-  int kpos0;          // request position of row 0 (page mode)
+  int ver;
   bool gather;
+  int g0;              // gather: index of the tile's first gathered row
+  int n_rows;          // gather: gathered rows in the tile (1..128)
+  long long phys[2];   // page mode: physical row of each page's row 0
+  int nv[2];           // page mode: valid rows of each page (0 = absent)
+  int kpos[2];         // page mode: request position of each page's row 0
 };
 
-// Describe tile k of sequence b.  Page mode: the k-th page of the
-// concatenated segments (segments start on page boundaries, so a page holds
-// rows of one segment).  Gather mode: gathered rows [64k, 64k + 64).
-// Deterministic: every role computes the same description.
+// Number of 128-row tiles of a segment of len rows (pages are paired inside
+// a segment, so a tile never mixes relocation versions).
+__device__ __forceinline__ int seg_tiles(int len) {
+  const int np = (len + kPg - 1) / kPg;
+  return (np + 1) / 2;
+}
+
 __device__ __forceinline__ Tile describe(const DecodeArgs& a, int b, int k) {
   Tile t;
   t.gather = a.gather_rows != nullptr;
-  t.n_valid = 0;
   t.ver = 0;
-  t.phys0 = 0;
-  t.kpos0 = 0;
+  t.g0 = 0;
+  t.n_rows = 0;
+  for (int i = 0; i < 2; ++i) {
+    t.phys[i] = 0;
+    t.nv[i] = 0;
+    t.kpos[i] = 0;
+  }
   const mla_seg_t* sg = a.segs + (size_t)b * a.max_segs;
   if (t.gather) {
     const int ng = a.n_gather[b];
-    t.n_valid = min(kN, ng - k * kN);
-    const int r0 = a.gather_rows[(size_t)b * a.max_gather + k * kN];
+    t.g0 = k * kT;
+    t.n_rows = min(kT, ng - t.g0);
+    const int r0 = a.gather_rows[(size_t)b * a.max_gather + t.g0];
     for (int s = 0; s < a.max_segs; ++s)
       if (r0 >= sg[s].row_begin && r0 < sg[s].row_end) { t.ver = sg[s].q_version; break; }
     return t;
@@ -113,26 +120,35 @@ __device__ __forceinline__ Tile describe(const DecodeArgs& a, int b, int k) {
   for (int s = 0; s < a.max_segs; ++s) {
     const int len = sg[s].row_end - sg[s].row_begin;
     if (len <= 0) continue;
-    const int np = (len + kN - 1) / kN;
-    if (rem < np) {
-      const int row0 = sg[s].row_begin + rem * kN;
-      const int page = a.block_table[(size_t)b * a.max_pages + row0 / kN];
+    const int nt = seg_tiles(len);
+    if (rem < nt) {
       t.ver = sg[s].q_version;
-      t.kpos0 = sg[s].key_pos_base + (row0 - sg[s].row_begin);
-      if (page >= 0 && page < a.n_pages) {
-        t.n_valid = min(kN, sg[s].row_end - row0);
-        t.phys0 = (long long)page * kN;
-      } else {
-        set_status(MLA_ERR_BAD_INDEX);   // the page's rows are left out, never read
+      const int np = (len + kPg - 1) / kPg;
+      for (int i = 0; i < 2; ++i) {
+        const int pi = 2 * rem + i;
+        if (pi >= np) break;
+        const int row0 = sg[s].row_begin + pi * kPg;
+        const int page = a.block_table[(size_t)b * a.max_pages + row0 / kPg];
+        t.kpos[i] = sg[s].key_pos_base + (row0 - sg[s].row_begin);
+        if (page >= 0 && page < a.n_pages) {
+          t.nv[i] = min(kPg, sg[s].row_end - row0);
+          t.phys[i] = (long long)page * kPg;
+        } else {
+          set_status(MLA_ERR_BAD_INDEX);   // the page's rows are left out, never read
+        }
       }
       return t;
     }
-    rem -= np;
+    rem -= nt;
   }
   return t;
 }
 
-// Walk of one worker's units in (stream, page) order.
+// rows of tile half i (tile rows [64 i, 64 i + 64)) that hold data
+__device__ __forceinline__ int half_rows(const Tile& t, int i) {
+  return t.gather ? max(0, min(kPg, t.n_rows - kPg * i)) : t.nv[i];
+}
+
 struct Walk {
   int s, k, u, u1;
 };
@@ -147,7 +163,7 @@ __device__ __forceinline__ bool walk_begin(const Params& p, int g, Walk& w) {
   if (u0 >= U) return false;
   w.u = (int)u0;
   w.u1 = (int)min((long long)U, u0 + C);
-  int lo = 0, hi = p.plan->n_streams - 1;   // last stream with off <= u0
+  int lo = 0, hi = p.plan->n_streams - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (p.stream_off[mid] <= w.u) lo = mid; else hi = mid - 1;
@@ -182,13 +198,13 @@ __device__ __forceinline__ StreamPos stream_pos(const Params& p, int s) {
 
 // ----------------------------------------------------------------- barriers
 struct Bars {
-  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t full[kStages], empty[kStages];
   uint64_t q_full, q_empty;
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full[2], p_empty[2];
   uint64_t o_done, o_free;
-  uint64_t x_full, x_empty;
   uint64_t mma_drain;
+  uint64_t row_sync[2], l_sync;     // the 128 softmax threads of one CTA
   uint32_t tmem_base;
 };
 static_assert(sizeof(Bars) <= kBarBytes, "barrier block too large");
@@ -196,6 +212,41 @@ static_assert(sizeof(Bars) <= kBarBytes, "barrier block too large");
 __device__ __forceinline__ void fail(bool& ok) {
   if (ok) set_status(MLA_ERR_TIMEOUT);
   ok = false;
+}
+
+// Bounded waits whose outcome is the same for every lane of the warp, so a
+// timeout makes the whole warp leave together.
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+}
+__device__ __forceinline__ bool wait_warp_cluster(uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_wait_cluster(bar, parity));
+}
+
+// Arrive on a barrier of the pair's rank-0 CTA (local or remote).
+__device__ __forceinline__ void arrive_leader(uint64_t* bar, uint32_t rank) {
+  if (rank == 0) mbar_arrive(bar);
+  else mbar_arrive_cluster_addr(mapa(smem_u32(bar), 0));
+}
+
+// Load `rows` rows (starting at physical cache row y) of one 64-column panel
+// into smem with row pitch 128 B, as power-of-two boxes (heights 64..1).
+__device__ __forceinline__ void load_rows(uint8_t* dst, const CUtensorMap* const* maps,
+                                          uint32_t bar, int x, long long y, int rows) {
+  int r = 0;
+#pragma unroll 1
+  for (int hb = 0; hb < kNumBoxHeights; ++hb) {
+    const int h = 64 >> hb;
+    if (rows & h) {
+      tma_load_2d_pair(dst + r * 128, maps[hb], bar, x, (int)(y + r));
+      r += h;
+    }
+  }
+}
+
+__device__ __forceinline__ void zero_rows(uint8_t* dst, int r0, int r1, int lane) {
+  for (int e = lane; e < (r1 - r0) * 8; e += 32)
+    *reinterpret_cast<uint4*>(dst + (r0 + e / 8) * 128 + (e % 8) * 16) = make_uint4(0, 0, 0, 0);
 }
 
 // ----------------------------------------------------------------- kernel
@@ -213,47 +264,47 @@ decode_tc_kernel(const __grid_constant__ Params p,
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + kOffQ;
-  uint8_t* sKV = smem + kOffKV;
+  uint8_t* sRing = smem + kOffRing;
   uint8_t* sP = smem + kOffP;
-  float* sX = reinterpret_cast<float*>(smem + kOffX);
+  float* sMax = reinterpret_cast<float*>(smem + kOffMisc);         // [2][128]
+  float* sL = sMax + 2 * kM;                                       // [128]
   Bars* bar = reinterpret_cast<Bars*>(smem + kOffBar);
 
   const DecodeArgs& a = p.a;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
-  const uint32_t peer = rank ^ 1u;
   const int g = blockIdx.x >> 1;
-  const int panels = (rank == 0) ? 5 : 4;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&bar->kv_full[i], 1);
-      mbar_init(&bar->kv_empty[i], 1);
+      mbar_init(&bar->full[i], 2);   // rank 0 arms both CTAs' bytes; rank 1 arrives after
+      mbar_init(&bar->empty[i], 1);  // its zero-fill and loads are issued
     }
-    mbar_init(&bar->q_full, 1);
+    mbar_init(&bar->q_full, 2);
     mbar_init(&bar->q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar->s_full[i], 1);
-      mbar_init(&bar->s_empty[i], 4);
-      mbar_init(&bar->p_full[i], 4);
+      mbar_init(&bar->s_empty[i], 8);
+      mbar_init(&bar->p_full[i], 8);
       mbar_init(&bar->p_empty[i], 1);
     }
     mbar_init(&bar->o_done, 1);
-    mbar_init(&bar->o_free, 4);
-    mbar_init(&bar->x_full, kM);
-    mbar_init(&bar->x_empty, kM);
+    mbar_init(&bar->o_free, 8);
     mbar_init(&bar->mma_drain, 1);
+    mbar_init(&bar->row_sync[0], kM);
+    mbar_init(&bar->row_sync[1], kM);
+    mbar_init(&bar->l_sync, kM);
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(&bar->tmem_base, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(&bar->tmem_base, kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();     // both CTAs' barriers and TMEM exist before any cross-CTA use
   tc_fence_after();
-  cluster_sync();   // peer barriers initialised before any remote arrive
   const uint32_t tmem = bar->tmem_base;
 
   Walk w;
@@ -261,124 +312,190 @@ decode_tc_kernel(const __grid_constant__ Params p,
   bool ok = true;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ loads
     if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_kv0);
+      prefetch_tmap(&tm_kv1);
     }
-    const CUtensorMap* kvmaps[kNumBoxHeights] = {&tm_kv0, &tm_kv1, &tm_kv2, &tm_kv3,
-                                                 &tm_kv4, &tm_kv5, &tm_kv6};
-    int it = 0, n_qload = 0, cur_s = -1, cur_v = -1;
+    const CUtensorMap* maps[kNumBoxHeights] = {&tm_kv0, &tm_kv1, &tm_kv2, &tm_kv3,
+                                               &tm_kv4, &tm_kv5, &tm_kv6};
+    int n_stage = 0, n_qload = 0, cur_s = -1, cur_v = -1;
+    // wait for the next ring stage to be free
+    auto stage_begin = [&](uint8_t*& dst, uint32_t& fb) -> bool {
+      const int slot = n_stage % kStages;
+      if (!wait_warp(&bar->empty[slot], ((n_stage / kStages) & 1) ^ 1)) return false;
+      dst = sRing + slot * kPanel;
+      fb = mapa(smem_u32(&bar->full[slot]), 0);
+      return true;
+    };
+    // the P.c operand of tile t: for N block nb and 32-row chunk kc, this
+    // CTA's latent columns [256 nb + 128 rank, +128) of tile rows [32 kc, +32)
+    auto load_v = [&](const Tile& t, int b) -> bool {
+      for (int nb = 0; nb < 2; ++nb) {
+        for (int kc = 0; kc < 4; ++kc) {
+          uint8_t* dst;
+          uint32_t fb;
+          if (!stage_begin(dst, fb)) return false;
+          const int hi = kc >> 1, r0 = 32 * (kc & 1);
+          const int rows = max(0, min(32, half_rows(t, hi) - r0));
+          if (rows < 32) {
+            zero_rows(dst, rows, 32, lane);
+            zero_rows(dst + 4096, rows, 32, lane);
+            fence_proxy_async();
+          }
+          __syncwarp();
+          if (rank == 0 && lane == 0)
+            mbar_arrive_expect_tx(&bar->full[n_stage % kStages], 2 * rows * 256);
+          __syncwarp();
+          const int x0 = 256 * nb + 128 * (int)rank;
+          if (!t.gather) {
+            if (lane == 0) {
+              load_rows(dst, maps, fb, x0, t.phys[hi] + r0, rows);
+              load_rows(dst + 4096, maps, fb, x0 + 64, t.phys[hi] + r0, rows);
+            }
+          } else {
+            for (int i = lane; i < rows; i += 32) {
+              long long phys;
+              int kp, vv;
+              if (!locate_row(a, b, t.g0 + 32 * kc + i, &phys, &kp, &vv)) phys = -1;
+              if (phys >= 0) {
+                tma_load_2d_pair(dst + i * 128, maps[kNumBoxHeights - 1], fb, x0, (int)phys);
+                tma_load_2d_pair(dst + 4096 + i * 128, maps[kNumBoxHeights - 1], fb, x0 + 64,
+                                 (int)phys);
+              } else {
+                for (int c = 0; c < 8; ++c) {
+                  *reinterpret_cast<uint4*>(dst + i * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+                  *reinterpret_cast<uint4*>(dst + 4096 + i * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async();
+                asm volatile("mbarrier.complete_tx.shared::cluster.b64 [%0], %1;"
+                             ::"r"(fb), "r"(256) : "memory");
+              }
+            }
+          }
+          __syncwarp();
+          if (rank == 1 && lane == 0) mbar_arrive_cluster_addr(fb);
+          ++n_stage;
+        }
+      }
+      return true;
+    };
+    Tile prev;
+    int prev_b = 0;
+    bool have_prev = false;
     for (bool more = has_work; more && ok; more = (w.u < w.u1)) {
       const StreamPos sp = stream_pos(p, w.s);
       const Tile t = describe(a, sp.b, w.k);
       if (w.s != cur_s || t.ver != cur_v) {
-        if (n_qload > 0 && !mbar_wait(&bar->q_empty, (n_qload - 1) & 1)) { fail(ok); break; }
+        if (n_qload > 0 && !wait_warp(&bar->q_empty, (n_qload - 1) & 1)) { fail(ok); break; }
         if (lane == 0) {
           const int qi = sp.b * a.s_q + sp.j;
-          const int y = (t.ver * a.n_q + qi) * a.H + a.h0 + sp.hb * kM;
-          mbar_arrive_expect_tx(&bar->q_full, panels * kPanelQ);
-          for (int pn = 0; pn < panels; ++pn) {
-            const int x = (pn == 4) ? kDc : (int)rank * 256 + pn * 64;
-            tma_load_2d(sQ + pn * kPanelQ, &tm_q, &bar->q_full, x, y);
-          }
+          const int y = (t.ver * a.n_q + qi) * a.H + a.h0 + sp.hb * kM + kMh * (int)rank;
+          const uint32_t qb = mapa(smem_u32(&bar->q_full), 0);
+          if (rank == 0) mbar_arrive_expect_tx(&bar->q_full, 2 * kQPanels * kPanel);
+          for (int pn = 0; pn < kQPanels; ++pn)
+            tma_load_2d_pair(sQ + pn * kPanel, &tm_q, qb, 64 * pn, y);
+          if (rank == 1) mbar_arrive_cluster_addr(qb);
         }
         ++n_qload;
         cur_s = w.s;
         cur_v = t.ver;
       }
-      const int st = it % kStages;
-      if (!mbar_wait(&bar->kv_empty[st], ((it / kStages) & 1) ^ 1)) { fail(ok); break; }
-      uint8_t* stage = sKV + st * kStageBytes;
-      if (t.n_valid < kN) {
-        // rows without data must read as zero in the P.c product
-        const int zrows = kN - t.n_valid;
-        for (int e = lane; e < panels * zrows * 8; e += 32) {
-          const int pn = e / (zrows * 8);
-          const int rr = t.n_valid + (e / 8) % zrows;
-          const int ch = e % 8;
-          *reinterpret_cast<uint4*>(stage + pn * kPanelKV + rr * 128 + ch * 16) =
-              make_uint4(0, 0, 0, 0);
+      // score operand: this CTA's tile half (rows [64 rank, +64)), 9 panels
+      const int rows = half_rows(t, rank);
+      const int both = half_rows(t, 0) + half_rows(t, 1);
+      for (int pn = 0; pn < kQPanels && ok; ++pn) {
+        uint8_t* dst;
+        uint32_t fb;
+        if (!stage_begin(dst, fb)) { fail(ok); break; }
+        if (rows < kPg) {
+          zero_rows(dst, rows, kPg, lane);
+          fence_proxy_async();
         }
-        fence_proxy_async();
         __syncwarp();
-      }
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&bar->kv_full[st], t.n_valid * panels * 128);
+        if (rank == 0 && lane == 0) mbar_arrive_expect_tx(&bar->full[n_stage % kStages], both * 128);
+        __syncwarp();
         if (!t.gather) {
-          int row = 0;
-          for (int hb = 0; hb < kNumBoxHeights; ++hb) {
-            const int h = kN >> hb;
-            if (t.n_valid & h) {
-              for (int pn = 0; pn < panels; ++pn) {
-                const int x = (pn == 4) ? kDc : (int)rank * 256 + pn * 64;
-                tma_load_2d(stage + pn * kPanelKV + row * 128, kvmaps[hb], &bar->kv_full[st],
-                            x, (int)(t.phys0 + row));
-              }
-              row += h;
-            }
-          }
-        }
-      }
-      if (t.gather) {
-        // one row per box; lanes split the rows, lane 0 already armed the barrier
-        __syncwarp();
-        for (int i = lane; i < t.n_valid; i += 32) {
-          long long phys;
-          int kpos, ver;
-          if (!locate_row(a, sp.b, w.k * kN + i, &phys, &kpos, &ver)) phys = -1;
-          for (int pn = 0; pn < panels; ++pn) {
-            const int x = (pn == 4) ? kDc : (int)rank * 256 + pn * 64;
+          if (lane == 0) load_rows(dst, maps, fb, 64 * pn, t.phys[rank], rows);
+        } else {
+          for (int i = lane; i < rows; i += 32) {
+            long long phys;
+            int kp, vv;
+            if (!locate_row(a, sp.b, t.g0 + kPg * (int)rank + i, &phys, &kp, &vv)) phys = -1;
             if (phys >= 0) {
-              tma_load_2d(stage + pn * kPanelKV + i * 128, kvmaps[kNumBoxHeights - 1],
-                          &bar->kv_full[st], x, (int)phys);
+              tma_load_2d_pair(dst + i * 128, maps[kNumBoxHeights - 1], fb, 64 * pn, (int)phys);
             } else {
-              // unlocatable row: zero it and account its bytes as arrived
-              for (int ch = 0; ch < 8; ++ch)
-                *reinterpret_cast<uint4*>(stage + pn * kPanelKV + i * 128 + ch * 16) =
-                    make_uint4(0, 0, 0, 0);
+              for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(dst + i * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+              fence_proxy_async();
+              asm volatile("mbarrier.complete_tx.shared::cluster.b64 [%0], %1;"
+                           ::"r"(fb), "r"(128) : "memory");
             }
           }
-          if (phys < 0) {
-            fence_proxy_async();
-            asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;"
-                         ::"r"(smem_u32(&bar->kv_full[st])), "r"(panels * 128) : "memory");
-          }
         }
+        __syncwarp();
+        if (rank == 1 && lane == 0) mbar_arrive_cluster_addr(fb);
+        ++n_stage;
       }
-      ++it;
+      if (!ok) break;
+      if (have_prev && !load_v(prev, prev_b)) { fail(ok); break; }
+      prev = t;
+      prev_b = sp.b;
+      have_prev = true;
       walk_next(p, w);
     }
-    // drain: every load issued by this warp has landed before the CTA exits
-    for (int d = 1; d <= kStages && d <= it; ++d) {
-      const int n = it - d;
-      if (!mbar_wait(&bar->kv_full[n % kStages], (n / kStages) & 1)) { fail(ok); break; }
+    if (ok && have_prev && !load_v(prev, prev_b)) fail(ok);
+    // drain: every load this warp issued has landed before the CTA exits
+    // (rank 0 observes the shared barriers; both ranks wait for their ring)
+    if (rank == 0) {
+      for (int d = 1; d <= kStages && d <= n_stage; ++d) {
+        const int n = n_stage - d;
+        if (!wait_warp(&bar->full[n % kStages], (n / kStages) & 1)) { fail(ok); break; }
+      }
     }
-    if (n_qload > 0 && !mbar_wait(&bar->q_full, (n_qload - 1) & 1)) fail(ok);
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(kM, kN, false, false);
+    // ------------------------------------------------------------ MMA (rank 0)
+    if (rank == 0 && lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kM, kT, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kM, 256, false, true);
-      int it = 0, n_q = 0, cur_s = -1, cur_v = -1, n_streams = 0;
+      int it = 0, n_stage = 0, n_q = 0, cur_s = -1, cur_v = -1, n_streams = 0;
       int prev_first = 0, prev_stream_idx = 0;
+      auto stage_wait = [&]() -> uint32_t {
+        const int slot = n_stage % kStages;
+        if (!mbar_wait_cluster(&bar->full[slot], (n_stage / kStages) & 1)) return 0;
+        tc_fence_after();
+        return smem_u32(sRing + slot * kPanel);
+      };
+      auto stage_release = [&]() {
+        mma_pair_commit_both(&bar->empty[n_stage % kStages]);
+        ++n_stage;
+      };
       auto issue_pv = [&](int t, int first, int stream_idx) -> bool {
         const int pb = t & 1;
-        if (!mbar_wait(&bar->p_full[pb], (t >> 1) & 1)) return false;
-        if (first && stream_idx > 0 && !mbar_wait(&bar->o_free, (stream_idx - 1) & 1))
+        if (!mbar_wait_cluster(&bar->p_full[pb], (t >> 1) & 1)) return false;
+        if (first && stream_idx > 0 && !mbar_wait_cluster(&bar->o_free, (stream_idx - 1) & 1))
           return false;
         tc_fence_after();
-        const uint32_t pa = smem_u32(sP + pb * kPBytes);
-        const uint32_t vb = smem_u32(sKV + (t % kStages) * kStageBytes);
+        const uint32_t pa = smem_u32(sP + pb * kPBuf);
+        for (int nb = 0; nb < 2; ++nb) {
+          for (int kc = 0; kc < 4; ++kc) {
+            const uint32_t vb = stage_wait();
+            if (!vb) return false;
 #pragma unroll
-        for (int ks = 0; ks < kN / 16; ++ks) {
-          const uint64_t ad = smem_desc_sw128(pa + ks * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(vb + ks * 16 * 128, kPanelKV, 1024);
-          mma_bf16_ss(tmem + kColO, ad, bd, idesc_pv, (first && ks == 0) ? 0u : 1u);
+            for (int j = 0; j < 2; ++j) {
+              const int ks = 2 * kc + j;
+              const uint64_t ad =
+                  smem_desc_sw128(pa + (ks >> 2) * kPanel + (ks & 3) * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(vb + j * 2048, 4096, 1024);
+              mma_pair_bf16_ss(tmem + kColO + nb * 128, ad, bd, idesc_pv,
+                               (first && ks == 0) ? 0u : 1u);
+            }
+            stage_release();
+          }
         }
-        mma_commit(&bar->kv_empty[t % kStages]);
-        mma_commit(&bar->p_empty[pb]);
-        mma_commit(&bar->o_done);
+        mma_pair_commit_both(&bar->p_empty[pb]);
+        mma_pair_commit_both(&bar->o_done);
         return true;
       };
       for (bool more = has_work; more && ok; more = (w.u < w.u1)) {
@@ -387,33 +504,33 @@ decode_tc_kernel(const __grid_constant__ Params p,
         const bool first = (w.s != cur_s);
         if (first) ++n_streams;
         if (first || t.ver != cur_v) {
-          if (!mbar_wait(&bar->q_full, n_q & 1)) { fail(ok); break; }
+          if (!mbar_wait_cluster(&bar->q_full, n_q & 1)) { fail(ok); break; }
           ++n_q;
           cur_s = w.s;
           cur_v = t.ver;
         }
-        const int st = it % kStages;
-        if (!mbar_wait(&bar->kv_full[st], (it / kStages) & 1)) { fail(ok); break; }
         const int sb = it & 1;
-        if (!mbar_wait(&bar->s_empty[sb], ((it >> 1) & 1) ^ 1)) { fail(ok); break; }
+        if (!mbar_wait_cluster(&bar->s_empty[sb], ((it >> 1) & 1) ^ 1)) { fail(ok); break; }
         tc_fence_after();
         const uint32_t qa = smem_u32(sQ);
-        const uint32_t kb = smem_u32(sKV + st * kStageBytes);
-        for (int pn = 0; pn < panels; ++pn) {
+        for (int pn = 0; pn < kQPanels; ++pn) {
+          const uint32_t kb = stage_wait();
+          if (!kb) { fail(ok); break; }
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t ad = smem_desc_sw128(qa + pn * kPanelQ + ks * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(kb + pn * kPanelKV + ks * 32, 16, 1024);
-            mma_bf16_ss(tmem + kColS + sb * kN, ad, bd, idesc_qk, (pn | ks) ? 1u : 0u);
+            const uint64_t ad = smem_desc_sw128(qa + pn * kPanel + ks * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(kb + ks * 32, 16, 1024);
+            mma_pair_bf16_ss(tmem + kColS + sb * 64, ad, bd, idesc_qk, (pn | ks) ? 1u : 0u);
           }
+          stage_release();
         }
-        mma_commit(&bar->s_full[sb]);
-        // does the next unit of this worker need another Q?
+        if (!ok) break;
+        mma_pair_commit_both(&bar->s_full[sb]);
         Walk nx = w;
         walk_next(p, nx);
         if (nx.u < nx.u1) {
           const Tile tn = describe(a, stream_pos(p, nx.s).b, nx.k);
-          if (nx.s != w.s || tn.ver != t.ver) mma_commit(&bar->q_empty);
+          if (nx.s != w.s || tn.ver != t.ver) mma_pair_commit_both(&bar->q_empty);
         }
         if (it > 0 && !issue_pv(it - 1, prev_first, prev_stream_idx)) { fail(ok); break; }
         prev_first = first;
@@ -422,98 +539,87 @@ decode_tc_kernel(const __grid_constant__ Params p,
         w = nx;
       }
       if (ok && it > 0 && !issue_pv(it - 1, prev_first, prev_stream_idx)) fail(ok);
-      // every tcgen05 op issued here completes before TMEM is released
-      mma_commit(&bar->mma_drain);
+      mma_pair_commit_own(&bar->mma_drain);
       if (!mbar_wait(&bar->mma_drain, 0)) fail(ok);
     }
   } else {
     // ------------------------------------------------------------ softmax
     const int quad = warp & 3;
-    const int m = quad * 32 + lane;
+    const int t = quad * 32 + lane;           // TMEM lane
+    const int half = t >> 6;                  // tile rows [64 half, +64)
+    const int hl = t & 63;                    // head row of this CTA
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-    const uint32_t x_own = smem_u32(sX);
-    const uint32_t x_peer = mapa(x_own, peer);
-    const uint32_t xfull_peer = mapa(smem_u32(&bar->x_full), peer);
-    const uint32_t xempty_peer = mapa(smem_u32(&bar->x_empty), peer);
-    int it = 0, n_streams_done = 0;
+    int it = 0, n_epi = 0, n_od = 0;
+    auto wait_o_done = [&](int target) -> bool {
+      for (; n_od <= target; ++n_od)
+        if (!wait_warp(&bar->o_done, n_od & 1)) return false;
+      return true;
+    };
     while (has_work && ok && w.u < w.u1) {
       const int s = w.s;
       const StreamPos sp = stream_pos(p, s);
       const int qi = sp.b * a.s_q + sp.j;
       const int qp = a.q_pos[qi];
-      const int hrow = sp.hb * kM + m;          // head index within [h0, h0 + n_h)
+      const int hrow = sp.hb * kM + kMh * (int)rank + hl;   // head within [h0, h0 + n_h)
       const bool row_valid = hrow < a.n_h;
       const int T = stream_tiles(p, s);
       float m_run = -INFINITY, l_run = 0.f;
       bool have_o = false;
       while (ok && w.u < w.u1 && w.s == s) {
-        const Tile t = describe(a, sp.b, w.k);
+        const Tile tl = describe(a, sp.b, w.k);
         const int sb = it & 1;
-        if (!mbar_wait(&bar->s_full[sb], (it >> 1) & 1)) { fail(ok); break; }
+        if (!wait_warp(&bar->s_full[sb], (it >> 1) & 1)) { fail(ok); break; }
         tc_fence_after();
         float sv[64];
         {
           float tmp[32];
-          tmem_ld32(trow + kColS + sb * kN, tmp);
+          tmem_ld32(trow + kColS + sb * 64, tmp);
 #pragma unroll
           for (int i = 0; i < 32; ++i) sv[i] = tmp[i];
-          tmem_ld32(trow + kColS + sb * kN + 32, tmp);
+          tmem_ld32(trow + kColS + sb * 64 + 32, tmp);
 #pragma unroll
           for (int i = 0; i < 32; ++i) sv[32 + i] = tmp[i];
           tmem_wait_ld();
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar->s_empty[sb]);
+        if (lane == 0) arrive_leader(&bar->s_empty[sb], rank);
 
-        // exchange partial scores with the peer CTA
-        if (!mbar_wait_cluster(&bar->x_empty, (it & 1) ^ 1)) { fail(ok); break; }
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const uint32_t off = m * 256 + ((c ^ (m & 15)) << 4);
-          st_cluster_v4(x_peer + off, sv[4 * c], sv[4 * c + 1], sv[4 * c + 2], sv[4 * c + 3]);
-        }
-        mbar_arrive_remote(xfull_peer);
-        if (!mbar_wait_cluster(&bar->x_full, it & 1)) { fail(ok); break; }
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float4 o = *reinterpret_cast<const float4*>(
-              reinterpret_cast<const uint8_t*>(sX) + m * 256 + ((c ^ (m & 15)) << 4));
-          // both CTAs add (own + peer) in an order-independent way: a + b == b + a
-          sv[4 * c] += o.x;
-          sv[4 * c + 1] += o.y;
-          sv[4 * c + 2] += o.z;
-          sv[4 * c + 3] += o.w;
-        }
-        mbar_arrive_remote(xempty_peer);
-
-        // mask, scale (log2 domain), online softmax with lazy rescaling
-        float mt = -INFINITY;
-        if (t.gather) {
-          const int i0 = w.k * kN + lane, i1 = i0 + 32;
+        // mask, scale (log2 domain)
+        float mh = -INFINITY;
+        const int nvh = half_rows(tl, half);
+        if (tl.gather) {
+          const int i0 = tl.g0 + kPg * half + lane;
           int kp0 = INT32_MAX, kp1 = INT32_MAX;
           long long ph;
           int vv;
-          if (lane < t.n_valid && !locate_row(a, sp.b, i0, &ph, &kp0, &vv)) kp0 = INT32_MAX;
-          if (lane + 32 < t.n_valid && !locate_row(a, sp.b, i1, &ph, &kp1, &vv)) kp1 = INT32_MAX;
+          if (lane < nvh && !locate_row(a, sp.b, i0, &ph, &kp0, &vv)) kp0 = INT32_MAX;
+          if (lane + 32 < nvh && !locate_row(a, sp.b, i0 + 32, &ph, &kp1, &vv)) kp1 = INT32_MAX;
 #pragma unroll
           for (int i = 0; i < 64; ++i) {
             const int kp = __shfl_sync(0xffffffffu, (i < 32) ? kp0 : kp1, i & 31);
-            const bool vis = (i < t.n_valid) && (kp <= qp);
+            const bool vis = (i < nvh) && (kp <= qp);
             sv[i] = vis ? sv[i] * p.scale_log2 : -INFINITY;
-            mt = fmaxf(mt, sv[i]);
+            mh = fmaxf(mh, sv[i]);
           }
         } else {
+          const int kp0 = tl.kpos[half];
 #pragma unroll
           for (int i = 0; i < 64; ++i) {
-            const bool vis = (i < t.n_valid) && (t.kpos0 + i <= qp);
+            const bool vis = (i < nvh) && (kp0 + i <= qp);
             sv[i] = vis ? sv[i] * p.scale_log2 : -INFINITY;
-            mt = fmaxf(mt, sv[i]);
+            mh = fmaxf(mh, sv[i]);
           }
         }
+        // the two lanes of a head row agree on the tile max
+        sMax[(it & 1) * kM + t] = mh;
+        mbar_arrive(&bar->row_sync[it & 1]);
+        if (!wait_warp(&bar->row_sync[it & 1], (it >> 1) & 1)) { fail(ok); break; }
+        const float mt = fmaxf(mh, sMax[(it & 1) * kM + (t ^ 64)]);
+
         const bool need = mt > m_run + kRescaleThreshold;
         const float m_new = need ? mt : m_run;
-        const float factor = need ? exp2f(m_run - m_new) : 1.f;   // exp2(-inf) = 0
+        const float factor = need ? exp2f(m_run - m_new) : 1.f;
         uint32_t pk[32];
         float lsum = 0.f;
 #pragma unroll
@@ -527,9 +633,12 @@ decode_tc_kernel(const __grid_constant__ Params p,
         l_run = l_run * factor + lsum;
         m_run = m_new;
 
-        // correct O when this row's reference max moved (warp-uniform TMEM access)
+        // o_done completes once per P.c product; its phases are waited in
+        // order (a parity wait can only tell apart adjacent phases)
+        if (have_o) {
+          if (!wait_o_done(it - 1)) { fail(ok); break; }
+        }
         if (have_o && __any_sync(0xffffffffu, need)) {
-          if (!mbar_wait(&bar->o_done, (it - 1) & 1)) { fail(ok); break; }
           tc_fence_after();
           const float f = need ? factor : 1.f;
 #pragma unroll 1
@@ -544,48 +653,50 @@ decode_tc_kernel(const __grid_constant__ Params p,
           tmem_wait_st();
         }
 
-        // P (bf16, 128-byte swizzled K-major rows) for the P.c product
         const int pb = it & 1;
-        if (!mbar_wait(&bar->p_empty[pb], ((it >> 1) & 1) ^ 1)) { fail(ok); break; }
-        uint8_t* prow = sP + pb * kPBytes + m * 128;
+        if (!wait_warp(&bar->p_empty[pb], ((it >> 1) & 1) ^ 1)) { fail(ok); break; }
+        uint8_t* prow = sP + pb * kPBuf + half * kPanel + hl * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          *reinterpret_cast<uint4*>(prow + ((c ^ (m & 7)) << 4)) =
+          *reinterpret_cast<uint4*>(prow + ((c ^ (hl & 7)) << 4)) =
               make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         }
         fence_proxy_async();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar->p_full[pb]);
+        if (lane == 0) arrive_leader(&bar->p_full[pb], rank);
         have_o = true;
         ++it;
         walk_next(p, w);
       }
       if (!ok) break;
 
-      // epilogue: O is complete once the last P.c product of the stream is done
-      if (!mbar_wait(&bar->o_done, (it - 1) & 1)) { fail(ok); break; }
+      // epilogue: O of the stream is complete once its last P.c is done
+      if (!wait_o_done(it - 1)) { fail(ok); break; }
       tc_fence_after();
+      sL[t] = l_run;
+      mbar_arrive(&bar->l_sync);
+      if (!wait_warp(&bar->l_sync, n_epi & 1)) { fail(ok); break; }
+      ++n_epi;
+      const float l_tot = l_run + sL[t ^ 64];
       const int off_s = p.stream_off[s];
       const int range_u0 = g * p.plan->C;
       const bool whole = (off_s >= range_u0) && (off_s + T <= w.u1);
-      const bool empty = !(l_run > 0.f);
-      const float inv = empty ? 0.f : 1.f / l_run;
-      const float lse = empty ? -INFINITY : (m_run + log2f(l_run)) * 0.6931471805599453f;
-      float* dst;
-      size_t lse_idx;
-      float* lse_base;
+      const bool empty = !(l_tot > 0.f);
+      const float inv = empty ? 0.f : 1.f / l_tot;
+      const float lse = empty ? -INFINITY : (m_run + log2f(l_tot)) * 0.6931471805599453f;
+      float* orow;
+      float* lse_ptr;
       if (whole) {
-        const size_t orow = (size_t)qi * a.H + a.h0 + hrow;
-        dst = a.o_lat + orow * kDc + rank * 256;
-        lse_base = a.lse;
-        lse_idx = orow;
+        const size_t r = (size_t)qi * a.H + a.h0 + hrow;
+        orow = a.o_lat + r * kDc;
+        lse_ptr = a.lse + r;
       } else {
         const int slot = 2 * g + ((off_s <= range_u0) ? 0 : 1);
         float* sl = p.partial + (size_t)slot * kSlotFloats;
-        dst = sl + (size_t)m * kDc + rank * 256;
-        lse_base = sl + (size_t)kM * kDc;
-        lse_idx = m;
+        const int m = kMh * (int)rank + hl;
+        orow = sl + (size_t)m * kDc;
+        lse_ptr = sl + (size_t)kM * kDc + m;
       }
 #pragma unroll 1
       for (int c = 0; c < 256; c += 32) {
@@ -593,28 +704,27 @@ decode_tc_kernel(const __grid_constant__ Params p,
         tmem_ld32(trow + kColO + c, ov);
         tmem_wait_ld();
         if (row_valid) {
+          const int lat = 256 * (c >> 7) + 128 * half + (c & 127);
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            *reinterpret_cast<float4*>(dst + c + i) =
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(orow + lat + i) =
                 make_float4(ov[i] * inv, ov[i + 1] * inv, ov[i + 2] * inv, ov[i + 3] * inv);
-          }
         }
       }
-      if (row_valid && rank == 0) lse_base[lse_idx] = lse;
+      if (row_valid && half == 0) *lse_ptr = lse;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar->o_free);
-      ++n_streams_done;
+      if (lane == 0) arrive_leader(&bar->o_free, rank);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  cluster_sync();   // no CTA leaves while its peer may still touch its shared memory
+  cluster_sync();   // no CTA leaves while its peer may still touch its memory
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc_pair(tmem, kTmemCols);
   }
 }
 
@@ -624,7 +734,6 @@ __global__ void plan_kernel(DecodeArgs a, int n_hb, int G, PlanHeader* plan, int
                             int* stream_bad) {
   const int n_rt = a.s_q * n_hb;
   const int n_streams = a.B * n_rt;
-  __shared__ int s_total;
   for (int b = threadIdx.x; b < a.B; b += blockDim.x) {
     int tiles = 0;
     bool bad = false;
@@ -633,22 +742,22 @@ __global__ void plan_kernel(DecodeArgs a, int n_hb, int G, PlanHeader* plan, int
     for (int s = 0; s < a.max_segs; ++s) {
       const int rb = sg[s].row_begin, re = sg[s].row_end;
       if (re == rb) continue;
-      if (rb < prev_end || re < rb || rb % kN != 0 || re > a.max_pages * kN ||
+      if (rb < prev_end || re < rb || rb % kPg != 0 || re > a.max_pages * kPg ||
           sg[s].q_version < 0 || sg[s].q_version >= a.n_ver) {
         bad = true;
         break;
       }
       prev_end = re;
-      tiles += (re - rb + kN - 1) / kN;
+      tiles += seg_tiles(re - rb);
     }
-    if (a.gather_rows) {
+    if (a.gather_rows && !bad) {
       const int ng = a.n_gather[b];
       if (ng < 0 || ng > a.max_gather) bad = true;
-      tiles = bad ? 0 : (ng + kN - 1) / kN;
-      // every tile of gathered rows must share one query version
+      tiles = bad ? 0 : (ng + kT - 1) / kT;
+      // the gathered rows of one tile must share one relocation version
       for (int k = 0; !bad && k < tiles; ++k) {
         int v0 = -1;
-        for (int i = k * kN; i < min(ng, k * kN + kN); ++i) {
+        for (int i = k * kT; i < min(ng, k * kT + kT); ++i) {
           const int r = a.gather_rows[(size_t)b * a.max_gather + i];
           int v = -1;
           for (int s = 0; s < a.max_segs; ++s)
@@ -663,7 +772,7 @@ __global__ void plan_kernel(DecodeArgs a, int n_hb, int G, PlanHeader* plan, int
       tiles = 0;
     }
     for (int r = 0; r < n_rt; ++r) {
-      stream_off[b * n_rt + r] = tiles;     // counts for now
+      stream_off[b * n_rt + r] = tiles;
       stream_bad[b * n_rt + r] = bad ? 1 : 0;
     }
   }
@@ -676,7 +785,6 @@ __global__ void plan_kernel(DecodeArgs a, int n_hb, int G, PlanHeader* plan, int
       acc += c;
     }
     stream_off[n_streams] = acc;
-    s_total = acc;
     plan->U = acc;
     plan->G = G;
     plan->n_streams = n_streams;
@@ -685,76 +793,60 @@ __global__ void plan_kernel(DecodeArgs a, int n_hb, int G, PlanHeader* plan, int
 }
 
 // ----------------------------------------------------------------- combine
-// One CTA per stream: merge the split partials by log-sum-exp, or write the
-// empty result for streams with no tiles (NaN when the sequence was invalid).
+// grid (n_streams, kM / 8), a warp per query row.  Streams covered by one
+// pair were written directly; split streams are merged here by log-sum-exp;
+// streams without tiles get the empty result (NaN for an invalid sequence).
 __global__ void __launch_bounds__(256) combine_kernel(DecodeArgs a, int n_hb,
                                                       const PlanHeader* plan,
                                                       const int* stream_off,
                                                       const int* stream_bad,
                                                       const float* partial) {
   const int s = blockIdx.x;
+  const int m = blockIdx.y * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
   const int hb = s % n_hb;
-  const int qi = s / n_hb;             // (b * s_q + j)
+  const int qi = s / n_hb;
   const int rows = min(kM, a.n_h - hb * kM);
+  if (m >= rows) return;
   const int T = stream_off[s + 1] - stream_off[s];
-  const int C = plan->C;
-  __shared__ int slot_s[8];
+  const size_t orow = (size_t)qi * a.H + a.h0 + hb * kM + m;
+  float* o = a.o_lat + orow * kDc;
   if (T == 0) {
     const float fill = stream_bad[s] ? __int_as_float(0x7fc00000) : 0.f;
-    const float lfill = stream_bad[s] ? __int_as_float(0x7fc00000) : -INFINITY;
-    for (int e = threadIdx.x; e < rows * kDc; e += blockDim.x) {
-      const int m = e / kDc, c = e % kDc;
-      a.o_lat[((size_t)qi * a.H + a.h0 + hb * kM + m) * kDc + c] = fill;
-    }
-    for (int m = threadIdx.x; m < rows; m += blockDim.x)
-      a.lse[(size_t)qi * a.H + a.h0 + hb * kM + m] = lfill;
+    for (int c = lane; c < kDc; c += 32) o[c] = fill;
+    if (lane == 0) a.lse[orow] = stream_bad[s] ? __int_as_float(0x7fc00000) : -INFINITY;
     return;
   }
+  const int C = plan->C;
   const int off = stream_off[s];
   const int g0 = off / C, g1 = (off + T - 1) / C;
-  if (g0 == g1) return;   // a single worker covered the stream and wrote it
-  const int ns = g1 - g0 + 1;
-  // merge in groups of up to 8 splits (running log-sum-exp across groups)
-  for (int m = 0; m < rows; ++m) {
-    const size_t orow = (size_t)qi * a.H + a.h0 + hb * kM + m;
-    float run_l = -INFINITY;
-    for (int gb = 0; gb < ns; gb += 8) {
-      const int cnt = min(8, ns - gb);
-      __syncthreads();
-      if (threadIdx.x < cnt) {
-        const int gg = g0 + gb + threadIdx.x;
-        slot_s[threadIdx.x] = 2 * gg + ((off <= gg * C) ? 0 : 1);
-      }
-      __syncthreads();
-      float l_i[8];
-      float lmax = run_l;
-      for (int i = 0; i < cnt; ++i) {
-        l_i[i] = partial[(size_t)slot_s[i] * kSlotFloats + (size_t)kM * kDc + m];
-        lmax = fmaxf(lmax, l_i[i]);
-      }
-      float wrun = 0.f, wi[8], tot = 0.f;
-      if (lmax != -INFINITY) {
-        wrun = (run_l == -INFINITY) ? 0.f : __expf(run_l - lmax);
-        tot = wrun;
-        for (int i = 0; i < cnt; ++i) {
-          wi[i] = (l_i[i] == -INFINITY) ? 0.f : __expf(l_i[i] - lmax);
-          tot += wi[i];
-        }
-      } else {
-        for (int i = 0; i < cnt; ++i) wi[i] = 0.f;
-      }
-      const float inv = (tot > 0.f) ? 1.f / tot : 0.f;
-      for (int c = threadIdx.x; c < kDc; c += blockDim.x) {
-        float acc = (gb == 0) ? 0.f : a.o_lat[orow * kDc + c] * wrun;
-        for (int i = 0; i < cnt; ++i) {
-          if (wi[i] != 0.f) acc += wi[i] * partial[(size_t)slot_s[i] * kSlotFloats + (size_t)m * kDc + c];
-        }
-        a.o_lat[orow * kDc + c] = acc * inv;
-      }
-      run_l = (tot > 0.f) ? lmax + logf(tot) : -INFINITY;
-    }
-    if (threadIdx.x == 0) a.lse[orow] = run_l;
+  if (g0 == g1) return;   // one pair covered the stream and wrote it
+  float lmax = -INFINITY;
+  for (int gg = g0; gg <= g1; ++gg) {
+    const int slot = 2 * gg + ((off <= gg * C) ? 0 : 1);
+    lmax = fmaxf(lmax, partial[(size_t)slot * kSlotFloats + (size_t)kM * kDc + m]);
   }
+  float acc[kDc / 32];
+#pragma unroll
+  for (int i = 0; i < kDc / 32; ++i) acc[i] = 0.f;
+  float tot = 0.f;
+  if (lmax != -INFINITY) {
+    for (int gg = g0; gg <= g1; ++gg) {
+      const int slot = 2 * gg + ((off <= gg * C) ? 0 : 1);
+      const float* sl = partial + (size_t)slot * kSlotFloats;
+      const float li = sl[(size_t)kM * kDc + m];
+      if (li == -INFINITY) continue;
+      const float wgt = __expf(li - lmax);
+      tot += wgt;
+      const float* src = sl + (size_t)m * kDc;
+#pragma unroll
+      for (int i = 0; i < kDc / 32; ++i) acc[i] = fmaf(wgt, src[lane + 32 * i], acc[i]);
+    }
+  }
+  const float inv = tot > 0.f ? 1.f / tot : 0.f;
+#pragma unroll
+  for (int i = 0; i < kDc / 32; ++i) o[lane + 32 * i] = acc[i] * inv;
+  if (lane == 0) a.lse[orow] = tot > 0.f ? lmax + logf(tot) : -INFINITY;
 }
 
 }  // namespace tc

@@ -250,10 +250,10 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
   if (!aligned(workspace, 256)) return MLA_ERR_INVALID_ARG;
 
   CUtensorMap tm_q, tm_kv[tc::kNumBoxHeights];
-  if (!make_map_576(&tm_q, q_abs, (uint64_t)n_ver * B * s_q * dims->H, tc::kM))
+  if (!make_map_576(&tm_q, q_abs, (uint64_t)n_ver * B * s_q * dims->H, tc::kMh))
     return MLA_ERR_CUDA;
   for (int i = 0; i < tc::kNumBoxHeights; ++i)
-    if (!make_map_576(&tm_kv[i], cache, (uint64_t)n_pages * kPage, (uint32_t)(tc::kN >> i)))
+    if (!make_map_576(&tm_kv[i], cache, (uint64_t)n_pages * kPage, (uint32_t)(64 >> i)))
       return MLA_ERR_CUDA;
 
   if (!dev->tc_attr_set) {
@@ -283,7 +283,8 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
       p, tm_q, tm_kv[0], tm_kv[1], tm_kv[2], tm_kv[3], tm_kv[4], tm_kv[5], tm_kv[6]);
   if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
 
-  tc::combine_kernel<<<n_streams, 256, 0, st>>>(a, n_hb, plan, stream_off, stream_bad, partial);
+  tc::combine_kernel<<<dim3(n_streams, tc::kM / 8), 256, 0, st>>>(a, n_hb, plan, stream_off,
+                                                                  stream_bad, partial);
   return launch_ok();
 }
 
