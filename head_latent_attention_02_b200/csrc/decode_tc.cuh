@@ -11,19 +11,28 @@
 // Decomposition.  A cluster of two CTAs on two SMs shares one tcgen05 MMA
 // (cta_group::2): CTA r holds the query rows of heads [64r, 64r + 64) and the
 // cache rows of page 2k + r of a 128-row tile; the pair computes the full
-// 128 x 128 score tile, each CTA receiving its 64 head rows in TMEM (tokens
-// 0-63 in lanes 0-63, tokens 64-127 in lanes 64-127 of the same columns).
-// The softmax of a head row is shared by lanes t and t + 64 (the row max is
-// combined through shared memory).  P . c runs as two M=128 x N=256 pair
-// MMAs (latent halves); each CTA supplies the c columns of its N half for all
-// 128 rows, re-read through L2 in 8 KB stages, and accumulates O for its 64
-// heads in 256 TMEM columns (lanes 0-63: latent [0,128) and [256,384);
-// lanes 64-127: [128,256) and [384,512)).  No scores or probabilities cross
-// between the SMs: only the MMA operands do, inside the pair instruction.
+// 128 x 128 score tile (as two N=64 MMAs over 32-row halves of the pages),
+// each CTA receiving its 64 head rows in TMEM (tokens 0-63 in lanes 0-63,
+// tokens 64-127 in lanes 64-127 of the same columns).  The softmax of a head
+// row is shared by lanes t and t + 64 (the row max is combined through
+// shared memory).  P . c runs as M=128 x N=256 pair MMAs over the two latent
+// halves; each CTA supplies the c columns of its N half for all 128 rows,
+// re-read through L2, and accumulates O for its 64 heads in 256 TMEM columns
+// (lanes 0-63: latent [0,128) and [256,384); lanes 64-127: [128,256) and
+// [384,512)).  No scores or probabilities cross between the SMs: only the
+// MMA operands do, inside the pair instruction.
 //
-// Roles per CTA (192 threads): warp 0 streams Q, cache and value stages
-// (TMA), warp 1 of CTA 0 issues every MMA of the pair, warps 2-5 own one
-// TMEM lane each for softmax and the epilogue.  Work is split over CTA pairs
+// Loads.  Full rows are fetched with multi-dimensional TMA boxes so that each
+// request covers contiguous row bytes: a score stage is one box of 32 cache
+// rows x all 9 64-column panels (36 KB, whole 1152-byte rows), a value stage
+// one box of 32 rows x this CTA's four latent panels (16 KB), Q one box of
+// 64 rows x 9 panels.  Partial pages and gathered rows use per-panel boxes of
+// power-of-two heights, and rows without data come from boxes placed past the
+// end of the cache, which the hardware fills with zeros.
+//
+// Roles per CTA (224 threads): warp 0 streams Q and the score stages, warp 6
+// the value stages (TMA), warp 1 of CTA 0 issues every MMA of the pair,
+// warps 2-5 own one TMEM lane each for softmax and the epilogue.  Work is split over CTA pairs
 // as contiguous runs of (sequence, head block, tile) units; a pair writes
 // the final result of a sequence it covers entirely, else a normalised
 // partial (o, lse) that the combine kernel merges.
@@ -41,23 +50,28 @@ constexpr int kM = 128;                  // query rows of the pair
 constexpr int kMh = 64;                  // query rows per CTA
 constexpr int kT = 128;                  // cache rows per tile (two pages)
 constexpr int kPg = 64;                  // rows per page
-constexpr int kPanel = 8192;             // 64 rows x 128 B, 128-byte swizzle
+constexpr int kR = 32;                   // cache rows per load stage
 constexpr int kQPanels = 9;              // 8 latent + 1 rotary 64-column panels
-constexpr int kStages = 14;              // 8 KB ring stages (K panels and V halves)
+constexpr int kQPanel = kMh * 128;       // 64 rows x 128 B = 8 KB
+constexpr int kSPanel = kR * 128;        // 32 rows x 128 B = 4 KB
+constexpr int kKStage = kQPanels * kSPanel;   // 36 KB: 32 rows x 9 panels
+constexpr int kVStage = 4 * kSPanel;          // 16 KB: 32 rows x this CTA's 4 latent panels
+constexpr int kKStages = 2, kVStages = 3;
 constexpr int kOffQ = 0;
-constexpr int kOffRing = kOffQ + kQPanels * kPanel;
-constexpr int kOffP = kOffRing + kStages * kPanel;
-constexpr int kPBuf = 2 * kPanel;        // 64 rows x 128 tokens bf16
+constexpr int kOffK = kOffQ + kQPanels * kQPanel;
+constexpr int kOffV = kOffK + kKStages * kKStage;
+constexpr int kOffP = kOffV + kVStages * kVStage;
+constexpr int kPBuf = 2 * kQPanel;       // 64 rows x 128 tokens bf16 (two 64-token panels)
 constexpr int kOffMisc = kOffP + 2 * kPBuf;
-constexpr int kMiscBytes = 2048;
+constexpr int kMiscBytes = 1536;
 constexpr int kOffBar = kOffMisc + kMiscBytes;
 constexpr int kBarBytes = 512;
 constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;   // + alignment slack
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
 constexpr int kTmemCols = 512;
 constexpr int kColO = 0, kColS = 256;
 constexpr int kMinChunk = 2;
-constexpr int kNumBoxHeights = 7;        // 64, 32, 16, 8, 4, 2, 1 rows
+constexpr int kNumBoxHeights = 6;        // 32, 16, 8, 4, 2, 1 rows
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: lazy rescale margin
 constexpr size_t kSlotFloats = (size_t)kM * kDc + kM;   // partial: o rows + lse
@@ -65,6 +79,18 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct PlanHeader {
   int U, C, G, n_streams;
+};
+
+// TMA descriptors (all 64 columns wide, 128-byte swizzle):
+//   q   3-D (col, q_abs row, panel): 64 rows x 9 panels of one head block
+//   k   3-D (col, cache row, panel): 32 rows x 9 panels
+//   v   4-D (col, cache row, panel in group, group): 32 rows x 2 x 2 panels,
+//       panel p of group g covering latent columns 256 g + 64 p
+//   row 2-D (col, cache row): boxes of 32 >> i rows (i = 0..5) for partial
+//       pages, gathered rows and zero rows past the end of the cache
+struct Maps {
+  CUtensorMap q, k, v;
+  CUtensorMap row[kNumBoxHeights];
 };
 
 struct Params {
@@ -83,9 +109,9 @@ struct Tile {
   bool gather;
   int g0;              // gather: index of the tile's first gathered row
   int n_rows;          // gather: gathered rows in the tile (1..128)
-  long long phys[2];   // page mode: physical row of each page's row 0
-  int nv[2];           // page mode: valid rows of each page (0 = absent)
-  int kpos[2];         // page mode: request position of each page's row 0
+  long long phys0, phys1;   // page mode: physical row of each page's row 0
+  int nv0, nv1;             // page mode: valid rows of each page (0 = absent)
+  int kpos0, kpos1;         // page mode: request position of each page's row 0
 };
 
 // Number of 128-row tiles of a segment of len rows (pages are paired inside
@@ -101,11 +127,9 @@ __device__ __forceinline__ Tile describe(const DecodeArgs& a, int b, int k) {
   t.ver = 0;
   t.g0 = 0;
   t.n_rows = 0;
-  for (int i = 0; i < 2; ++i) {
-    t.phys[i] = 0;
-    t.nv[i] = 0;
-    t.kpos[i] = 0;
-  }
+  t.phys0 = t.phys1 = 0;
+  t.nv0 = t.nv1 = 0;
+  t.kpos0 = t.kpos1 = 0;
   const mla_seg_t* sg = a.segs + (size_t)b * a.max_segs;
   if (t.gather) {
     const int ng = a.n_gather[b];
@@ -124,18 +148,23 @@ __device__ __forceinline__ Tile describe(const DecodeArgs& a, int b, int k) {
     if (rem < nt) {
       t.ver = sg[s].q_version;
       const int np = (len + kPg - 1) / kPg;
+#pragma unroll
       for (int i = 0; i < 2; ++i) {
         const int pi = 2 * rem + i;
         if (pi >= np) break;
         const int row0 = sg[s].row_begin + pi * kPg;
         const int page = a.block_table[(size_t)b * a.max_pages + row0 / kPg];
-        t.kpos[i] = sg[s].key_pos_base + (row0 - sg[s].row_begin);
+        const int kp = sg[s].key_pos_base + (row0 - sg[s].row_begin);
+        int nv = 0;
+        long long ph = 0;
         if (page >= 0 && page < a.n_pages) {
-          t.nv[i] = min(kPg, sg[s].row_end - row0);
-          t.phys[i] = (long long)page * kPg;
+          nv = min(kPg, sg[s].row_end - row0);
+          ph = (long long)page * kPg;
         } else {
           set_status(MLA_ERR_BAD_INDEX);   // the page's rows are left out, never read
         }
+        if (i == 0) { t.kpos0 = kp; t.nv0 = nv; t.phys0 = ph; }
+        else        { t.kpos1 = kp; t.nv1 = nv; t.phys1 = ph; }
       }
       return t;
     }
@@ -146,8 +175,11 @@ __device__ __forceinline__ Tile describe(const DecodeArgs& a, int b, int k) {
 
 // rows of tile half i (tile rows [64 i, 64 i + 64)) that hold data
 __device__ __forceinline__ int half_rows(const Tile& t, int i) {
-  return t.gather ? max(0, min(kPg, t.n_rows - kPg * i)) : t.nv[i];
+  if (t.gather) return max(0, min(kPg, t.n_rows - kPg * i));
+  return i ? t.nv1 : t.nv0;
 }
+__device__ __forceinline__ long long half_phys(const Tile& t, int i) { return i ? t.phys1 : t.phys0; }
+__device__ __forceinline__ int half_kpos(const Tile& t, int i) { return i ? t.kpos1 : t.kpos0; }
 
 struct Walk {
   int s, k, u, u1;
@@ -198,7 +230,8 @@ __device__ __forceinline__ StreamPos stream_pos(const Params& p, int s) {
 
 // ----------------------------------------------------------------- barriers
 struct Bars {
-  uint64_t full[kStages], empty[kStages];
+  uint64_t kfull[kKStages], kempty[kKStages];
+  uint64_t vfull[kVStages], vempty[kVStages];
   uint64_t q_full, q_empty;
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full[2], p_empty[2];
@@ -229,42 +262,32 @@ __device__ __forceinline__ void arrive_leader(uint64_t* bar, uint32_t rank) {
   else mbar_arrive_cluster_addr(mapa(smem_u32(bar), 0));
 }
 
-// Load `rows` rows (starting at physical cache row y) of one 64-column panel
-// into smem with row pitch 128 B, as power-of-two boxes (heights 64..1).
-__device__ __forceinline__ void load_rows(uint8_t* dst, const CUtensorMap* const* maps,
-                                          uint32_t bar, int x, long long y, int rows) {
-  int r = 0;
+// Fill smem rows [r0, r0 + n) (pitch 128 B) of one 64-column panel from
+// cache rows starting at y, as power-of-two boxes.  A y at or past the end of
+// the cache (oob) makes the hardware fill the rows with zeros, so rows
+// without data read as 0 in the P.c product without any generic-proxy store.
+__device__ __forceinline__ void load_rows(uint8_t* dst, const Maps& mp, uint32_t bar, int x,
+                                          long long y, int r0, int n) {
+  int r = r0;
 #pragma unroll 1
   for (int hb = 0; hb < kNumBoxHeights; ++hb) {
-    const int h = 64 >> hb;
-    if (rows & h) {
-      tma_load_2d_pair(dst + r * 128, maps[hb], bar, x, (int)(y + r));
+    const int h = kR >> hb;
+    if (n & h) {
+      tma_load_2d_pair(dst + r * 128, &mp.row[hb], bar, x, (int)(y + (r - r0)));
       r += h;
     }
   }
 }
 
-__device__ __forceinline__ void zero_rows(uint8_t* dst, int r0, int r1, int lane) {
-  for (int e = lane; e < (r1 - r0) * 8; e += 32)
-    *reinterpret_cast<uint4*>(dst + (r0 + e / 8) * 128 + (e % 8) * 16) = make_uint4(0, 0, 0, 0);
-}
-
 // ----------------------------------------------------------------- kernel
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-decode_tc_kernel(const __grid_constant__ Params p,
-                 const __grid_constant__ CUtensorMap tm_q,
-                 const __grid_constant__ CUtensorMap tm_kv0,
-                 const __grid_constant__ CUtensorMap tm_kv1,
-                 const __grid_constant__ CUtensorMap tm_kv2,
-                 const __grid_constant__ CUtensorMap tm_kv3,
-                 const __grid_constant__ CUtensorMap tm_kv4,
-                 const __grid_constant__ CUtensorMap tm_kv5,
-                 const __grid_constant__ CUtensorMap tm_kv6) {
+decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + kOffQ;
-  uint8_t* sRing = smem + kOffRing;
+  uint8_t* sK = smem + kOffK;
+  uint8_t* sV = smem + kOffV;
   uint8_t* sP = smem + kOffP;
   float* sMax = reinterpret_cast<float*>(smem + kOffMisc);         // [2][128]
   float* sL = sMax + 2 * kM;                                       // [128]
@@ -277,11 +300,15 @@ decode_tc_kernel(const __grid_constant__ Params p,
   const int g = blockIdx.x >> 1;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&bar->full[i], 2);   // rank 0 arms both CTAs' bytes; rank 1 arrives after
-      mbar_init(&bar->empty[i], 1);  // its zero-fill and loads are issued
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(&bar->kfull[i], 1);    // rank 0 arms both CTAs' bytes
+      mbar_init(&bar->kempty[i], 1);
     }
-    mbar_init(&bar->q_full, 2);
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(&bar->vfull[i], 1);
+      mbar_init(&bar->vempty[i], 1);
+    }
+    mbar_init(&bar->q_full, 1);
     mbar_init(&bar->q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar->s_full[i], 1);
@@ -311,166 +338,134 @@ decode_tc_kernel(const __grid_constant__ Params p,
   const bool has_work = walk_begin(p, g, w);
   bool ok = true;
 
-  if (warp == 0) {
+  if (warp == 0 || warp == 6) {
     // ------------------------------------------------------------ loads
+    // Every stage lands the same byte count in each CTA, all by TMA (rows
+    // without data come from out-of-bounds boxes, which read as zero), so
+    // rank 0 arms each stage with both CTAs' bytes and rank 1 never signals.
+    const long long y_oob = a.n_pages * kPg;   // first row past the cache
+    int nk = 0, nv = 0, n_qload = 0, cur_s = -1, cur_v = -1;
     if (lane == 0) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_kv0);
-      prefetch_tmap(&tm_kv1);
+      prefetch_tmap(&mp.q);
+      prefetch_tmap(&mp.k);
+      prefetch_tmap(&mp.v);
+      for (int i = 0; i < kNumBoxHeights; ++i) prefetch_tmap(&mp.row[i]);
     }
-    const CUtensorMap* maps[kNumBoxHeights] = {&tm_kv0, &tm_kv1, &tm_kv2, &tm_kv3,
-                                               &tm_kv4, &tm_kv5, &tm_kv6};
-    int n_stage = 0, n_qload = 0, cur_s = -1, cur_v = -1;
-    // wait for the next ring stage to be free
-    auto stage_begin = [&](uint8_t*& dst, uint32_t& fb) -> bool {
-      const int slot = n_stage % kStages;
-      if (!wait_warp(&bar->empty[slot], ((n_stage / kStages) & 1) ^ 1)) return false;
-      dst = sRing + slot * kPanel;
-      fb = mapa(smem_u32(&bar->full[slot]), 0);
+    // rows [r0, r0 + n) of one panel from gathered rows gi, gi+1, ... of
+    // sequence b (one box per row; rows that cannot be located read as zero)
+    auto gather_panel = [&](uint8_t* dst, uint32_t fb, int b, int gi, int n, int x) {
+      for (int i = lane; i < n; i += 32) {
+        long long phys;
+        int kp, vv;
+        if (!locate_row(a, b, gi + i, &phys, &kp, &vv)) phys = y_oob;
+        tma_load_2d_pair(dst + i * 128, &mp.row[kNumBoxHeights - 1], fb, x, (int)phys);
+      }
+    };
+    // score stage j of tile t: rows [32 j, +32) of this CTA's page, 9 panels
+    auto load_k = [&](const Tile& t, int b, int j) -> bool {
+      const int slot = nk % kKStages;
+      if (!wait_warp(&bar->kempty[slot], ((nk / kKStages) & 1) ^ 1)) return false;
+      uint8_t* dst = sK + slot * kKStage;
+      const uint32_t fb = mapa(smem_u32(&bar->kfull[slot]), 0);
+      if (rank == 0 && lane == 0) mbar_arrive_expect_tx(&bar->kfull[slot], 2 * kKStage);
+      const int rows = max(0, min(kR, half_rows(t, (int)rank) - kR * j));
+      if (t.gather) {
+        for (int pn = 0; pn < kQPanels; ++pn)
+          gather_panel(dst + pn * kSPanel, fb, b, t.g0 + kPg * (int)rank + kR * j, rows, 64 * pn);
+      }
+      if (lane == 0) {
+        if (!t.gather && rows == kR) {
+          tma_load_3d_pair(dst, &mp.k, fb, 0, (int)(half_phys(t, (int)rank) + kR * j), 0);
+        } else {
+          for (int pn = 0; pn < kQPanels; ++pn) {
+            if (!t.gather)
+              load_rows(dst + pn * kSPanel, mp, fb, 64 * pn, half_phys(t, (int)rank) + kR * j, 0, rows);
+            load_rows(dst + pn * kSPanel, mp, fb, 64 * pn, y_oob, rows, kR - rows);
+          }
+        }
+      }
+      __syncwarp();
+      ++nk;
       return true;
     };
-    // the P.c operand of tile t: for N block nb and 32-row chunk kc, this
-    // CTA's latent columns [256 nb + 128 rank, +128) of tile rows [32 kc, +32)
+    // value stage kc of tile t: tile rows [32 kc, +32), this CTA's latent
+    // columns [256 g + 128 rank, +128) of both groups g (4 panels)
     auto load_v = [&](const Tile& t, int b) -> bool {
-      for (int nb = 0; nb < 2; ++nb) {
-        for (int kc = 0; kc < 4; ++kc) {
-          uint8_t* dst;
-          uint32_t fb;
-          if (!stage_begin(dst, fb)) return false;
-          const int hi = kc >> 1, r0 = 32 * (kc & 1);
-          const int rows = max(0, min(32, half_rows(t, hi) - r0));
-          if (rows < 32) {
-            zero_rows(dst, rows, 32, lane);
-            zero_rows(dst + 4096, rows, 32, lane);
-            fence_proxy_async();
-          }
-          __syncwarp();
-          if (rank == 0 && lane == 0)
-            mbar_arrive_expect_tx(&bar->full[n_stage % kStages], 2 * rows * 256);
-          __syncwarp();
-          const int x0 = 256 * nb + 128 * (int)rank;
-          if (!t.gather) {
-            if (lane == 0) {
-              load_rows(dst, maps, fb, x0, t.phys[hi] + r0, rows);
-              load_rows(dst + 4096, maps, fb, x0 + 64, t.phys[hi] + r0, rows);
-            }
-          } else {
-            for (int i = lane; i < rows; i += 32) {
-              long long phys;
-              int kp, vv;
-              if (!locate_row(a, b, t.g0 + 32 * kc + i, &phys, &kp, &vv)) phys = -1;
-              if (phys >= 0) {
-                tma_load_2d_pair(dst + i * 128, maps[kNumBoxHeights - 1], fb, x0, (int)phys);
-                tma_load_2d_pair(dst + 4096 + i * 128, maps[kNumBoxHeights - 1], fb, x0 + 64,
-                                 (int)phys);
-              } else {
-                for (int c = 0; c < 8; ++c) {
-                  *reinterpret_cast<uint4*>(dst + i * 128 + c * 16) = make_uint4(0, 0, 0, 0);
-                  *reinterpret_cast<uint4*>(dst + 4096 + i * 128 + c * 16) = make_uint4(0, 0, 0, 0);
-                }
-                fence_proxy_async();
-                asm volatile("mbarrier.complete_tx.shared::cluster.b64 [%0], %1;"
-                             ::"r"(fb), "r"(256) : "memory");
-              }
-            }
-          }
-          __syncwarp();
-          if (rank == 1 && lane == 0) mbar_arrive_cluster_addr(fb);
-          ++n_stage;
+      for (int kc = 0; kc < 4; ++kc) {
+        const int slot = nv % kVStages;
+        if (!wait_warp(&bar->vempty[slot], ((nv / kVStages) & 1) ^ 1)) return false;
+        uint8_t* dst = sV + slot * kVStage;
+        const uint32_t fb = mapa(smem_u32(&bar->vfull[slot]), 0);
+        if (rank == 0 && lane == 0) mbar_arrive_expect_tx(&bar->vfull[slot], 2 * kVStage);
+        const int hi = kc >> 1, r0 = kR * (kc & 1);
+        const int rows = max(0, min(kR, half_rows(t, hi) - r0));
+        if (t.gather) {
+          for (int q = 0; q < 4; ++q)
+            gather_panel(dst + q * kSPanel, fb, b, t.g0 + kR * kc, rows,
+                         256 * (q >> 1) + 128 * (int)rank + 64 * (q & 1));
         }
+        if (lane == 0) {
+          if (!t.gather && rows == kR) {
+            tma_load_4d_pair(dst, &mp.v, fb, 0, (int)(half_phys(t, hi) + r0), 2 * (int)rank, 0);
+          } else {
+            for (int q = 0; q < 4; ++q) {
+              const int x = 256 * (q >> 1) + 128 * (int)rank + 64 * (q & 1);
+              if (!t.gather) load_rows(dst + q * kSPanel, mp, fb, x, half_phys(t, hi) + r0, 0, rows);
+              load_rows(dst + q * kSPanel, mp, fb, x, y_oob, rows, kR - rows);
+            }
+          }
+        }
+        __syncwarp();
+        ++nv;
       }
       return true;
     };
-    Tile prev;
-    int prev_b = 0;
-    bool have_prev = false;
+    const bool vwarp = (warp == 6);
     for (bool more = has_work; more && ok; more = (w.u < w.u1)) {
       const StreamPos sp = stream_pos(p, w.s);
       const Tile t = describe(a, sp.b, w.k);
+      if (vwarp) {
+        if (!load_v(t, sp.b)) { fail(ok); break; }
+        walk_next(p, w);
+        continue;
+      }
       if (w.s != cur_s || t.ver != cur_v) {
         if (n_qload > 0 && !wait_warp(&bar->q_empty, (n_qload - 1) & 1)) { fail(ok); break; }
         if (lane == 0) {
           const int qi = sp.b * a.s_q + sp.j;
           const int y = (t.ver * a.n_q + qi) * a.H + a.h0 + sp.hb * kM + kMh * (int)rank;
           const uint32_t qb = mapa(smem_u32(&bar->q_full), 0);
-          if (rank == 0) mbar_arrive_expect_tx(&bar->q_full, 2 * kQPanels * kPanel);
-          for (int pn = 0; pn < kQPanels; ++pn)
-            tma_load_2d_pair(sQ + pn * kPanel, &tm_q, qb, 64 * pn, y);
-          if (rank == 1) mbar_arrive_cluster_addr(qb);
+          if (rank == 0) mbar_arrive_expect_tx(&bar->q_full, 2 * kQPanels * kQPanel);
+          tma_load_3d_pair(sQ, &mp.q, qb, 0, y, 0);
         }
+        __syncwarp();
         ++n_qload;
         cur_s = w.s;
         cur_v = t.ver;
       }
-      // score operand: this CTA's tile half (rows [64 rank, +64)), 9 panels
-      const int rows = half_rows(t, rank);
-      const int both = half_rows(t, 0) + half_rows(t, 1);
-      for (int pn = 0; pn < kQPanels && ok; ++pn) {
-        uint8_t* dst;
-        uint32_t fb;
-        if (!stage_begin(dst, fb)) { fail(ok); break; }
-        if (rows < kPg) {
-          zero_rows(dst, rows, kPg, lane);
-          fence_proxy_async();
-        }
-        __syncwarp();
-        if (rank == 0 && lane == 0) mbar_arrive_expect_tx(&bar->full[n_stage % kStages], both * 128);
-        __syncwarp();
-        if (!t.gather) {
-          if (lane == 0) load_rows(dst, maps, fb, 64 * pn, t.phys[rank], rows);
-        } else {
-          for (int i = lane; i < rows; i += 32) {
-            long long phys;
-            int kp, vv;
-            if (!locate_row(a, sp.b, t.g0 + kPg * (int)rank + i, &phys, &kp, &vv)) phys = -1;
-            if (phys >= 0) {
-              tma_load_2d_pair(dst + i * 128, maps[kNumBoxHeights - 1], fb, 64 * pn, (int)phys);
-            } else {
-              for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4*>(dst + i * 128 + c * 16) = make_uint4(0, 0, 0, 0);
-              fence_proxy_async();
-              asm volatile("mbarrier.complete_tx.shared::cluster.b64 [%0], %1;"
-                           ::"r"(fb), "r"(128) : "memory");
-            }
-          }
-        }
-        __syncwarp();
-        if (rank == 1 && lane == 0) mbar_arrive_cluster_addr(fb);
-        ++n_stage;
-      }
-      if (!ok) break;
-      if (have_prev && !load_v(prev, prev_b)) { fail(ok); break; }
-      prev = t;
-      prev_b = sp.b;
-      have_prev = true;
+      if (!load_k(t, sp.b, 0) || !load_k(t, sp.b, 1)) { fail(ok); break; }
       walk_next(p, w);
     }
-    if (ok && have_prev && !load_v(prev, prev_b)) fail(ok);
-    // drain: every load this warp issued has landed before the CTA exits
-    // (rank 0 observes the shared barriers; both ranks wait for their ring)
+    // drain: every load issued here has landed before the CTA exits (the
+    // stage barriers live in rank 0, which waits on them for both CTAs)
     if (rank == 0) {
-      for (int d = 1; d <= kStages && d <= n_stage; ++d) {
-        const int n = n_stage - d;
-        if (!wait_warp(&bar->full[n % kStages], (n / kStages) & 1)) { fail(ok); break; }
+      for (int d = 1; d <= kKStages && d <= nk && ok; ++d) {
+        const int n = nk - d;
+        if (!wait_warp(&bar->kfull[n % kKStages], (n / kKStages) & 1)) fail(ok);
       }
+      for (int d = 1; d <= kVStages && d <= nv && ok; ++d) {
+        const int n = nv - d;
+        if (!wait_warp(&bar->vfull[n % kVStages], (n / kVStages) & 1)) fail(ok);
+      }
+      if (ok && !vwarp && n_qload > 0 && !wait_warp(&bar->q_full, (n_qload - 1) & 1)) fail(ok);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA (rank 0)
     if (rank == 0 && lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(kM, kT, false, false);
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kM, 64, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kM, 256, false, true);
-      int it = 0, n_stage = 0, n_q = 0, cur_s = -1, cur_v = -1, n_streams = 0;
+      int it = 0, nk = 0, nv = 0, n_q = 0, cur_s = -1, cur_v = -1, n_streams = 0;
       int prev_first = 0, prev_stream_idx = 0;
-      auto stage_wait = [&]() -> uint32_t {
-        const int slot = n_stage % kStages;
-        if (!mbar_wait_cluster(&bar->full[slot], (n_stage / kStages) & 1)) return 0;
-        tc_fence_after();
-        return smem_u32(sRing + slot * kPanel);
-      };
-      auto stage_release = [&]() {
-        mma_pair_commit_both(&bar->empty[n_stage % kStages]);
-        ++n_stage;
-      };
       auto issue_pv = [&](int t, int first, int stream_idx) -> bool {
         const int pb = t & 1;
         if (!mbar_wait_cluster(&bar->p_full[pb], (t >> 1) & 1)) return false;
@@ -478,21 +473,25 @@ decode_tc_kernel(const __grid_constant__ Params p,
           return false;
         tc_fence_after();
         const uint32_t pa = smem_u32(sP + pb * kPBuf);
-        for (int nb = 0; nb < 2; ++nb) {
-          for (int kc = 0; kc < 4; ++kc) {
-            const uint32_t vb = stage_wait();
-            if (!vb) return false;
+        for (int kc = 0; kc < 4; ++kc) {
+          const int slot = nv % kVStages;
+          if (!mbar_wait(&bar->vfull[slot], (nv / kVStages) & 1)) return false;
+          tc_fence_after();
+          const uint32_t vb = smem_u32(sV + slot * kVStage);
+#pragma unroll
+          for (int nb = 0; nb < 2; ++nb) {
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-              const int ks = 2 * kc + j;
+              const int ks = 2 * kc + j;     // 16-row step of the 128-row tile
               const uint64_t ad =
-                  smem_desc_sw128(pa + (ks >> 2) * kPanel + (ks & 3) * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(vb + j * 2048, 4096, 1024);
+                  smem_desc_sw128(pa + (ks >> 2) * kQPanel + (ks & 3) * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(vb + nb * 2 * kSPanel + j * 2048, kSPanel, 1024);
               mma_pair_bf16_ss(tmem + kColO + nb * 128, ad, bd, idesc_pv,
                                (first && ks == 0) ? 0u : 1u);
             }
-            stage_release();
           }
+          mma_pair_commit_both(&bar->vempty[slot]);
+          ++nv;
         }
         mma_pair_commit_both(&bar->p_empty[pb]);
         mma_pair_commit_both(&bar->o_done);
@@ -504,7 +503,7 @@ decode_tc_kernel(const __grid_constant__ Params p,
         const bool first = (w.s != cur_s);
         if (first) ++n_streams;
         if (first || t.ver != cur_v) {
-          if (!mbar_wait_cluster(&bar->q_full, n_q & 1)) { fail(ok); break; }
+          if (!mbar_wait(&bar->q_full, n_q & 1)) { fail(ok); break; }
           ++n_q;
           cur_s = w.s;
           cur_v = t.ver;
@@ -513,16 +512,22 @@ decode_tc_kernel(const __grid_constant__ Params p,
         if (!mbar_wait_cluster(&bar->s_empty[sb], ((it >> 1) & 1) ^ 1)) { fail(ok); break; }
         tc_fence_after();
         const uint32_t qa = smem_u32(sQ);
-        for (int pn = 0; pn < kQPanels; ++pn) {
-          const uint32_t kb = stage_wait();
-          if (!kb) { fail(ok); break; }
+        for (int j = 0; j < 2 && ok; ++j) {
+          const int slot = nk % kKStages;
+          if (!mbar_wait(&bar->kfull[slot], (nk / kKStages) & 1)) { fail(ok); break; }
+          tc_fence_after();
+          const uint32_t kb = smem_u32(sK + slot * kKStage);
+          for (int pn = 0; pn < kQPanels; ++pn) {
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t ad = smem_desc_sw128(qa + pn * kPanel + ks * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(kb + ks * 32, 16, 1024);
-            mma_pair_bf16_ss(tmem + kColS + sb * 64, ad, bd, idesc_qk, (pn | ks) ? 1u : 0u);
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t ad = smem_desc_sw128(qa + pn * kQPanel + ks * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(kb + pn * kSPanel + ks * 32, 16, 1024);
+              mma_pair_bf16_ss(tmem + kColS + sb * 64 + 32 * j, ad, bd, idesc_qk,
+                               (pn | ks) ? 1u : 0u);
+            }
           }
-          stage_release();
+          mma_pair_commit_both(&bar->kempty[slot]);
+          ++nk;
         }
         if (!ok) break;
         mma_pair_commit_both(&bar->s_full[sb]);
@@ -603,7 +608,7 @@ decode_tc_kernel(const __grid_constant__ Params p,
             mh = fmaxf(mh, sv[i]);
           }
         } else {
-          const int kp0 = tl.kpos[half];
+          const int kp0 = half_kpos(tl, half);
 #pragma unroll
           for (int i = 0; i < 64; ++i) {
             const bool vis = (i < nvh) && (kp0 + i <= qp);
@@ -655,7 +660,7 @@ decode_tc_kernel(const __grid_constant__ Params p,
 
         const int pb = it & 1;
         if (!wait_warp(&bar->p_empty[pb], ((it >> 1) & 1) ^ 1)) { fail(ok); break; }
-        uint8_t* prow = sP + pb * kPBuf + half * kPanel + hl * 128;
+        uint8_t* prow = sP + pb * kPBuf + half * kQPanel + hl * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           *reinterpret_cast<uint4*>(prow + ((c ^ (hl & 7)) << 4)) =

@@ -77,16 +77,27 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 map over a [rows, 576] matrix, box {64 columns, box_rows}, 128-byte swizzle.
-bool make_map_576(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+// Tensor map over a [rows, 576] bf16 matrix (row pitch 1152 B) with 64-column
+// boxes and 128-byte swizzle.  rank 2: (col, row), box {64, h}.  rank 3:
+// (col, row, 64-column panel), box {64, h, 9}.  rank 4: (col, row, panel
+// within a 256-column group, group), box {64, h, 2, 2}.
+bool make_map_576(CUtensorMap* m, const void* base, uint64_t rows, int rank, uint32_t h) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)tc::kRow, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)tc::kRow * 2};
-  cuuint32_t box[2] = {64, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  cuuint64_t dims[4] = {64, (cuuint64_t)rows, 9, 1};
+  cuuint64_t strides[3] = {(cuuint64_t)tc::kRow * 2, 128, 0};
+  cuuint32_t box[4] = {64, h, 9, 1};
+  if (rank == 2) dims[0] = tc::kRow;
+  if (rank == 4) {
+    dims[2] = 4;
+    dims[3] = 2;
+    strides[2] = 512;
+    box[2] = 2;
+    box[3] = 2;
+  }
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -195,7 +206,7 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
   if (B == 0) return MLA_OK;
   if (!q_abs || !cache || !block_table || !segs || !q_pos || !o_lat || !lse)
     return MLA_ERR_INVALID_ARG;
-  if (n_pages * kPage > INT32_MAX) return MLA_ERR_UNSUPPORTED;
+  if (n_pages * kPage + 2 * kPage > INT32_MAX) return MLA_ERR_UNSUPPORTED;
   const size_t es = elem_size(dims);
   if (!aligned(cache, 256) || !aligned(q_abs, 16) || !aligned(o_lat, 16) || !aligned(lse, 4))
     return MLA_ERR_INVALID_ARG;
@@ -249,11 +260,14 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
   if (!workspace || ws_bytes < wl.total) return MLA_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return MLA_ERR_INVALID_ARG;
 
-  CUtensorMap tm_q, tm_kv[tc::kNumBoxHeights];
-  if (!make_map_576(&tm_q, q_abs, (uint64_t)n_ver * B * s_q * dims->H, tc::kMh))
+  tc::Maps maps;
+  const uint64_t cache_rows = (uint64_t)n_pages * kPage;
+  if (!make_map_576(&maps.q, q_abs, (uint64_t)n_ver * B * s_q * dims->H, 3, tc::kMh) ||
+      !make_map_576(&maps.k, cache, cache_rows, 3, tc::kR) ||
+      !make_map_576(&maps.v, cache, cache_rows, 4, tc::kR))
     return MLA_ERR_CUDA;
   for (int i = 0; i < tc::kNumBoxHeights; ++i)
-    if (!make_map_576(&tm_kv[i], cache, (uint64_t)n_pages * kPage, (uint32_t)(64 >> i)))
+    if (!make_map_576(&maps.row[i], cache, cache_rows, 2, (uint32_t)(tc::kR >> i)))
       return MLA_ERR_CUDA;
 
   if (!dev->tc_attr_set) {
@@ -279,8 +293,7 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
   p.stream_off = stream_off;
   p.partial = partial;
   p.scale_log2 = dims->scale * tc::kLog2e;
-  tc::decode_tc_kernel<<<2 * G, tc::kThreads, tc::kSmemBytes, st>>>(
-      p, tm_q, tm_kv[0], tm_kv[1], tm_kv[2], tm_kv[3], tm_kv[4], tm_kv[5], tm_kv[6]);
+  tc::decode_tc_kernel<<<2 * G, tc::kThreads, tc::kSmemBytes, st>>>(p, maps);
   if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
 
   tc::combine_kernel<<<dim3(n_streams, tc::kM / 8), 256, 0, st>>>(a, n_hb, plan, stream_off,
