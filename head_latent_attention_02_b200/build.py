@@ -8,7 +8,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libmla.so")
 SOURCES = ["csrc/mla_lib.cu"]
-DEPENDS = ["csrc/mla_lib.cu", "csrc/common.cuh", "csrc/ptx.cuh", "csrc/kernels_simt.cuh",
+DEPENDS = ["csrc/mla_lib.cu", "csrc/common.cuh", "csrc/ptx.cuh", "csrc/kernels_simt.cuh", "csrc/wgemm.cuh",
            "csrc/decode_tc.cuh", "../include/mla.h"]
 
 NVCC_FLAGS = [

@@ -235,7 +235,7 @@ struct Bars {
   uint64_t q_full, q_empty;
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full[2], p_empty[2];
-  uint64_t o_done, o_free;
+  uint64_t o_done[2], o_free;       // o_done[t & 1]: P.c of tile t complete
   uint64_t mma_drain;
   uint64_t row_sync[2], l_sync;     // the 128 softmax threads of one CTA
   uint32_t tmem_base;
@@ -316,7 +316,8 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
       mbar_init(&bar->p_full[i], 8);
       mbar_init(&bar->p_empty[i], 1);
     }
-    mbar_init(&bar->o_done, 1);
+    mbar_init(&bar->o_done[0], 1);
+    mbar_init(&bar->o_done[1], 1);
     mbar_init(&bar->o_free, 8);
     mbar_init(&bar->mma_drain, 1);
     mbar_init(&bar->row_sync[0], kM);
@@ -494,7 +495,7 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
           ++nv;
         }
         mma_pair_commit_both(&bar->p_empty[pb]);
-        mma_pair_commit_both(&bar->o_done);
+        mma_pair_commit_both(&bar->o_done[pb]);
         return true;
       };
       for (bool more = has_work; more && ok; more = (w.u < w.u1)) {
@@ -554,11 +555,12 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
     const int half = t >> 6;                  // tile rows [64 half, +64)
     const int hl = t & 63;                    // head row of this CTA
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-    int it = 0, n_epi = 0, n_od = 0;
-    auto wait_o_done = [&](int target) -> bool {
-      for (; n_od <= target; ++n_od)
-        if (!wait_warp(&bar->o_done, n_od & 1)) return false;
-      return true;
+    int it = 0, n_epi = 0;
+    // P.c of tile t is complete.  o_done[t & 1] completes once per two tiles;
+    // the P buffer waits (p_empty) already ordered every earlier product of
+    // the same parity, so the barrier is never a phase ahead or behind.
+    auto wait_o_done = [&](int t) -> bool {
+      return wait_warp(&bar->o_done[t & 1], (t >> 1) & 1);
     };
     while (has_work && ok && w.u < w.u1) {
       const int s = w.s;
@@ -638,12 +640,8 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
         l_run = l_run * factor + lsum;
         m_run = m_new;
 
-        // o_done completes once per P.c product; its phases are waited in
-        // order (a parity wait can only tell apart adjacent phases)
-        if (have_o) {
-          if (!wait_o_done(it - 1)) { fail(ok); break; }
-        }
         if (have_o && __any_sync(0xffffffffu, need)) {
+          if (!wait_o_done(it - 1)) { fail(ok); break; }
           tc_fence_after();
           const float f = need ? factor : 1.f;
 #pragma unroll 1

@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include "mla.h"
@@ -13,6 +14,7 @@
 #include "ptx.cuh"
 #include "kernels_simt.cuh"
 #include "decode_tc.cuh"
+#include "wgemm.cuh"
 
 using namespace mla;
 
@@ -101,6 +103,50 @@ bool make_map_576(CUtensorMap* m, const void* base, uint64_t rows, int rank, uin
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D bf16 map over a row-major [outer, inner] matrix, box {64, box_outer},
+// 128-byte swizzle.
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                 uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  cuuint64_t strides[1] = {(cuuint64_t)inner * 2};
+  cuuint32_t box[2] = {64, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool g_wg_attr_set[kMaxDevices] = {};
+
+// Launch one weight-streaming product for query rows [q0, q0 + n), K split in
+// chunks whose bf16 X slice fits the kernel's staging buffer.
+mla_status_t launch_wgemm(wg::Params p, const CUtensorMap& tw, int m_tiles, int heads,
+                          cudaStream_t st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return MLA_ERR_CUDA;
+  if (!g_wg_attr_set[dev]) {
+    if (cudaFuncSetAttribute(wg::wgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             wg::kSmemBytes) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    g_wg_attr_set[dev] = true;
+  }
+  const int total_n = p.n;
+  for (int q0 = 0; q0 < total_n; q0 += 128) {
+    p.q0 = q0;
+    p.n = min(128, total_n - q0);
+    p.n_pad = (p.n + 15) / 16 * 16;
+    int kc = wg::kXBytesMax / (p.n_pad * 2);
+    kc = max(wg::kKP, kc / wg::kKP * wg::kKP);
+    p.k_chunk = min(p.K, kc);
+    dim3 grid(m_tiles, heads, (p.K + p.k_chunk - 1) / p.k_chunk);
+    wg::wgemm_kernel<<<grid, wg::kThreads, wg::kSmemBytes, st>>>(p, tw);
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  }
+  return MLA_OK;
+}
+
 struct WsLayout {
   size_t off_plan, off_streams, off_bad, off_partial, total;
 };
@@ -171,6 +217,32 @@ mla_status_t mla_absorb_q(const mla_dims_t* dims, int32_t n_q, const void* q_nop
   a.q_pos = q_pos;
   a.w_uk = w_uk;
   a.q_abs = q_abs;
+  cudaStream_t st0 = reinterpret_cast<cudaStream_t>(stream);
+  if (dims->dtype == MLA_BF16 && dims->d_c % wg::kMT == 0 && dims->d_n % wg::kKP == 0) {
+    CUtensorMap tw;
+    if (!make_map_2d(&tw, w_uk, dims->d_c, (uint64_t)dims->H * dims->d_n, 64)) return MLA_ERR_CUDA;
+    wg::Params p{};
+    p.mode = wg::kAbsorb;
+    p.n = n_q;
+    p.n_total = n_q;
+    p.K = dims->d_n;
+    p.H = dims->H;
+    p.d_c = dims->d_c;
+    p.d_r = dims->d_r;
+    p.d_n = dims->d_n;
+    p.d_v = dims->d_v;
+    p.d_model = dims->d_model;
+    p.x = q_nope;
+    p.x_row_stride = (long long)dims->H * dims->d_n;
+    p.x_head_stride = dims->d_n;
+    p.out = q_abs;
+    p.n_ver = n_ver;
+    for (int i = 0; i < kMaxVersions; ++i) p.delta[i] = i < n_ver ? delta[i] : 0;
+    p.rope_base = dims->rope_base;
+    p.q_rope = q_rope;
+    p.q_pos = q_pos;
+    return launch_wgemm(p, tw, dims->d_c / wg::kMT, dims->H, st0);
+  }
   dim3 grid(dims->H, (n_q + kAbsQ - 1) / kAbsQ);
   const size_t smem = sizeof(float) * kAbsQ * dims->d_n;
   if (smem > 48 * 1024) return MLA_ERR_UNSUPPORTED;
@@ -323,6 +395,44 @@ mla_status_t mla_out_proj(const mla_dims_t* dims, int32_t n_q, const float* o_la
   if (!o_lat || !w_uv || !v || (w_o && (!out || dims->d_model < 1))) return MLA_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int H = dims->H, d_c = dims->d_c, d_v = dims->d_v;
+  if (dims->dtype == MLA_BF16 && d_v % wg::kMT == 0 && d_c % wg::kKP == 0 &&
+      (!w_o || dims->d_model % wg::kMT == 0) && aligned(o_lat, 16) && aligned(v, 16)) {
+    if (w_o) {
+      const long long n_out = (long long)n_q * dims->d_model;
+      const unsigned zb = (unsigned)std::min<long long>((n_out + 255) / 256, 4096);
+      wg::zero_kernel<<<zb, 256, 0, st>>>(out, n_out);
+      if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    }
+    CUtensorMap tv;
+    if (!make_map_2d(&tv, w_uv, d_c, (uint64_t)H * d_v, wg::kMT)) return MLA_ERR_CUDA;
+    wg::Params p{};
+    p.mode = wg::kValue;
+    p.n = n_q;
+    p.n_total = n_q;
+    p.K = d_c;
+    p.H = H;
+    p.d_c = d_c;
+    p.d_r = dims->d_r;
+    p.d_n = dims->d_n;
+    p.d_v = d_v;
+    p.d_model = dims->d_model;
+    p.x = o_lat;
+    p.x_row_stride = (long long)H * d_c;
+    p.x_head_stride = d_c;
+    p.out = v;
+    mla_status_t rc = launch_wgemm(p, tv, d_v / wg::kMT, H, st);
+    if (rc != MLA_OK || !w_o) return rc;
+    CUtensorMap to;
+    if (!make_map_2d(&to, w_o, (uint64_t)H * d_v, dims->d_model, wg::kMT)) return MLA_ERR_CUDA;
+    p.mode = wg::kOutput;
+    p.n = n_q;
+    p.K = H * d_v;
+    p.x = v;
+    p.x_row_stride = (long long)H * d_v;
+    p.x_head_stride = 0;
+    p.out = out;
+    return launch_wgemm(p, to, dims->d_model / wg::kMT, 1, st);
+  }
   dim3 g1(H, (d_v + 7) / 8);
   if (dims->dtype == MLA_BF16)
     vproj_simt_kernel<__nv_bfloat16><<<g1, 256, 0, st>>>(
