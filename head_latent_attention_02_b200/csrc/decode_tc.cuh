@@ -279,6 +279,45 @@ __device__ __forceinline__ void load_rows(uint8_t* dst, const Maps& mp, uint32_t
   }
 }
 
+// Visibility of the 64 tile rows [64 half, +64) of tile t for a query at q_pos
+// qp, as a bitmask (bit i: row 64 half + i exists and key_pos <= qp).  Page
+// rows have consecutive key positions, so the mask is a prefix; gathered rows
+// are located one per lane and combined by ballot.
+__device__ __noinline__ uint64_t gather_visible(const DecodeArgs& a, const Tile& t, int b, int half,
+                                               int qp, int lane) {
+  const int nvh = half_rows(t, half);
+  const int i0 = t.g0 + kPg * half + lane;
+  int kp0 = INT32_MAX, kp1 = INT32_MAX;
+  long long ph;
+  int vv;
+  if (lane < nvh && !locate_row(a, b, i0, &ph, &kp0, &vv)) kp0 = INT32_MAX;
+  if (lane + 32 < nvh && !locate_row(a, b, i0 + 32, &ph, &kp1, &vv)) kp1 = INT32_MAX;
+  const uint32_t lo = __ballot_sync(0xffffffffu, kp0 <= qp);
+  const uint32_t hi = __ballot_sync(0xffffffffu, kp1 <= qp);
+  return (uint64_t)lo | ((uint64_t)hi << 32);
+}
+
+__device__ __forceinline__ uint64_t visible_rows(const DecodeArgs& a, const Tile& t, int b,
+                                                 int half, int qp, int lane) {
+  if (t.gather) return gather_visible(a, t, b, half, qp, lane);
+  const int n = min(half_rows(t, half), max(0, qp - half_kpos(t, half) + 1));
+  return n >= 64 ? ~0ull : ((1ull << n) - 1ull);
+}
+
+// Rescale this warp's 32 TMEM lanes of O (256 columns) by f.
+__device__ __noinline__ void scale_o(uint32_t taddr, float f) {
+#pragma unroll 1
+  for (int c = 0; c < 256; c += 32) {
+    float ov[32];
+    tmem_ld32(taddr + c, ov);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) ov[i] *= f;
+    tmem_st32(taddr + c, ov);
+  }
+  tmem_wait_st();
+}
+
 // ----------------------------------------------------------------- kernel
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
@@ -575,99 +614,78 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
       while (ok && w.u < w.u1 && w.s == s) {
         const Tile tl = describe(a, sp.b, w.k);
         const int sb = it & 1;
+        const uint64_t vis = visible_rows(a, tl, sp.b, half, qp, lane);
         if (!wait_warp(&bar->s_full[sb], (it >> 1) & 1)) { fail(ok); break; }
         tc_fence_after();
-        float sv[64];
-        {
-          float tmp[32];
-          tmem_ld32(trow + kColS + sb * 64, tmp);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) sv[i] = tmp[i];
-          tmem_ld32(trow + kColS + sb * 64 + 32, tmp);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) sv[32 + i] = tmp[i];
-          tmem_wait_ld();
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) arrive_leader(&bar->s_empty[sb], rank);
+        const uint32_t s_col = trow + kColS + sb * 64;
 
-        // mask, scale (log2 domain)
+        // pass 1: max of the visible scores of this lane's 64 rows
         float mh = -INFINITY;
-        const int nvh = half_rows(tl, half);
-        if (tl.gather) {
-          const int i0 = tl.g0 + kPg * half + lane;
-          int kp0 = INT32_MAX, kp1 = INT32_MAX;
-          long long ph;
-          int vv;
-          if (lane < nvh && !locate_row(a, sp.b, i0, &ph, &kp0, &vv)) kp0 = INT32_MAX;
-          if (lane + 32 < nvh && !locate_row(a, sp.b, i0 + 32, &ph, &kp1, &vv)) kp1 = INT32_MAX;
+#pragma unroll 1
+        for (int c = 0; c < 64; c += 16) {
+          float x[16];
+          tmem_ld16(s_col + c, x);
+          tmem_wait_ld();
+          const uint32_t bits = (uint32_t)(vis >> c);
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const int kp = __shfl_sync(0xffffffffu, (i < 32) ? kp0 : kp1, i & 31);
-            const bool vis = (i < nvh) && (kp <= qp);
-            sv[i] = vis ? sv[i] * p.scale_log2 : -INFINITY;
-            mh = fmaxf(mh, sv[i]);
-          }
-        } else {
-          const int kp0 = half_kpos(tl, half);
-#pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const bool vis = (i < nvh) && (kp0 + i <= qp);
-            sv[i] = vis ? sv[i] * p.scale_log2 : -INFINITY;
-            mh = fmaxf(mh, sv[i]);
-          }
+          for (int i = 0; i < 16; ++i)
+            if (bits & (1u << i)) mh = fmaxf(mh, x[i]);
         }
+        mh *= p.scale_log2;                   // scale > 0: max commutes, -inf stays
         // the two lanes of a head row agree on the tile max
         sMax[(it & 1) * kM + t] = mh;
         mbar_arrive(&bar->row_sync[it & 1]);
         if (!wait_warp(&bar->row_sync[it & 1], (it >> 1) & 1)) { fail(ok); break; }
         const float mt = fmaxf(mh, sMax[(it & 1) * kM + (t ^ 64)]);
 
+        // lazy rescaling: keep the reference max unless it grows by > 2^8
         const bool need = mt > m_run + kRescaleThreshold;
         const float m_new = need ? mt : m_run;
-        const float factor = need ? exp2f(m_run - m_new) : 1.f;
-        uint32_t pk[32];
-        float lsum = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = (m_new == -INFINITY) ? 0.f : exp2f(sv[2 * i] - m_new);
-          const float p1 = (m_new == -INFINITY) ? 0.f : exp2f(sv[2 * i + 1] - m_new);
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-          lsum += __low2float(h2) + __high2float(h2);
-          pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
-        }
-        l_run = l_run * factor + lsum;
-        m_run = m_new;
-
+        const float factor = need ? exp2f(m_run - m_new) : 1.f;   // exp2(-inf) = 0
         if (have_o && __any_sync(0xffffffffu, need)) {
           if (!wait_o_done(it - 1)) { fail(ok); break; }
           tc_fence_after();
-          const float f = need ? factor : 1.f;
-#pragma unroll 1
-          for (int c = 0; c < 256; c += 32) {
-            float ov[32];
-            tmem_ld32(trow + kColO + c, ov);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] *= f;
-            tmem_st32(trow + kColO + c, ov);
-          }
-          tmem_wait_st();
+          scale_o(trow + kColO, need ? factor : 1.f);
         }
 
+        // pass 2: P = 2^(scale*S - m_new) on visible rows, bf16, 128-byte
+        // swizzled K-major rows of the P.c operand
         const int pb = it & 1;
         if (!wait_warp(&bar->p_empty[pb], ((it >> 1) & 1) ^ 1)) { fail(ok); break; }
         uint8_t* prow = sP + pb * kPBuf + half * kQPanel + hl * 128;
+        float lsum = 0.f;
+        const bool any = (m_new != -INFINITY);
+#pragma unroll 1
+        for (int c = 0; c < 64; c += 16) {
+          float x[16];
+          tmem_ld16(s_col + c, x);
+          tmem_wait_ld();
+          const uint32_t bits = any ? (uint32_t)(vis >> c) : 0u;
+          uint32_t pk[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          *reinterpret_cast<uint4*>(prow + ((c ^ (hl & 7)) << 4)) =
-              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          for (int i = 0; i < 16; i += 2) {
+            const float p0 = (bits & (1u << i)) ? ex2_approx(fmaf(x[i], p.scale_log2, -m_new)) : 0.f;
+            const float p1 =
+                (bits & (2u << i)) ? ex2_approx(fmaf(x[i + 1], p.scale_log2, -m_new)) : 0.f;
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+            lsum += __low2float(h2) + __high2float(h2);
+            pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+          const int ch = c >> 3;
+          *reinterpret_cast<uint4*>(prow + ((ch ^ (hl & 7)) << 4)) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(prow + (((ch + 1) ^ (hl & 7)) << 4)) =
+              make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
-        fence_proxy_async();
+        l_run = l_run * factor + lsum;
+        m_run = m_new;
         tc_fence_before();
+        fence_proxy_async();
         __syncwarp();
-        if (lane == 0) arrive_leader(&bar->p_full[pb], rank);
+        if (lane == 0) {
+          arrive_leader(&bar->s_empty[sb], rank);
+          arrive_leader(&bar->p_full[pb], rank);
+        }
         have_o = true;
         ++it;
         walk_next(p, w);
