@@ -46,6 +46,8 @@ _SIGS = {
     "mla_decode": ([ctypes.POINTER(Dims), _i32, _i32, _vp, _i32, _i32, _i32, _vp, _i64, _vp, _i32,
                     _vp, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
     "mla_decode_workspace_size": ([ctypes.POINTER(Dims), _i32, _i32, _i32], _sz),
+    "mla_decode_static_ws": ([ctypes.POINTER(Dims), _i32, _i32, _vp, _i32, _i32, _i32, _vp, _i64,
+                              _vp, _i32, _vp, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _vp], _i32),
     "mla_merge_lse": ([_i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
     "mla_out_proj": ([ctypes.POINTER(Dims), _i32, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
 }
@@ -131,6 +133,17 @@ def decode(dims: Dims, B: int, s_q: int, q_abs, n_ver: int, h0: int, n_h: int, c
         ctypes.byref(dims), B, s_q, _p(q_abs), n_ver, h0, n_h, _p(cache), n_pages,
         _p(block_table), max_pages, _p(segs), max_segs, _p(gather_rows), _p(n_gather),
         max_gather, _p(q_pos), _p(o_lat), _p(lse), _p(workspace), ws_bytes, _s(stream)))
+
+
+def decode_static_ws(dims: Dims, B: int, s_q: int, q_abs, n_ver: int, h0: int, n_h: int, cache,
+                     block_table, segs, q_pos, o_lat, lse, gather_rows=None, n_gather=None,
+                     stream=None):
+    """mla_decode with the library's fixed scratch array instead of a workspace."""
+    max_gather = gather_rows.shape[1] if gather_rows is not None else 0
+    _check("mla_decode_static_ws", lib().mla_decode_static_ws(
+        ctypes.byref(dims), B, s_q, _p(q_abs), n_ver, h0, n_h, _p(cache), cache.shape[0],
+        _p(block_table), block_table.shape[1], _p(segs), segs.shape[1], _p(gather_rows),
+        _p(n_gather), max_gather, _p(q_pos), _p(o_lat), _p(lse), _s(stream)))
 
 
 def merge_lse(n_q: int, H: int, h0: int, n_h: int, d: int, o_a, lse_a, o_b, lse_b, o, lse,

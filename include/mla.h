@@ -12,7 +12,8 @@
  *   - Every pointer is a DEVICE pointer owned by the caller unless a comment
  *     says "host".  The library never allocates device memory and keeps no
  *     state between calls except cached per-device properties and TMA
- *     descriptors.  Buffers must not alias unless a call says so.
+ *     descriptors (mla_decode_static_ws adds one fixed static scratch
+ *     array).  Buffers must not alias unless a call says so.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
  *     legacy default stream) and returns an mla_status_t synchronously.
  *     Argument errors are reported before anything is launched and leave the
@@ -170,6 +171,39 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
  * (0 if the arguments are invalid or the device cannot be queried). */
 size_t mla_decode_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q,
                                  int32_t n_h);
+
+/* ---------------------------------------------------------------------------
+ * mla_decode_static_ws -- mla_decode without a caller workspace.  The papers
+ * have no counterpart: this is a library convenience for callers that cannot
+ * allocate device memory at decode time (a server whose KV page pool holds
+ * all free device memory; a C host without a device allocator).
+ *
+ * Arguments, layouts, results and errors are those of mla_decode minus
+ * workspace/ws_bytes.  The scratch is a static device array of
+ * MLA_DECODE_STATIC_WS_BYTES (40 MiB) inside the library, reserved when its
+ * module loads; nothing is allocated per call.
+ *   - Sizes whose mla_decode_workspace_size exceeds the array are rejected
+ *     with MLA_ERR_WORKSPACE before anything is launched (on a 148-SM device
+ *     the split partials take 38.9 MB, leaving room for about 380,000
+ *     streams of B * s_q * ceil(n_h / 128)).  Invalid dims or sizes give
+ *     MLA_ERR_INVALID_ARG.
+ *   - The first call on each device looks up the array's address with that
+ *     device current (a runtime query that may load the module); make that
+ *     first call before any stream capture.
+ *   - Every call on a device shares the one array, which keeps the previous
+ *     call's contents (nothing in it needs clearing).  Calls that overlap on
+ *     the GPU -- other streams, other host threads -- race on it: serialise
+ *     them on one stream. */
+#define MLA_DECODE_STATIC_WS_BYTES ((size_t)40 << 20)
+
+mla_status_t mla_decode_static_ws(const mla_dims_t* dims, int32_t B, int32_t s_q,
+                                  const void* q_abs, int32_t n_ver, int32_t h0, int32_t n_h,
+                                  const void* cache, int64_t n_pages,
+                                  const int32_t* block_table, int32_t max_pages,
+                                  const mla_seg_t* segs, int32_t max_segs,
+                                  const int32_t* gather_rows, const int32_t* n_gather,
+                                  int32_t max_gather, const int32_t* q_pos, float* o_lat,
+                                  float* lse, mla_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * mla_merge_lse -- merge two partial attentions over disjoint key sets.
