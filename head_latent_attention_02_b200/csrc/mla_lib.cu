@@ -26,6 +26,7 @@ struct DeviceInfo {
   bool ready = false;
   int num_sms = 0;
   bool tc_attr_set = false;
+  bool wg_attr_set = false;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -118,30 +119,53 @@ bool make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t oute
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool g_wg_attr_set[kMaxDevices] = {};
-
-// Launch one weight-streaming product for query rows [q0, q0 + n), K split in
-// chunks whose bf16 X slice fits the kernel's staging buffer.
-mla_status_t launch_wgemm(wg::Params p, const CUtensorMap& tw, int m_tiles, int heads,
-                          cudaStream_t st) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return MLA_ERR_CUDA;
-  if (!g_wg_attr_set[dev]) {
+// Launch one weight-streaming product, one launch per 128 query rows.  The
+// weight is walked in units of 128 rows x 64 K; `split_k` lets a CTA's run of
+// units start and end inside an m-tile (the output product, which adds into a
+// zeroed `out`), otherwise runs are whole m-tiles.  `x_bf16` (absorb) is the
+// bf16 activation matrix [n_total, x_cols] read by TMA.
+mla_status_t launch_wgemm(wg::Params p, const CUtensorMap& tw, int groups, int m_tiles, int K,
+                          bool split_k, const void* x_bf16, uint64_t x_cols, cudaStream_t st) {
+  DeviceInfo* d = nullptr;
+  if (device_info(&d) != MLA_OK) return MLA_ERR_CUDA;
+  if (!d->wg_attr_set) {
     if (cudaFuncSetAttribute(wg::wgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             wg::kSmemBytes) != cudaSuccess)
+                             wg::kSmemMax) != cudaSuccess)
       return MLA_ERR_CUDA;
-    g_wg_attr_set[dev] = true;
+    d->wg_attr_set = true;
   }
+  p.groups = groups;
+  p.m_tiles = m_tiles;
+  p.k_stages = K / wg::kKP;
+  const int units = groups * m_tiles * p.k_stages;
+  int grid, chunk;
+  if (split_k) {
+    grid = std::min(d->num_sms, units);
+    chunk = (units + grid - 1) / grid;
+    grid = (units + chunk - 1) / chunk;
+  } else {
+    const int tiles = groups * m_tiles;
+    grid = std::min(d->num_sms, tiles);
+    const int per = (tiles + grid - 1) / grid;
+    chunk = per * p.k_stages;
+    grid = (tiles + per - 1) / per;
+  }
+  p.chunk = chunk;
+  float* zero = p.zero;
   const int total_n = p.n;
   for (int q0 = 0; q0 < total_n; q0 += 128) {
     p.q0 = q0;
-    p.n = min(128, total_n - q0);
+    p.n = std::min(128, total_n - q0);
     p.n_pad = (p.n + 15) / 16 * 16;
-    int kc = wg::kXBytesMax / (p.n_pad * 2);
-    kc = max(wg::kKP, kc / wg::kKP * wg::kKP);
-    p.k_chunk = min(p.K, kc);
-    dim3 grid(m_tiles, heads, (p.K + p.k_chunk - 1) / p.k_chunk);
-    wg::wgemm_kernel<<<grid, wg::kThreads, wg::kSmemBytes, st>>>(p, tw);
+    const int stage_bytes = wg::kWStage + p.n_pad * 128;
+    p.stages = std::min(wg::kMaxStages, (wg::kSmemMax - wg::kSmemFixed) / stage_bytes);
+    const int smem = p.stages * stage_bytes + wg::kSmemFixed;
+    p.zero = q0 == 0 ? zero : nullptr;
+    CUtensorMap tx;
+    std::memset(&tx, 0, sizeof(tx));
+    if (x_bf16 && !make_map_2d(&tx, x_bf16, x_cols, (uint64_t)p.n_total, (uint32_t)p.n_pad))
+      return MLA_ERR_CUDA;
+    wg::wgemm_kernel<<<grid, wg::kThreads, smem, st>>>(p, tw, tx);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
   }
   return MLA_OK;
@@ -218,30 +242,28 @@ mla_status_t mla_absorb_q(const mla_dims_t* dims, int32_t n_q, const void* q_nop
   a.w_uk = w_uk;
   a.q_abs = q_abs;
   cudaStream_t st0 = reinterpret_cast<cudaStream_t>(stream);
-  if (dims->dtype == MLA_BF16 && dims->d_c % wg::kMT == 0 && dims->d_n % wg::kKP == 0) {
+  if (dims->dtype == MLA_BF16 && dims->d_c % wg::kMT == 0 && dims->d_n % wg::kKP == 0 &&
+      aligned(q_nope, 16) && aligned(q_abs, 4)) {
     CUtensorMap tw;
     if (!make_map_2d(&tw, w_uk, dims->d_c, (uint64_t)dims->H * dims->d_n, 64)) return MLA_ERR_CUDA;
     wg::Params p{};
     p.mode = wg::kAbsorb;
     p.n = n_q;
     p.n_total = n_q;
-    p.K = dims->d_n;
     p.H = dims->H;
     p.d_c = dims->d_c;
     p.d_r = dims->d_r;
     p.d_n = dims->d_n;
     p.d_v = dims->d_v;
     p.d_model = dims->d_model;
-    p.x = q_nope;
-    p.x_row_stride = (long long)dims->H * dims->d_n;
-    p.x_head_stride = dims->d_n;
     p.out = q_abs;
     p.n_ver = n_ver;
     for (int i = 0; i < kMaxVersions; ++i) p.delta[i] = i < n_ver ? delta[i] : 0;
     p.rope_base = dims->rope_base;
     p.q_rope = q_rope;
     p.q_pos = q_pos;
-    return launch_wgemm(p, tw, dims->d_c / wg::kMT, dims->H, st0);
+    return launch_wgemm(p, tw, dims->H, dims->d_c / wg::kMT, dims->d_n, false, q_nope,
+                        (uint64_t)dims->H * dims->d_n, st0);
   }
   dim3 grid(dims->H, (n_q + kAbsQ - 1) / kAbsQ);
   const size_t smem = sizeof(float) * kAbsQ * dims->d_n;
@@ -397,19 +419,12 @@ mla_status_t mla_out_proj(const mla_dims_t* dims, int32_t n_q, const float* o_la
   const int H = dims->H, d_c = dims->d_c, d_v = dims->d_v;
   if (dims->dtype == MLA_BF16 && d_v % wg::kMT == 0 && d_c % wg::kKP == 0 &&
       (!w_o || dims->d_model % wg::kMT == 0) && aligned(o_lat, 16) && aligned(v, 16)) {
-    if (w_o) {
-      const long long n_out = (long long)n_q * dims->d_model;
-      const unsigned zb = (unsigned)std::min<long long>((n_out + 255) / 256, 4096);
-      wg::zero_kernel<<<zb, 256, 0, st>>>(out, n_out);
-      if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
-    }
     CUtensorMap tv;
     if (!make_map_2d(&tv, w_uv, d_c, (uint64_t)H * d_v, wg::kMT)) return MLA_ERR_CUDA;
     wg::Params p{};
     p.mode = wg::kValue;
     p.n = n_q;
     p.n_total = n_q;
-    p.K = d_c;
     p.H = H;
     p.d_c = d_c;
     p.d_r = dims->d_r;
@@ -420,18 +435,23 @@ mla_status_t mla_out_proj(const mla_dims_t* dims, int32_t n_q, const float* o_la
     p.x_row_stride = (long long)H * d_c;
     p.x_head_stride = d_c;
     p.out = v;
-    mla_status_t rc = launch_wgemm(p, tv, d_v / wg::kMT, H, st);
+    if (w_o) {   // the value launch zeroes `out` for the split-K output product
+      p.zero = out;
+      p.zero_n = (long long)n_q * dims->d_model;
+    }
+    mla_status_t rc = launch_wgemm(p, tv, H, d_v / wg::kMT, d_c, false, nullptr, 0, st);
     if (rc != MLA_OK || !w_o) return rc;
     CUtensorMap to;
     if (!make_map_2d(&to, w_o, (uint64_t)H * d_v, dims->d_model, wg::kMT)) return MLA_ERR_CUDA;
     p.mode = wg::kOutput;
     p.n = n_q;
-    p.K = H * d_v;
     p.x = v;
     p.x_row_stride = (long long)H * d_v;
     p.x_head_stride = 0;
     p.out = out;
-    return launch_wgemm(p, to, dims->d_model / wg::kMT, 1, st);
+    p.zero = nullptr;
+    p.zero_n = 0;
+    return launch_wgemm(p, to, 1, dims->d_model / wg::kMT, H * d_v, true, nullptr, 0, st);
   }
   dim3 g1(H, (d_v + 7) / 8);
   if (dims->dtype == MLA_BF16)

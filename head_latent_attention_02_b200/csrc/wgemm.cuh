@@ -9,14 +9,23 @@
 //   value   v[q, h, d] = sum_c W_UV[h][d][c] o_lat[q, h, c]
 //           ("Move the Value Expansion After the Weighted Sum");
 //   output  out[q, m] = sum_j W_O[m][j] v[q, j]  (the shared projection).
-// Each is computed transposed, D[m, n] = sum_k W[m, k] X[n, k], so the weight
-// rows fill the 128-row MMA tile and the query rows are the (padded) N
-// dimension.  One CTA owns 128 weight rows and a K range: its X slice is
-// converted to bf16 into shared memory once, the weight streams through a
-// 4-stage TMA ring, one thread issues tcgen05.mma (fp32 accumulator in TMEM),
-// and the epilogue writes D transposed.  The output product splits K over
-// CTAs and adds partial sums with fp32 atomics (the value kernel zeroes
-// `out` first).
+// Each is computed transposed, D[m, n] = sum_k W[m, k] X[n, k], so 128 weight
+// rows fill the MMA's M and the query rows are its (padded) N.
+//
+// The weight is cut into units of 128 rows x 64 K (16 KB, one TMA box); a
+// group (head) x m-tile x k-stage walk orders them with K fastest.  Each CTA
+// is persistent on one SM and takes a contiguous run of units -- whole
+// m-tiles for absorb/value (their outputs are written once), any run for the
+// output product (partial sums are added with fp32 atomics into `out`, which
+// the value launch zeroes).  Roles per CTA (320 threads):
+//   warp 0     TMA producer: weight stages (and the bf16 query panel of the
+//              absorb product) into a ring of up to 16 stages;
+//   warp 1     MMA issuer (one thread): tcgen05.mma into one of two TMEM
+//              accumulators, so the epilogue of one m-tile overlaps the next;
+//   warps 2-5  epilogue: TMEM -> registers -> global (stores or atomics);
+//   warps 6-9  convert the fp32 activation panel of each stage to bf16 in
+//              the 128-byte-swizzled K-major layout (value/output), or apply
+//              the rotary relocation (absorb).
 #pragma once
 #include <cuda.h>
 
@@ -26,29 +35,32 @@
 namespace mla {
 namespace wg {
 
-constexpr int kMT = 128;                 // weight rows per CTA
-constexpr int kKP = 64;                  // K per panel (128 B of bf16)
+constexpr int kMT = 128;                 // weight rows per unit (MMA M)
+constexpr int kKP = 64;                  // K per unit (one 128-byte panel)
 constexpr int kWStage = kMT * kKP * 2;   // 16 KB
-constexpr int kStages = 4;
-constexpr int kXBytesMax = 32 * 1024;    // bf16 X slice (N_pad rows x K range)
-constexpr int kSmemBytes = kStages * kWStage + kXBytesMax + 256 + 1024;
-constexpr int kThreads = 128;
+constexpr int kMaxStages = 16;
+constexpr int kSmemMax = 232448;         // dynamic shared memory per CTA
+constexpr int kSmemFixed = 512 + 1024;   // barriers + alignment slack
+constexpr int kThreads = 320;
 
 enum Mode : int { kAbsorb = 0, kValue = 1, kOutput = 2 };
 
 struct Params {
   int mode;
-  int n;          // query rows of this launch (q0 .. q0 + n - 1)
+  int n;          // query rows of this launch (q0 .. q0 + n - 1), <= 128
   int q0;         // first query row
   int n_total;    // query rows of the whole call (layout of q_abs)
-  int n_pad;      // n padded to a multiple of 16 (<= 128)
-  int K;          // reduction length of one product
-  int k_chunk;    // K range of one CTA (multiple of 64)
+  int n_pad;      // n padded to a multiple of 16
+  int stages;     // ring depth
+  int groups, m_tiles, k_stages;   // units = groups x m_tiles x k_stages
+  int chunk;      // units per CTA
   int H, d_c, d_r, d_n, d_v, d_model;
-  const void* x;  // activations: bf16 (absorb) or fp32
+  const void* x;  // activations: fp32 (value/output); absorb reads them by TMA
   long long x_row_stride;   // elements between query rows of X
-  long long x_head_stride;  // elements between heads of X
+  long long x_head_stride;  // elements between groups of X
   void* out;
+  float* zero;    // value: `out` of the following output product, zeroed here
+  long long zero_n;
   // absorb only
   int n_ver;
   int delta[kMaxVersions];
@@ -57,181 +69,265 @@ struct Params {
   const int32_t* q_pos;
 };
 
-// Weight tile: absorb reads W_UK[h] ([d_n rows, d_c cols], the M dimension
-// contiguous) as two 64-column boxes of 64 rows; the others read 128 weight
-// rows x 64 K as one box.  Both land in the canonical 128-byte-swizzled
-// layout the MMA descriptors below describe.
-__global__ void __launch_bounds__(kThreads) wgemm_kernel(const __grid_constant__ Params p,
-                                                         const __grid_constant__ CUtensorMap tw) {
+struct Unit {
+  int g, mt, ks;
+};
+__device__ __forceinline__ Unit unit_of(const Params& p, int u) {
+  Unit r;
+  r.ks = u % p.k_stages;
+  const int t = u / p.k_stages;
+  r.mt = t % p.m_tiles;
+  r.g = t / p.m_tiles;
+  return r;
+}
+
+__device__ __forceinline__ uint32_t acc_cols(int n_pad) {
+  return n_pad <= 32 ? 32u : (n_pad <= 64 ? 64u : 128u);
+}
+
+// Weight unit (128 rows x 64 K) in the canonical 128-byte-swizzled layout:
+// absorb reads W_UK[h] ([d_n, d_c], M contiguous) as two 64-row boxes of 64
+// M columns (M-major operand); the others read 128 rows x 64 K (K-major).
+__global__ void __launch_bounds__(kThreads, 1)
+wgemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tw,
+             const __grid_constant__ CUtensorMap tx) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int S = p.stages;
+  const int x_stage = p.n_pad * 128;
   uint8_t* sW = smem;
-  uint8_t* sX = smem + kStages * kWStage;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sX + kXBytesMax);
-  uint64_t* empty = full + kStages;
-  uint64_t* done = empty + kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint8_t* sX = smem + S * kWStage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sX + S * x_stage);
+  uint64_t* empty = full + kMaxStages;
+  uint64_t* acc_full = empty + kMaxStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kMT;           // first weight row (within a head)
-  const int h = blockIdx.y;                  // head (absorb / value), 0 for output
-  const int k0 = blockIdx.z * p.k_chunk;
-  const int kc = min(p.k_chunk, p.K - k0);
-  const int n_panels = kc / kKP;
-  const uint32_t ncols = p.n_pad <= 32 ? 32 : (p.n_pad <= 64 ? 64 : (p.n_pad <= 128 ? 128 : 256));
+  const bool absorb = p.mode == kAbsorb;
+  const uint32_t ncols = acc_cols(p.n_pad);
+  const int U = p.groups * p.m_tiles * p.k_stages;
+  const int u0 = min(U, (int)blockIdx.x * p.chunk);
+  const int u1 = min(U, u0 + p.chunk);
 
+  if (p.zero) {
+    for (long long i = (long long)blockIdx.x * kThreads + threadIdx.x; i < p.zero_n;
+         i += (long long)gridDim.x * kThreads)
+      p.zero[i] = 0.f;
+  }
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full[i], 1);
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], absorb ? 1 : 2);   // TMA bytes (+ the converter warp)
       mbar_init(&empty[i], 1);
     }
-    mbar_init(done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
     fence_mbar_init();
   }
-  if (warp == 0) tmem_alloc(tmem_slot, ncols);
+  if (warp == 1) tmem_alloc(tmem_slot, 2 * ncols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // weight ring: thread 0 starts the first loads before X is staged
-  auto load_w = [&](int i) {
-    const int s = i % kStages;
-    uint8_t* dst = sW + s * kWStage;
-    mbar_arrive_expect_tx(&full[s], kWStage);
-    const int kk = k0 + i * kKP;
-    if (p.mode == kAbsorb) {
-      // rows kk..kk+63 of W_UK[h] (global row h*d_n + kk), columns m0..m0+127
-      tma_load_2d(dst, &tw, &full[s], m0, h * p.d_n + kk);
-      tma_load_2d(dst + kWStage / 2, &tw, &full[s], m0 + 64, h * p.d_n + kk);
-    } else {
-      const int row = (p.mode == kValue ? h * p.d_v : 0) + m0;
-      tma_load_2d(dst, &tw, &full[s], kk, row);
-    }
-  };
-  bool ok = true;
-  if (threadIdx.x == 0) {
-    prefetch_tmap(&tw);
-    for (int i = 0; i < kStages && i < n_panels; ++i) load_w(i);
-  }
-
-  // X slice -> bf16, K-major, 128-byte swizzle: panel j holds K [64 j, 64 j + 64)
-  // of all n_pad rows (rows >= n are zero)
-  const int chunks = p.n_pad * n_panels * 8;            // 16-byte chunks
-  for (int e = threadIdx.x; e < chunks; e += kThreads) {
-    const int c = e & 7;
-    const int r = (e >> 3) % p.n_pad;
-    const int j = (e >> 3) / p.n_pad;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (r < p.n) {
-      const long long base = (long long)(p.q0 + r) * p.x_row_stride + (long long)h * p.x_head_stride +
-                             k0 + j * kKP + c * 8;
-      if (p.mode == kAbsorb) {
-        val = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.x) + base);
-      } else {
-        const float* xf = static_cast<const float*>(p.x) + base;
-        const float4 a = *reinterpret_cast<const float4*>(xf);
-        const float4 b = *reinterpret_cast<const float4*>(xf + 4);
-        __nv_bfloat162 t0 = __floats2bfloat162_rn(a.x, a.y), t1 = __floats2bfloat162_rn(a.z, a.w);
-        __nv_bfloat162 t2 = __floats2bfloat162_rn(b.x, b.y), t3 = __floats2bfloat162_rn(b.z, b.w);
-        val = make_uint4(*reinterpret_cast<uint32_t*>(&t0), *reinterpret_cast<uint32_t*>(&t1),
-                         *reinterpret_cast<uint32_t*>(&t2), *reinterpret_cast<uint32_t*>(&t3));
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA
+    if (lane == 0) {
+      prefetch_tmap(&tw);
+      if (absorb) prefetch_tmap(&tx);
+      const uint32_t bytes = kWStage + (absorb ? x_stage : 0);
+      for (int u = u0, i = 0; u < u1; ++u, ++i) {
+        const int slot = i % S;
+        if (!mbar_wait(&empty[slot], ((i / S) & 1) ^ 1)) { set_status(MLA_ERR_TIMEOUT); break; }
+        const Unit w = unit_of(p, u);
+        uint8_t* dst = sW + slot * kWStage;
+        mbar_arrive_expect_tx(&full[slot], bytes);
+        if (absorb) {
+          // rows 64 ks .. +63 of W_UK[g] (global row g d_n + 64 ks), columns
+          // 128 mt .. +127; the query panel: q_nope[q0.., g, 64 ks .. +63]
+          const int row = w.g * p.d_n + w.ks * kKP;
+          tma_load_2d(dst, &tw, &full[slot], w.mt * kMT, row);
+          tma_load_2d(dst + kWStage / 2, &tw, &full[slot], w.mt * kMT + 64, row);
+          tma_load_2d(sX + slot * x_stage, &tx, &full[slot], row, p.q0);
+        } else {
+          const int row = (p.mode == kValue ? w.g * p.d_v : 0) + w.mt * kMT;
+          tma_load_2d(dst, &tw, &full[slot], w.ks * kKP, row);
+        }
       }
     }
-    *reinterpret_cast<uint4*>(sX + j * p.n_pad * 128 + r * 128 + ((c ^ (r & 7)) << 4)) = val;
-  }
-  fence_proxy_async();
-  __syncthreads();
-
-  if (threadIdx.x == 0) {
-    const uint32_t idesc = idesc_bf16_f32(kMT, p.n_pad, p.mode == kAbsorb, false);
-    for (int i = 0; i < n_panels && ok; ++i) {
-      const int s = i % kStages;
-      if (!mbar_wait(&full[s], (i / kStages) & 1)) { set_status(MLA_ERR_TIMEOUT); ok = false; break; }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kMT, p.n_pad, absorb, false);
+      int seg = 0;
+      for (int u = u0, i = 0; u < u1; ++u, ++i) {
+        const int ks = u % p.k_stages;
+        const bool first = ks == 0 || u == u0;
+        const bool last = ks == p.k_stages - 1 || u == u1 - 1;
+        const int ab = seg & 1;
+        if (first && !mbar_wait(&acc_empty[ab], ((seg >> 1) & 1) ^ 1)) {
+          set_status(MLA_ERR_TIMEOUT);
+          break;
+        }
+        const int slot = i % S;
+        if (!mbar_wait(&full[slot], (i / S) & 1)) { set_status(MLA_ERR_TIMEOUT); break; }
+        tc_fence_after();
+        const uint32_t wa = smem_u32(sW + slot * kWStage);
+        const uint32_t xb = smem_u32(sX + slot * x_stage);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          // absorb: W is M-major (two 64-column blocks 8 KB apart, 16 K rows
+          // = 2 KB per step); otherwise K-major (16 K = 32 bytes per step)
+          const uint64_t ad = absorb ? smem_desc_sw128(wa + k * 2048, kWStage / 2, 1024)
+                                     : smem_desc_sw128(wa + k * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(xb + k * 32, 16, 1024);
+          mma_bf16_ss(tmem + ab * ncols, ad, bd, idesc, (first && k == 0) ? 0u : 1u);
+        }
+        mma_commit(&empty[slot]);
+        if (last) {
+          mma_commit(&acc_full[ab]);
+          ++seg;
+        }
+      }
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3;
+    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+    int seg = 0;
+    for (int u = u0; u < u1; ++u) {
+      const int ks = u % p.k_stages;
+      if (!(ks == p.k_stages - 1 || u == u1 - 1)) continue;
+      const Unit w = unit_of(p, u);
+      const int ab = seg & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[ab], (seg >> 1) & 1))) {
+        if (lane == 0) set_status(MLA_ERR_TIMEOUT);
+        break;
+      }
       tc_fence_after();
-      const uint32_t wa = smem_u32(sW + s * kWStage);
-      const uint32_t xb = smem_u32(sX + i * p.n_pad * 128);
+      const int m = w.mt * kMT + quad * 32 + lane;     // weight row of this lane
+#pragma unroll 1
+      for (int c0 = 0; c0 < p.n_pad; c0 += 16) {
+        float d[16];
+        tmem_ld16(trow + ab * ncols + c0, d);
+        tmem_wait_ld();
+        const int nq = min(16, p.n - c0);
+        if (p.mode == kOutput) {
+          float* o = static_cast<float*>(p.out) + (size_t)(p.q0 + c0) * p.d_model + m;
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        // absorb: W tile is M-major (two 64-column blocks 8 KB apart, 16 K
-        // rows per step); otherwise K-major (16 K = 32 bytes per step)
-        const uint64_t ad = (p.mode == kAbsorb)
-                                ? smem_desc_sw128(wa + ks * 2048, kWStage / 2, 1024)
-                                : smem_desc_sw128(wa + ks * 32, 16, 1024);
-        const uint64_t bd = smem_desc_sw128(xb + ks * 32, 16, 1024);
-        mma_bf16_ss(tmem, ad, bd, idesc, (i | ks) ? 1u : 0u);
-      }
-      mma_commit(&empty[s]);
-      if (i + kStages < n_panels) {
-        if (!mbar_wait(&empty[s], (i / kStages) & 1)) { set_status(MLA_ERR_TIMEOUT); ok = false; break; }
-        load_w(i + kStages);
-      }
-    }
-    mma_commit(done);
-  }
-  __syncwarp();
-  const bool done_ok = __all_sync(0xffffffffu, mbar_wait(done, 0));
-  if (!done_ok && lane == 0) set_status(MLA_ERR_TIMEOUT);
-  tc_fence_after();
-
-  // epilogue: lane = weight row m0 + 32 warp + lane, columns = query rows
-  const int m = m0 + warp * 32 + lane;
-  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-  for (int c0 = 0; c0 < p.n_pad; c0 += 32) {
-    float d[32];
-    tmem_ld32(trow + c0, d);
-    tmem_wait_ld();
-    if (!done_ok) continue;
+          for (int i = 0; i < 16; ++i)
+            if (i < nq) atomicAdd(o + (size_t)i * p.d_model, d[i]);
+        } else if (p.mode == kValue) {
+          float* o = static_cast<float*>(p.out) + ((size_t)(p.q0 + c0) * p.H + w.g) * p.d_v + m;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      if (c0 + i >= p.n) continue;
-      const int q = p.q0 + c0 + i;
-      if (p.mode == kOutput) {
-        atomicAdd(static_cast<float*>(p.out) + (size_t)q * p.d_model + m, d[i]);
-      } else if (p.mode == kValue) {
-        static_cast<float*>(p.out)[((size_t)q * p.H + h) * p.d_v + m] = d[i];
-      } else {
-        const int row = p.d_c + p.d_r;
-        for (int v = 0; v < p.n_ver; ++v)
-          static_cast<__nv_bfloat16*>(p.out)[(((size_t)v * p.n_total + q) * p.H + h) * row + m] =
-              __float2bfloat16_rn(d[i]);
+          for (int i = 0; i < 16; ++i)
+            if (i < nq) o[(size_t)i * p.H * p.d_v] = d[i];
+        } else {
+          const int row = p.d_c + p.d_r;
+          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out);
+          for (int v = 0; v < p.n_ver; ++v) {
+            __nv_bfloat16* ov = o + (((size_t)v * p.n_total + p.q0 + c0) * p.H + w.g) * row + m;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (i < nq) ov[(size_t)i * p.H * row] = __float2bfloat16_rn(d[i]);
+          }
+        }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      ++seg;
     }
-  }
-
-  // absorb: the rotary part of this head, once (by the CTA with m0 == 0):
-  // pair i rotated by (q_pos - delta_v) * base^(-2i/d_r), angles in double
-  if (p.mode == kAbsorb && blockIdx.x == 0) {
+  } else if (!absorb) {
+    // ------------------------------------------------------------ X panels
+    // Stage i is converted by warp 6 + (i mod 4): rows q0 .. q0 + n_pad - 1
+    // (zero past n) x K [64 ks, +64) of group g, fp32 -> bf16, 16-byte chunk
+    // c of row r stored at chunk c ^ (r mod 8) of the row's 128 bytes.
+    const int cw = warp - 6;
+    const float* xf = static_cast<const float*>(p.x);
+    for (int u = u0, i = 0; u < u1; ++u, ++i) {
+      if ((i & 3) != cw) continue;
+      const int slot = i % S;
+      if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], ((i / S) & 1) ^ 1))) {
+        if (lane == 0) set_status(MLA_ERR_TIMEOUT);
+        break;
+      }
+      const Unit w = unit_of(p, u);
+      const float* src = xf + (long long)p.q0 * p.x_row_stride + (long long)w.g * p.x_head_stride +
+                         w.ks * kKP;
+      uint8_t* dst = sX + slot * x_stage;
+      for (int e0 = lane; e0 < p.n_pad * 8; e0 += 128) {
+        float4 lo[4], hi[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int e = e0 + 32 * j, r = e >> 3, c = e & 7;
+          lo[j] = hi[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (r < p.n) {
+            const float* s = src + (long long)r * p.x_row_stride + c * 8;
+            lo[j] = *reinterpret_cast<const float4*>(s);
+            hi[j] = *reinterpret_cast<const float4*>(s + 4);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int e = e0 + 32 * j, r = e >> 3, c = e & 7;
+          const __nv_bfloat162 t0 = __floats2bfloat162_rn(lo[j].x, lo[j].y);
+          const __nv_bfloat162 t1 = __floats2bfloat162_rn(lo[j].z, lo[j].w);
+          const __nv_bfloat162 t2 = __floats2bfloat162_rn(hi[j].x, hi[j].y);
+          const __nv_bfloat162 t3 = __floats2bfloat162_rn(hi[j].z, hi[j].w);
+          *reinterpret_cast<uint4*>(dst + r * 128 + ((c ^ (r & 7)) << 4)) =
+              make_uint4(*reinterpret_cast<const uint32_t*>(&t0),
+                         *reinterpret_cast<const uint32_t*>(&t1),
+                         *reinterpret_cast<const uint32_t*>(&t2),
+                         *reinterpret_cast<const uint32_t*>(&t3));
+        }
+      }
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full[slot]);
+    }
+  } else {
+    // ------------------------------------------------------------ rotary part
+    // Rows (q, h) of this launch are shared out over the CTAs; a warp takes
+    // one row at a time, a lane one rotary pair i, rotated by
+    // (q_pos - delta_v) * base^(-2i/d_r) with the angle in double.
+    const int cw = warp - 6;
+    const int rows = p.n * p.H;
+    const int per = (rows + gridDim.x - 1) / gridDim.x;
+    const int r0 = blockIdx.x * per, r1 = min(rows, r0 + per);
     const int half = p.d_r / 2, row = p.d_c + p.d_r;
     const __nv_bfloat16* qr = static_cast<const __nv_bfloat16*>(p.q_rope);
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-    for (int t = threadIdx.x; t < p.n * p.n_ver * half; t += kThreads) {
-      const int i = t % half, v = (t / half) % p.n_ver, q = p.q0 + t / (half * p.n_ver);
-      const double theta = pow(p.rope_base, -2.0 * i / p.d_r);
-      double sn, cs;
-      sincos((double)(p.q_pos[q] - p.delta[v]) * theta, &sn, &cs);
-      const size_t src = ((size_t)q * p.H + h) * p.d_r + 2 * i;
-      const double x0 = __bfloat162float(qr[src]), x1 = __bfloat162float(qr[src + 1]);
-      const size_t dst = (((size_t)v * p.n_total + q) * p.H + h) * row + p.d_c + 2 * i;
-      out[dst] = __float2bfloat16_rn((float)(x0 * cs - x1 * sn));
-      out[dst + 1] = __float2bfloat16_rn((float)(x0 * sn + x1 * cs));
+    for (int r = r0 + cw; r < r1; r += 4) {
+      const int q = p.q0 + r / p.H, h = r % p.H;
+      const int pos = p.q_pos[q];
+      for (int i = lane; i < half; i += 32) {
+        const double theta = pow(p.rope_base, -2.0 * i / p.d_r);
+        const size_t src = ((size_t)q * p.H + h) * p.d_r + 2 * i;
+        const double x0 = __bfloat162float(qr[src]), x1 = __bfloat162float(qr[src + 1]);
+        for (int v = 0; v < p.n_ver; ++v) {
+          double sn, cs;
+          sincos((double)(pos - p.delta[v]) * theta, &sn, &cs);
+          const size_t dst = (((size_t)v * p.n_total + q) * p.H + h) * row + p.d_c + 2 * i;
+          __nv_bfloat162 y;
+          y.x = __float2bfloat16_rn((float)(x0 * cs - x1 * sn));
+          y.y = __float2bfloat16_rn((float)(x0 * sn + x1 * cs));
+          *reinterpret_cast<__nv_bfloat162*>(out + dst) = y;
+        }
+      }
     }
   }
 
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, ncols);
+    tmem_dealloc(tmem, 2 * ncols);
   }
-}
-
-// out[q, :] = 0 before the split-K output product adds into it.
-__global__ void zero_kernel(float* out, long long n) {
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
-       i += (long long)gridDim.x * blockDim.x)
-    out[i] = 0.f;
 }
 
 }  // namespace wg
