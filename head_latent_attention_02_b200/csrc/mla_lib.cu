@@ -104,28 +104,40 @@ bool make_map_576(CUtensorMap* m, const void* base, uint64_t rows, int rank, uin
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 2-D bf16 map over a row-major [outer, inner] matrix, box {64, box_outer},
-// 128-byte swizzle.
-bool make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
-                 uint32_t box_outer) {
+// 3-D bf16 map over a row-major [rows, cols] matrix seen as (64-column
+// offset, row, 64-column panel), box {64, box_rows, box_panels}, 128-byte
+// swizzle: a box is box_panels panels of box_rows x 128 bytes, and each row of
+// it is 128 * box_panels contiguous bytes of the matrix.
+bool make_map_panels(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
+                     uint32_t box_rows, uint32_t box_panels) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
-  cuuint64_t strides[1] = {(cuuint64_t)inner * 2};
-  cuuint32_t box[2] = {64, box_outer};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+  cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)(cols / 64)};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, box_panels};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Launch one weight-streaming product, one launch per 128 query rows.  The
-// weight is walked in units of 128 rows x 64 K; `split_k` lets a CTA's run of
-// units start and end inside an m-tile (the output product, which adds into a
-// zeroed `out`), otherwise runs are whole m-tiles.  `x_bf16` (absorb) is the
-// bf16 activation matrix [n_total, x_cols] read by TMA.
-mla_status_t launch_wgemm(wg::Params p, const CUtensorMap& tw, int groups, int m_tiles, int K,
-                          bool split_k, const void* x_bf16, uint64_t x_cols, cudaStream_t st) {
+// Panels per weight unit: long contiguous row runs for the TMA engine, but
+// at least three ring stages in shared memory, and K a whole number of units.
+int wgemm_panels(int K, int n_pad) {
+  int P = n_pad <= 32 ? 4 : 2;
+  while (P > 1 && K % (wg::kKP * P) != 0) P /= 2;
+  return P;
+}
+
+// Launch one weight-streaming product, one launch per 128 query rows.  W is
+// the bf16 weight as a row-major [w_rows, w_cols] matrix (absorb: W_UK seen as
+// [H d_n, d_c], read M-major; otherwise [M rows, K cols]).  `split_k` lets a
+// CTA's run of units start and end inside an m-tile (the output product,
+// which adds into a zeroed `out`), otherwise runs are whole m-tiles.  `x_bf16`
+// (absorb) is the bf16 activation matrix [n_total, x_cols] read by TMA.
+mla_status_t launch_wgemm(wg::Params p, const void* w, uint64_t w_rows, uint64_t w_cols,
+                          int groups, int m_tiles, int K, bool split_k, const void* x_bf16,
+                          uint64_t x_cols, cudaStream_t st) {
   DeviceInfo* d = nullptr;
   if (device_info(&d) != MLA_OK) return MLA_ERR_CUDA;
   if (!d->wg_attr_set) {
@@ -134,36 +146,43 @@ mla_status_t launch_wgemm(wg::Params p, const CUtensorMap& tw, int groups, int m
       return MLA_ERR_CUDA;
     d->wg_attr_set = true;
   }
-  p.groups = groups;
-  p.m_tiles = m_tiles;
-  p.k_stages = K / wg::kKP;
-  const int units = groups * m_tiles * p.k_stages;
-  int grid, chunk;
-  if (split_k) {
-    grid = std::min(d->num_sms, units);
-    chunk = (units + grid - 1) / grid;
-    grid = (units + chunk - 1) / chunk;
-  } else {
-    const int tiles = groups * m_tiles;
-    grid = std::min(d->num_sms, tiles);
-    const int per = (tiles + grid - 1) / grid;
-    chunk = per * p.k_stages;
-    grid = (tiles + per - 1) / per;
-  }
-  p.chunk = chunk;
-  float* zero = p.zero;
+  const bool absorb = p.mode == wg::kAbsorb;
   const int total_n = p.n;
+  float* zero = p.zero;
   for (int q0 = 0; q0 < total_n; q0 += 128) {
     p.q0 = q0;
     p.n = std::min(128, total_n - q0);
     p.n_pad = (p.n + 15) / 16 * 16;
-    const int stage_bytes = wg::kWStage + p.n_pad * 128;
+    p.P = wgemm_panels(K, p.n_pad);
+    p.groups = groups;
+    p.m_tiles = m_tiles;
+    p.k_stages = K / (wg::kKP * p.P);
+    const int units = groups * m_tiles * p.k_stages;
+    int grid, chunk;
+    if (split_k) {
+      grid = std::min(d->num_sms, units);
+      chunk = (units + grid - 1) / grid;
+      grid = (units + chunk - 1) / chunk;
+    } else {
+      const int tiles = groups * m_tiles;
+      grid = std::min(d->num_sms, tiles);
+      const int per = (tiles + grid - 1) / grid;
+      chunk = per * p.k_stages;
+      grid = (tiles + per - 1) / per;
+    }
+    p.chunk = chunk;
+    const int stage_bytes = p.P * (wg::kWPanel + p.n_pad * 128);
     p.stages = std::min(wg::kMaxStages, (wg::kSmemMax - wg::kSmemFixed) / stage_bytes);
+    if (p.stages < 2) return MLA_ERR_UNSUPPORTED;
     const int smem = p.stages * stage_bytes + wg::kSmemFixed;
     p.zero = q0 == 0 ? zero : nullptr;
-    CUtensorMap tx;
+    CUtensorMap tw, tx;
     std::memset(&tx, 0, sizeof(tx));
-    if (x_bf16 && !make_map_2d(&tx, x_bf16, x_cols, (uint64_t)p.n_total, (uint32_t)p.n_pad))
+    if (!make_map_panels(&tw, w, w_cols, w_rows, absorb ? wg::kKP * p.P : wg::kMT,
+                         absorb ? 2 : p.P))
+      return MLA_ERR_CUDA;
+    if (x_bf16 && !make_map_panels(&tx, x_bf16, x_cols, (uint64_t)p.n_total, (uint32_t)p.n_pad,
+                                   (uint32_t)p.P))
       return MLA_ERR_CUDA;
     wg::wgemm_kernel<<<grid, wg::kThreads, smem, st>>>(p, tw, tx);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
@@ -244,8 +263,6 @@ mla_status_t mla_absorb_q(const mla_dims_t* dims, int32_t n_q, const void* q_nop
   cudaStream_t st0 = reinterpret_cast<cudaStream_t>(stream);
   if (dims->dtype == MLA_BF16 && dims->d_c % wg::kMT == 0 && dims->d_n % wg::kKP == 0 &&
       aligned(q_nope, 16) && aligned(q_abs, 4)) {
-    CUtensorMap tw;
-    if (!make_map_2d(&tw, w_uk, dims->d_c, (uint64_t)dims->H * dims->d_n, 64)) return MLA_ERR_CUDA;
     wg::Params p{};
     p.mode = wg::kAbsorb;
     p.n = n_q;
@@ -262,7 +279,8 @@ mla_status_t mla_absorb_q(const mla_dims_t* dims, int32_t n_q, const void* q_nop
     p.rope_base = dims->rope_base;
     p.q_rope = q_rope;
     p.q_pos = q_pos;
-    return launch_wgemm(p, tw, dims->H, dims->d_c / wg::kMT, dims->d_n, false, q_nope,
+    return launch_wgemm(p, w_uk, (uint64_t)dims->H * dims->d_n, dims->d_c, dims->H,
+                        dims->d_c / wg::kMT, dims->d_n, false, q_nope,
                         (uint64_t)dims->H * dims->d_n, st0);
   }
   dim3 grid(dims->H, (n_q + kAbsQ - 1) / kAbsQ);
@@ -419,8 +437,6 @@ mla_status_t mla_out_proj(const mla_dims_t* dims, int32_t n_q, const float* o_la
   const int H = dims->H, d_c = dims->d_c, d_v = dims->d_v;
   if (dims->dtype == MLA_BF16 && d_v % wg::kMT == 0 && d_c % wg::kKP == 0 &&
       (!w_o || dims->d_model % wg::kMT == 0) && aligned(o_lat, 16) && aligned(v, 16)) {
-    CUtensorMap tv;
-    if (!make_map_2d(&tv, w_uv, d_c, (uint64_t)H * d_v, wg::kMT)) return MLA_ERR_CUDA;
     wg::Params p{};
     p.mode = wg::kValue;
     p.n = n_q;
@@ -439,10 +455,9 @@ mla_status_t mla_out_proj(const mla_dims_t* dims, int32_t n_q, const float* o_la
       p.zero = out;
       p.zero_n = (long long)n_q * dims->d_model;
     }
-    mla_status_t rc = launch_wgemm(p, tv, H, d_v / wg::kMT, d_c, false, nullptr, 0, st);
+    mla_status_t rc = launch_wgemm(p, w_uv, (uint64_t)H * d_v, d_c, H, d_v / wg::kMT, d_c, false,
+                                   nullptr, 0, st);
     if (rc != MLA_OK || !w_o) return rc;
-    CUtensorMap to;
-    if (!make_map_2d(&to, w_o, (uint64_t)H * d_v, dims->d_model, wg::kMT)) return MLA_ERR_CUDA;
     p.mode = wg::kOutput;
     p.n = n_q;
     p.x = v;
@@ -451,7 +466,8 @@ mla_status_t mla_out_proj(const mla_dims_t* dims, int32_t n_q, const float* o_la
     p.out = out;
     p.zero = nullptr;
     p.zero_n = 0;
-    return launch_wgemm(p, to, 1, dims->d_model / wg::kMT, H * d_v, true, nullptr, 0, st);
+    return launch_wgemm(p, w_o, dims->d_model, (uint64_t)H * d_v, 1, dims->d_model / wg::kMT,
+                        H * d_v, true, nullptr, 0, st);
   }
   dim3 g1(H, (d_v + 7) / 8);
   if (dims->dtype == MLA_BF16)
