@@ -11,22 +11,23 @@
 // Decomposition.  A cluster of two CTAs on two SMs shares one tcgen05 MMA
 // (cta_group::2): CTA r holds the query rows of heads [64r, 64r + 64) and the
 // cache rows of page 2k + r of a 128-row tile; the pair computes the full
-// 128 x 128 score tile (as two N=64 MMAs over 32-row halves of the pages),
-// each CTA receiving its 64 head rows in TMEM (tokens 0-63 in lanes 0-63,
-// tokens 64-127 in lanes 64-127 of the same columns).  The softmax of a head
-// row is shared by lanes t and t + 64 (the row max is combined through
-// shared memory).  P . c runs as M=128 x N=256 pair MMAs over the two latent
-// halves; each CTA supplies the c columns of its N half for all 128 rows,
-// re-read through L2, and accumulates O for its 64 heads in 256 TMEM columns
-// (lanes 0-63: latent [0,128) and [256,384); lanes 64-127: [128,256) and
-// [384,512)).  No scores or probabilities cross between the SMs: only the
-// MMA operands do, inside the pair instruction.
+// 128 x 128 score tile (N=128 MMAs accumulated over two column stages of the
+// pages), each CTA receiving its 64 head rows in TMEM (tokens 0-63 in lanes
+// 0-63, tokens 64-127 in lanes 64-127 of the same columns).  The softmax of
+// a head row is shared by lanes t and t + 64 (the row max is combined
+// through shared memory).  P . c runs as M=128 x N=256 pair MMAs; in MMA nb
+// CTA r supplies latent columns [256 r + 128 nb, +128) for all 128 rows
+// (re-read through L2), so each CTA's value columns are one contiguous half
+// and O for its 64 heads lies in 256 TMEM columns with latent [0, 256) in
+// lanes 0-63 and [256, 512) in lanes 64-127.  No scores or probabilities
+// cross between the SMs: only the MMA operands do, inside the pair
+// instruction.
 //
 // Loads.  Full rows are fetched with multi-dimensional TMA boxes so that each
-// request covers contiguous row bytes: a score stage is one box of 32 cache
-// rows x all 9 64-column panels (36 KB, whole 1152-byte rows), a value stage
-// one box of 32 rows x this CTA's four latent panels (16 KB), Q one box of
-// 64 rows x 9 panels.  Partial pages and gathered rows use per-panel boxes of
+// request covers long contiguous row runs: a score stage is one box of 64
+// cache rows x 5 or 4 64-column panels (640/512-byte runs), a value stage
+// one box of 32 rows x this CTA's four latent panels (512-byte runs, 16 KB),
+// Q one box of 64 rows x 9 panels.  Partial pages and gathered rows use per-panel boxes of
 // power-of-two heights, and rows without data come from boxes placed past the
 // end of the cache, which the hardware fills with zeros.
 //
@@ -50,16 +51,22 @@ constexpr int kM = 128;                  // query rows of the pair
 constexpr int kMh = 64;                  // query rows per CTA
 constexpr int kT = 128;                  // cache rows per tile (two pages)
 constexpr int kPg = 64;                  // rows per page
-constexpr int kR = 32;                   // cache rows per load stage
+constexpr int kR = 32;                   // cache rows per value stage
 constexpr int kQPanels = 9;              // 8 latent + 1 rotary 64-column panels
 constexpr int kQPanel = kMh * 128;       // 64 rows x 128 B = 8 KB
 constexpr int kSPanel = kR * 128;        // 32 rows x 128 B = 4 KB
-constexpr int kKStage = kQPanels * kSPanel;   // 36 KB: 32 rows x 9 panels
+constexpr int kKPanel = kPg * 128;       // 64 rows x 128 B = 8 KB
+// Score stages split a page's rows by columns: stage 0 holds panels 0-4 and
+// stage 1 panels 5-8 of all 64 rows, so each score MMA spans the page (N=128
+// for the pair) and the two stages of a tile alternate between fixed slots.
+constexpr int kKSplit = 5;                              // panels in stage 0
+constexpr int kKStage0 = kKSplit * kKPanel;             // 40 KB
+constexpr int kKStage1 = (kQPanels - kKSplit) * kKPanel;  // 32 KB
 constexpr int kVStage = 4 * kSPanel;          // 16 KB: 32 rows x this CTA's 4 latent panels
 constexpr int kKStages = 2, kVStages = 3;
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kQPanels * kQPanel;
-constexpr int kOffV = kOffK + kKStages * kKStage;
+constexpr int kOffV = kOffK + kKStage0 + kKStage1;
 constexpr int kOffP = kOffV + kVStages * kVStage;
 constexpr int kPBuf = 2 * kQPanel;       // 64 rows x 128 tokens bf16 (two 64-token panels)
 constexpr int kOffMisc = kOffP + 2 * kPBuf;
@@ -71,10 +78,12 @@ constexpr int kThreads = 224;
 constexpr int kTmemCols = 512;
 constexpr int kColO = 0, kColS = 256;
 constexpr int kMinChunk = 2;
+constexpr int kPrefetchTiles = 2;        // tiles of own-page rows requested into L2 ahead
+constexpr int kFlagTiles = 256;          // per-tile issue flags precomputed in shared memory
 constexpr int kNumBoxHeights = 6;        // 32, 16, 8, 4, 2, 1 rows
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: lazy rescale margin
-constexpr size_t kSlotFloats = (size_t)kM * kDc + kM;   // partial: o rows + lse
+constexpr int kStoreCols = 32;           // fp32 columns per output store box (128 B)
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct PlanHeader {
@@ -83,14 +92,19 @@ struct PlanHeader {
 
 // TMA descriptors (all 64 columns wide, 128-byte swizzle):
 //   q   3-D (col, q_abs row, panel): 64 rows x 9 panels of one head block
-//   k   3-D (col, cache row, panel): 32 rows x 9 panels
-//   v   4-D (col, cache row, panel in group, group): 32 rows x 2 x 2 panels,
-//       panel p of group g covering latent columns 256 g + 64 p
+//   k0  3-D (col, cache row, panel): 64 rows x panels 0-4 (score stage 0)
+//   k1  3-D (col, cache row, panel): 64 rows x panels 5-8 (score stage 1)
+//   v   3-D (col, cache row, panel): 32 rows x 4 panels (one latent half)
 //   row 2-D (col, cache row): boxes of 32 >> i rows (i = 0..5) for partial
 //       pages, gathered rows and zero rows past the end of the cache
+// and two fp32 store maps (32 columns x 32 rows, 128-byte swizzle):
+//   o   3-D (col, head - h0, query row) over o_lat: heads past n_h are
+//       clipped by the map, so a store never reaches another head range
+//   part 2-D (col, slot row) over the split partials [2G x 128, 512]
 struct Maps {
-  CUtensorMap q, k, v;
+  CUtensorMap q, k0, k1, v;
   CUtensorMap row[kNumBoxHeights];
+  CUtensorMap o, part;
 };
 
 struct Params {
@@ -99,7 +113,8 @@ struct Params {
   int G;
   const PlanHeader* plan;
   const int* stream_off;
-  float* partial;
+  const int* pair_stream;  // stream holding the first unit of each pair's run
+  float* partial_lse;     // [2G x 128] (the rows live behind the part map)
   float scale_log2;
 };
 
@@ -173,6 +188,29 @@ __device__ __forceinline__ Tile describe(const DecodeArgs& a, int b, int k) {
   return t;
 }
 
+// Relocation version of tile k of sequence b, from the segment table alone
+// (no block-table read: the MMA issuer only needs to know when the query
+// panel changes).  0 if the tile lies in no segment, as in describe(): the
+// loader and the issuer must take the same query-reload decisions.
+__device__ __forceinline__ int tile_version(const DecodeArgs& a, int b, int k) {
+  const mla_seg_t* sg = a.segs + (size_t)b * a.max_segs;
+  if (a.gather_rows) {
+    const int r0 = a.gather_rows[(size_t)b * a.max_gather + k * kT];
+    for (int s = 0; s < a.max_segs; ++s)
+      if (r0 >= sg[s].row_begin && r0 < sg[s].row_end) return sg[s].q_version;
+    return 0;
+  }
+  int rem = k;
+  for (int s = 0; s < a.max_segs; ++s) {
+    const int len = sg[s].row_end - sg[s].row_begin;
+    if (len <= 0) continue;
+    const int nt = seg_tiles(len);
+    if (rem < nt) return sg[s].q_version;
+    rem -= nt;
+  }
+  return 0;
+}
+
 // rows of tile half i (tile rows [64 i, 64 i + 64)) that hold data
 __device__ __forceinline__ int half_rows(const Tile& t, int i) {
   if (t.gather) return max(0, min(kPg, t.n_rows - kPg * i));
@@ -189,19 +227,24 @@ __device__ __forceinline__ int stream_tiles(const Params& p, int s) {
   return p.stream_off[s + 1] - p.stream_off[s];
 }
 
+// The stream holding unit u: the last stream whose offset is <= u (streams
+// without tiles share their successor's offset, so this is never one).
+__device__ __forceinline__ int stream_of(const int* stream_off, int n_streams, int u, int lo) {
+  int hi = n_streams - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (stream_off[mid] <= u) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
 __device__ __forceinline__ bool walk_begin(const Params& p, int g, Walk& w) {
   const int U = p.plan->U, C = p.plan->C;
   const long long u0 = (long long)g * C;
   if (u0 >= U) return false;
   w.u = (int)u0;
   w.u1 = (int)min((long long)U, u0 + C);
-  int lo = 0, hi = p.plan->n_streams - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (p.stream_off[mid] <= w.u) lo = mid; else hi = mid - 1;
-  }
-  w.s = lo;
-  while (stream_tiles(p, w.s) == 0) ++w.s;
+  w.s = p.pair_stream[g];
   w.k = w.u - p.stream_off[w.s];
   return true;
 }
@@ -228,6 +271,19 @@ __device__ __forceinline__ StreamPos stream_pos(const Params& p, int s) {
   return r;
 }
 
+// Issue flags of unit u of a pair's run starting at u0: bit 0, the unit opens
+// a stream; bit 1, it needs another query panel (new stream or relocation
+// version).  The same decisions as the query loader's.
+__device__ __forceinline__ uint32_t unit_flags(const Params& p, int u, int u0, int s_lo) {
+  const int n_streams = p.plan->n_streams;
+  const int s = stream_of(p.stream_off, n_streams, u, s_lo);
+  const int ver = tile_version(p.a, stream_pos(p, s).b, u - p.stream_off[s]);
+  if (u == u0) return 3u;
+  const int sp = stream_of(p.stream_off, n_streams, u - 1, s_lo);
+  if (sp != s) return 3u;
+  return tile_version(p.a, stream_pos(p, sp).b, u - 1 - p.stream_off[sp]) != ver ? 2u : 0u;
+}
+
 // ----------------------------------------------------------------- barriers
 struct Bars {
   uint64_t kfull[kKStages], kempty[kKStages];
@@ -237,8 +293,10 @@ struct Bars {
   uint64_t p_full[2], p_empty[2];
   uint64_t o_done[2], o_free;       // o_done[t & 1]: P.c of tile t complete
   uint64_t mma_drain;
+  uint64_t k_started;               // this CTA's first query and score loads are issued
   uint64_t row_sync[2], l_sync;     // the 128 softmax threads of one CTA
   uint32_t tmem_base;
+  uint8_t tflags[kFlagTiles];       // unit_flags of the pair's tiles (runs <= kFlagTiles)
 };
 static_assert(sizeof(Bars) <= kBarBytes, "barrier block too large");
 
@@ -262,13 +320,16 @@ __device__ __forceinline__ void arrive_leader(uint64_t* bar, uint32_t rank) {
   else mbar_arrive_cluster_addr(mapa(smem_u32(bar), 0));
 }
 
-// Fill smem rows [r0, r0 + n) (pitch 128 B) of one 64-column panel from
-// cache rows starting at y, as power-of-two boxes.  A y at or past the end of
+// Fill smem rows [r0, r0 + n) (pitch 128 B, n <= 64) of one 64-column panel
+// from cache rows starting at y, as power-of-two boxes.  A y at or past the end of
 // the cache (oob) makes the hardware fill the rows with zeros, so rows
 // without data read as 0 in the P.c product without any generic-proxy store.
 __device__ __forceinline__ void load_rows(uint8_t* dst, const Maps& mp, uint32_t bar, int x,
                                           long long y, int r0, int n) {
   int r = r0;
+  for (; n - (r - r0) > kR; r += kR)   // n <= 64: at most one leading full box
+    tma_load_2d_pair(dst + r * 128, &mp.row[0], bar, x, (int)(y + (r - r0)));
+  n -= r - r0;
 #pragma unroll 1
   for (int hb = 0; hb < kNumBoxHeights; ++hb) {
     const int h = kR >> hb;
@@ -359,6 +420,7 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
     mbar_init(&bar->o_done[1], 1);
     mbar_init(&bar->o_free, 8);
     mbar_init(&bar->mma_drain, 1);
+    mbar_init(&bar->k_started, 1);
     mbar_init(&bar->row_sync[0], kM);
     mbar_init(&bar->row_sync[1], kM);
     mbar_init(&bar->l_sync, kM);
@@ -377,6 +439,12 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
   Walk w;
   const bool has_work = walk_begin(p, g, w);
   bool ok = true;
+  const int n_tiles = has_work ? w.u1 - w.u : 0;
+  if (warp == 1 && rank == 0 && n_tiles <= kFlagTiles) {
+    for (int i = lane; i < n_tiles; i += 32)
+      bar->tflags[i] = (uint8_t)unit_flags(p, w.u + i, w.u, w.s);
+    __syncwarp();
+  }
 
   if (warp == 0 || warp == 6) {
     // ------------------------------------------------------------ loads
@@ -387,7 +455,8 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
     int nk = 0, nv = 0, n_qload = 0, cur_s = -1, cur_v = -1;
     if (lane == 0) {
       prefetch_tmap(&mp.q);
-      prefetch_tmap(&mp.k);
+      prefetch_tmap(&mp.k0);
+      prefetch_tmap(&mp.k1);
       prefetch_tmap(&mp.v);
       for (int i = 0; i < kNumBoxHeights; ++i) prefetch_tmap(&mp.row[i]);
     }
@@ -401,26 +470,28 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
         tma_load_2d_pair(dst + i * 128, &mp.row[kNumBoxHeights - 1], fb, x, (int)phys);
       }
     };
-    // score stage j of tile t: rows [32 j, +32) of this CTA's page, 9 panels
+    // score stage j of tile t: all 64 rows of this CTA's page, panels
+    // [5 j, 5 j + 5) (stage 0) or [5, 9) (stage 1), in slot j
     auto load_k = [&](const Tile& t, int b, int j) -> bool {
-      const int slot = nk % kKStages;
-      if (!wait_warp(&bar->kempty[slot], ((nk / kKStages) & 1) ^ 1)) return false;
-      uint8_t* dst = sK + slot * kKStage;
-      const uint32_t fb = mapa(smem_u32(&bar->kfull[slot]), 0);
-      if (rank == 0 && lane == 0) mbar_arrive_expect_tx(&bar->kfull[slot], 2 * kKStage);
-      const int rows = max(0, min(kR, half_rows(t, (int)rank) - kR * j));
+      if (!wait_warp(&bar->kempty[j], ((nk / kKStages) & 1) ^ 1)) return false;
+      uint8_t* dst = sK + (j ? kKStage0 : 0);
+      const int p0 = j ? kKSplit : 0, p1 = j ? kQPanels : kKSplit;
+      const uint32_t fb = mapa(smem_u32(&bar->kfull[j]), 0);
+      if (rank == 0 && lane == 0)
+        mbar_arrive_expect_tx(&bar->kfull[j], 2 * (j ? kKStage1 : kKStage0));
+      const int rows = half_rows(t, (int)rank);
       if (t.gather) {
-        for (int pn = 0; pn < kQPanels; ++pn)
-          gather_panel(dst + pn * kSPanel, fb, b, t.g0 + kPg * (int)rank + kR * j, rows, 64 * pn);
+        for (int pn = p0; pn < p1; ++pn)
+          gather_panel(dst + (pn - p0) * kKPanel, fb, b, t.g0 + kPg * (int)rank, rows, 64 * pn);
       }
       if (lane == 0) {
-        if (!t.gather && rows == kR) {
-          tma_load_3d_pair(dst, &mp.k, fb, 0, (int)(half_phys(t, (int)rank) + kR * j), 0);
+        if (!t.gather && rows == kPg) {
+          tma_load_3d_pair(dst, j ? &mp.k1 : &mp.k0, fb, 0, (int)half_phys(t, (int)rank), p0);
         } else {
-          for (int pn = 0; pn < kQPanels; ++pn) {
+          for (int pn = p0; pn < p1; ++pn) {
             if (!t.gather)
-              load_rows(dst + pn * kSPanel, mp, fb, 64 * pn, half_phys(t, (int)rank) + kR * j, 0, rows);
-            load_rows(dst + pn * kSPanel, mp, fb, 64 * pn, y_oob, rows, kR - rows);
+              load_rows(dst + (pn - p0) * kKPanel, mp, fb, 64 * pn, half_phys(t, (int)rank), 0, rows);
+            load_rows(dst + (pn - p0) * kKPanel, mp, fb, 64 * pn, y_oob, rows, kPg - rows);
           }
         }
       }
@@ -429,7 +500,7 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
       return true;
     };
     // value stage kc of tile t: tile rows [32 kc, +32), this CTA's latent
-    // columns [256 g + 128 rank, +128) of both groups g (4 panels)
+    // columns [256 rank, +256) (4 panels)
     auto load_v = [&](const Tile& t, int b) -> bool {
       for (int kc = 0; kc < 4; ++kc) {
         const int slot = nv % kVStages;
@@ -442,14 +513,14 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
         if (t.gather) {
           for (int q = 0; q < 4; ++q)
             gather_panel(dst + q * kSPanel, fb, b, t.g0 + kR * kc, rows,
-                         256 * (q >> 1) + 128 * (int)rank + 64 * (q & 1));
+                         256 * (int)rank + 64 * q);
         }
         if (lane == 0) {
           if (!t.gather && rows == kR) {
-            tma_load_4d_pair(dst, &mp.v, fb, 0, (int)(half_phys(t, hi) + r0), 2 * (int)rank, 0);
+            tma_load_3d_pair(dst, &mp.v, fb, 0, (int)(half_phys(t, hi) + r0), 4 * (int)rank);
           } else {
             for (int q = 0; q < 4; ++q) {
-              const int x = 256 * (q >> 1) + 128 * (int)rank + 64 * (q & 1);
+              const int x = 256 * (int)rank + 64 * q;
               if (!t.gather) load_rows(dst + q * kSPanel, mp, fb, x, half_phys(t, hi) + r0, 0, rows);
               load_rows(dst + q * kSPanel, mp, fb, x, y_oob, rows, kR - rows);
             }
@@ -461,10 +532,19 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
       return true;
     };
     const bool vwarp = (warp == 6);
+    // L2 prefetch walker: the own-page rows of the next kPrefetchTiles tiles
+    // are requested into L2 while the ring is still full, so that the stage
+    // loads (and the peer's value loads of this page) hit L2.
+    Walk pw = w;
+    int n_tile = 0, n_pref = 1;
+    if (has_work) walk_next(p, pw);
     for (bool more = has_work; more && ok; more = (w.u < w.u1)) {
       const StreamPos sp = stream_pos(p, w.s);
       const Tile t = describe(a, sp.b, w.k);
       if (vwarp) {
+        // the first value loads queue behind the query and score loads, which
+        // the first MMAs need long before any value stage
+        if (n_tile++ == 0 && !wait_warp(&bar->k_started, 0)) { fail(ok); break; }
         if (!load_v(t, sp.b)) { fail(ok); break; }
         walk_next(p, w);
         continue;
@@ -484,6 +564,19 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
         cur_v = t.ver;
       }
       if (!load_k(t, sp.b, 0) || !load_k(t, sp.b, 1)) { fail(ok); break; }
+      if (n_tile == 0 && lane == 0) mbar_arrive(&bar->k_started);
+      for (; lane == 0 && n_pref <= n_tile + kPrefetchTiles && pw.u < pw.u1; ++n_pref) {
+        const Tile tp = describe(a, stream_pos(p, pw.s).b, pw.k);
+        const int rows = half_rows(tp, (int)rank);
+        if (!tp.gather && rows > 0) {
+          const int y = (int)half_phys(tp, (int)rank);
+          tma_prefetch_l2_3d(&mp.k0, 0, y, 0);
+          tma_prefetch_l2_3d(&mp.k1, 0, y, kKSplit);
+        }
+        walk_next(p, pw);
+      }
+      __syncwarp();
+      ++n_tile;
       walk_next(p, w);
     }
     // drain: every load issued here has landed before the CTA exits (the
@@ -502,9 +595,9 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA (rank 0)
     if (rank == 0 && lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(kM, 64, false, false);
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kM, 2 * kPg, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kM, 256, false, true);
-      int it = 0, nk = 0, nv = 0, n_q = 0, cur_s = -1, cur_v = -1, n_streams = 0;
+      int it = 0, nk = 0, nv = 0, n_q = 0, n_streams = 0;
       int prev_first = 0, prev_stream_idx = 0;
       auto issue_pv = [&](int t, int first, int stream_idx) -> bool {
         const int pb = t & 1;
@@ -537,51 +630,48 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
         mma_pair_commit_both(&bar->o_done[pb]);
         return true;
       };
-      for (bool more = has_work; more && ok; more = (w.u < w.u1)) {
-        const StreamPos sp = stream_pos(p, w.s);
-        const Tile t = describe(a, sp.b, w.k);
-        const bool first = (w.s != cur_s);
+      // per-tile flags: from shared memory, or computed here for long runs
+      auto flags_of = [&](int i) -> uint32_t {
+        return n_tiles <= kFlagTiles ? bar->tflags[i] : unit_flags(p, w.u + i, w.u, w.s);
+      };
+      uint32_t f = n_tiles > 0 ? flags_of(0) : 0u;
+      for (; it < n_tiles && ok; ++it) {
+        const bool first = f & 1u;
         if (first) ++n_streams;
-        if (first || t.ver != cur_v) {
+        if (f & 2u) {
           if (!mbar_wait(&bar->q_full, n_q & 1)) { fail(ok); break; }
           ++n_q;
-          cur_s = w.s;
-          cur_v = t.ver;
         }
         const int sb = it & 1;
         if (!mbar_wait_cluster(&bar->s_empty[sb], ((it >> 1) & 1) ^ 1)) { fail(ok); break; }
         tc_fence_after();
         const uint32_t qa = smem_u32(sQ);
+        // S (64 columns: page 0 rows in lanes 0-63, page 1 rows in lanes
+        // 64-127) accumulates over the two column stages of the tile
         for (int j = 0; j < 2 && ok; ++j) {
-          const int slot = nk % kKStages;
-          if (!mbar_wait(&bar->kfull[slot], (nk / kKStages) & 1)) { fail(ok); break; }
+          if (!mbar_wait(&bar->kfull[j], (nk / kKStages) & 1)) { fail(ok); break; }
           tc_fence_after();
-          const uint32_t kb = smem_u32(sK + slot * kKStage);
-          for (int pn = 0; pn < kQPanels; ++pn) {
+          const uint32_t kb = smem_u32(sK + (j ? kKStage0 : 0));
+          const int p0 = j ? kKSplit : 0, p1 = j ? kQPanels : kKSplit;
+          for (int pn = p0; pn < p1; ++pn) {
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
               const uint64_t ad = smem_desc_sw128(qa + pn * kQPanel + ks * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(kb + pn * kSPanel + ks * 32, 16, 1024);
-              mma_pair_bf16_ss(tmem + kColS + sb * 64 + 32 * j, ad, bd, idesc_qk,
-                               (pn | ks) ? 1u : 0u);
+              const uint64_t bd = smem_desc_sw128(kb + (pn - p0) * kKPanel + ks * 32, 16, 1024);
+              mma_pair_bf16_ss(tmem + kColS + sb * 64, ad, bd, idesc_qk, (pn | ks) ? 1u : 0u);
             }
           }
-          mma_pair_commit_both(&bar->kempty[slot]);
+          mma_pair_commit_both(&bar->kempty[j]);
           ++nk;
         }
         if (!ok) break;
         mma_pair_commit_both(&bar->s_full[sb]);
-        Walk nx = w;
-        walk_next(p, nx);
-        if (nx.u < nx.u1) {
-          const Tile tn = describe(a, stream_pos(p, nx.s).b, nx.k);
-          if (nx.s != w.s || tn.ver != t.ver) mma_pair_commit_both(&bar->q_empty);
-        }
+        const uint32_t fn = it + 1 < n_tiles ? flags_of(it + 1) : 0u;
+        if (fn & 2u) mma_pair_commit_both(&bar->q_empty);   // the next tile reloads Q
         if (it > 0 && !issue_pv(it - 1, prev_first, prev_stream_idx)) { fail(ok); break; }
         prev_first = first;
         prev_stream_idx = n_streams - 1;
-        ++it;
-        w = nx;
+        f = fn;
       }
       if (ok && it > 0 && !issue_pv(it - 1, prev_first, prev_stream_idx)) fail(ok);
       mma_pair_commit_own(&bar->mma_drain);
@@ -706,39 +796,51 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
       const bool empty = !(l_tot > 0.f);
       const float inv = empty ? 0.f : 1.f / l_tot;
       const float lse = empty ? -INFINITY : (m_run + log2f(l_tot)) * 0.6931471805599453f;
-      float* orow;
-      float* lse_ptr;
-      if (whole) {
-        const size_t r = (size_t)qi * a.H + a.h0 + hrow;
-        orow = a.o_lat + r * kDc;
-        lse_ptr = a.lse + r;
-      } else {
-        const int slot = 2 * g + ((off_s <= range_u0) ? 0 : 1);
-        float* sl = p.partial + (size_t)slot * kSlotFloats;
-        const int m = kMh * (int)rank + hl;
-        orow = sl + (size_t)m * kDc;
-        lse_ptr = sl + (size_t)kM * kDc + m;
-      }
+      // O rows go out through the P buffers (idle here: the last P.c is done
+      // and this warp writes no new P before the next tile's pass 2).  Each
+      // warp stages its own 32 rows x 32 columns per step in an 8 KB slice
+      // (two 4 KB halves, alternating) and lane 0 stores the box by TMA, so
+      // no cross-warp barrier is involved.
+      const int slot = 2 * g + ((off_s <= range_u0) ? 0 : 1);
+      const int row0 = kMh * (int)rank + 32 * (quad & 1);   // first head row of this warp
+      const bool store = !whole || sp.hb * kM + row0 < a.n_h;
 #pragma unroll 1
-      for (int c = 0; c < 256; c += 32) {
-        float ov[32];
+      for (int c = 0; c < 256; c += kStoreCols) {
+        const int k = c / kStoreCols;
+        uint8_t* stage = sP + quad * 8192 + (k & 1) * 4096;
+        if (k >= 2) {
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+        }
+        float ov[kStoreCols];
         tmem_ld32(trow + kColO + c, ov);
         tmem_wait_ld();
-        if (row_valid) {
-          const int lat = 256 * (c >> 7) + 128 * half + (c & 127);
 #pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(orow + lat + i) =
-                make_float4(ov[i] * inv, ov[i + 1] * inv, ov[i + 2] * inv, ov[i + 3] * inv);
+        for (int i = 0; i < kStoreCols; i += 4)
+          *reinterpret_cast<float4*>(stage + lane * 128 + (((i >> 2) ^ (lane & 7)) << 4)) =
+              make_float4(ov[i] * inv, ov[i + 1] * inv, ov[i + 2] * inv, ov[i + 3] * inv);
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0 && store) {
+          const int lat = 256 * half + c;
+          if (whole) tma_store_3d(&mp.o, stage, lat, sp.hb * kM + row0, qi);
+          else tma_store_2d(&mp.part, stage, lat, slot * kM + row0);
+          bulk_commit();
         }
       }
-      if (row_valid && half == 0) *lse_ptr = lse;
+      if (lane == 0) bulk_wait_read<0>();
+      __syncwarp();
+      if (row_valid && half == 0) {
+        if (whole) a.lse[(size_t)qi * a.H + a.h0 + hrow] = lse;
+        else p.partial_lse[(size_t)slot * kM + kMh * (int)rank + hl] = lse;
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) arrive_leader(&bar->o_free, rank);
     }
   }
 
+  if (warp >= 2 && warp < 6 && lane == 0) bulk_wait_all();   // epilogue stores have landed
   tc_fence_before();
   __syncthreads();
   cluster_sync();   // no CTA leaves while its peer may still touch its memory
@@ -752,7 +854,7 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
 // ----------------------------------------------------------------- planner
 // One CTA: per-sequence tile counts, validation, stream offsets, chunk size.
 __global__ void plan_kernel(DecodeArgs a, int n_hb, int G, PlanHeader* plan, int* stream_off,
-                            int* stream_bad) {
+                            int* stream_bad, int* pair_stream) {
   const int n_rt = a.s_q * n_hb;
   const int n_streams = a.B * n_rt;
   for (int b = threadIdx.x; b < a.B; b += blockDim.x) {
@@ -811,19 +913,28 @@ __global__ void plan_kernel(DecodeArgs a, int n_hb, int G, PlanHeader* plan, int
     plan->n_streams = n_streams;
     plan->C = max(kMinChunk, (acc + G - 1) / max(G, 1));
   }
+  __syncthreads();
+  // the stream holding each pair's first unit (walk start without a search)
+  const int U = plan->U, C = plan->C;
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    const long long u = (long long)g * C;
+    pair_stream[g] = u < U ? stream_of(stream_off, n_streams, (int)u, 0) : 0;
+  }
 }
 
 // ----------------------------------------------------------------- combine
-// grid (n_streams, kM / 8), a warp per query row.  Streams covered by one
-// pair were written directly; split streams are merged here by log-sum-exp;
+// grid (n_streams, kM / 4), a warp per query row.  Streams covered by one
+// pair were written directly; split streams are merged here by log-sum-exp
+// (all parts' loads are independent of one another, so they overlap);
 // streams without tiles get the empty result (NaN for an invalid sequence).
-__global__ void __launch_bounds__(256) combine_kernel(DecodeArgs a, int n_hb,
+__global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a, int n_hb,
                                                       const PlanHeader* plan,
                                                       const int* stream_off,
                                                       const int* stream_bad,
-                                                      const float* partial) {
+                                                      const float* partial,
+                                                      const float* partial_lse) {
   const int s = blockIdx.x;
-  const int m = blockIdx.y * 8 + (threadIdx.x >> 5);
+  const int m = blockIdx.y * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   const int hb = s % n_hb;
   const int qi = s / n_hb;
@@ -842,31 +953,40 @@ __global__ void __launch_bounds__(256) combine_kernel(DecodeArgs a, int n_hb,
   const int off = stream_off[s];
   const int g0 = off / C, g1 = (off + T - 1) / C;
   if (g0 == g1) return;   // one pair covered the stream and wrote it
+  auto slot_of = [&](int gg) { return 2 * gg + ((off <= gg * C) ? 0 : 1); };
   float lmax = -INFINITY;
-  for (int gg = g0; gg <= g1; ++gg) {
-    const int slot = 2 * gg + ((off <= gg * C) ? 0 : 1);
-    lmax = fmaxf(lmax, partial[(size_t)slot * kSlotFloats + (size_t)kM * kDc + m]);
-  }
-  float acc[kDc / 32];
+  for (int gg = g0 + lane; gg <= g1; gg += 32)
+    lmax = fmaxf(lmax, partial_lse[(size_t)slot_of(gg) * kM + m]);
 #pragma unroll
-  for (int i = 0; i < kDc / 32; ++i) acc[i] = 0.f;
+  for (int d = 16; d > 0; d >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, d));
+  float4 acc[kDc / 128];
+#pragma unroll
+  for (int i = 0; i < kDc / 128; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   float tot = 0.f;
   if (lmax != -INFINITY) {
+#pragma unroll 4
     for (int gg = g0; gg <= g1; ++gg) {
-      const int slot = 2 * gg + ((off <= gg * C) ? 0 : 1);
-      const float* sl = partial + (size_t)slot * kSlotFloats;
-      const float li = sl[(size_t)kM * kDc + m];
-      if (li == -INFINITY) continue;
-      const float wgt = __expf(li - lmax);
+      const int sl = slot_of(gg);
+      const float li = partial_lse[(size_t)sl * kM + m];
+      const float wgt = (li == -INFINITY) ? 0.f : __expf(li - lmax);
       tot += wgt;
-      const float* src = sl + (size_t)m * kDc;
+      const float4* src =
+          reinterpret_cast<const float4*>(partial + ((size_t)sl * kM + m) * kDc);
 #pragma unroll
-      for (int i = 0; i < kDc / 32; ++i) acc[i] = fmaf(wgt, src[lane + 32 * i], acc[i]);
+      for (int i = 0; i < kDc / 128; ++i) {
+        const float4 v = src[lane + 32 * i];
+        acc[i].x = fmaf(wgt, v.x, acc[i].x);
+        acc[i].y = fmaf(wgt, v.y, acc[i].y);
+        acc[i].z = fmaf(wgt, v.z, acc[i].z);
+        acc[i].w = fmaf(wgt, v.w, acc[i].w);
+      }
     }
   }
   const float inv = tot > 0.f ? 1.f / tot : 0.f;
+  float4* dst = reinterpret_cast<float4*>(o);
 #pragma unroll
-  for (int i = 0; i < kDc / 32; ++i) o[lane + 32 * i] = acc[i] * inv;
+  for (int i = 0; i < kDc / 128; ++i)
+    dst[lane + 32 * i] = make_float4(acc[i].x * inv, acc[i].y * inv, acc[i].z * inv, acc[i].w * inv);
   if (lane == 0) a.lse[orow] = tot > 0.f ? lmax + logf(tot) : -INFINITY;
 }
 

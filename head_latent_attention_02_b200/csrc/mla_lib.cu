@@ -82,14 +82,15 @@ EncodeTiledFn encode_fn() {
 
 // Tensor map over a [rows, 576] bf16 matrix (row pitch 1152 B) with 64-column
 // boxes and 128-byte swizzle.  rank 2: (col, row), box {64, h}.  rank 3:
-// (col, row, 64-column panel), box {64, h, 9}.  rank 4: (col, row, panel
+// (col, row, 64-column panel), box {64, h, panels}.  rank 4: (col, row, panel
 // within a 256-column group, group), box {64, h, 2, 2}.
-bool make_map_576(CUtensorMap* m, const void* base, uint64_t rows, int rank, uint32_t h) {
+bool make_map_576(CUtensorMap* m, const void* base, uint64_t rows, int rank, uint32_t h,
+                  uint32_t panels = 9) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[4] = {64, (cuuint64_t)rows, 9, 1};
   cuuint64_t strides[3] = {(cuuint64_t)tc::kRow * 2, 128, 0};
-  cuuint32_t box[4] = {64, h, 9, 1};
+  cuuint32_t box[4] = {64, h, panels, 1};
   if (rank == 2) dims[0] = tc::kRow;
   if (rank == 4) {
     dims[2] = 4;
@@ -101,6 +102,22 @@ bool make_map_576(CUtensorMap* m, const void* base, uint64_t rows, int rank, uin
   cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims,
             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp32 store map for decode outputs: (column, row[, plane]) over rows of 512
+// floats, box {32, 32[, 1]}, 128-byte swizzle.  rank 3: rows are heads
+// (extent n_rows) and planes are query rows (stride plane_stride floats).
+bool make_map_out(CUtensorMap* m, float* base, uint64_t n_rows, uint64_t n_planes,
+                  uint64_t plane_stride, int rank) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)tc::kDc, (cuuint64_t)n_rows, (cuuint64_t)n_planes};
+  cuuint64_t strides[2] = {(cuuint64_t)tc::kDc * 4, (cuuint64_t)plane_stride * 4};
+  cuuint32_t box[3] = {(cuuint32_t)tc::kStoreCols, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, (cuuint32_t)rank, base, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -191,7 +208,7 @@ mla_status_t launch_wgemm(wg::Params p, const void* w, uint64_t w_rows, uint64_t
 }
 
 struct WsLayout {
-  size_t off_plan, off_streams, off_bad, off_partial, total;
+  size_t off_plan, off_streams, off_bad, off_pairs, off_partial, off_plse, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -201,8 +218,11 @@ WsLayout ws_layout(int n_streams, int G) {
   w.off_plan = 0;
   w.off_streams = align256(sizeof(tc::PlanHeader));
   w.off_bad = w.off_streams + align256(sizeof(int) * (size_t)(n_streams + 1));
-  w.off_partial = w.off_bad + align256(sizeof(int) * (size_t)n_streams);
-  w.total = w.off_partial + sizeof(float) * tc::kSlotFloats * 2 * (size_t)G;
+  // split partials: two slots per CTA pair, 128 rows of o each, then their lse
+  w.off_pairs = w.off_bad + align256(sizeof(int) * (size_t)n_streams);
+  w.off_partial = w.off_pairs + align256(sizeof(int) * (size_t)G);
+  w.off_plse = w.off_partial + sizeof(float) * (size_t)tc::kDc * tc::kM * 2 * (size_t)G;
+  w.total = w.off_plse + sizeof(float) * (size_t)tc::kM * 2 * (size_t)G;
   return w;
 }
 
@@ -375,8 +395,9 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
   tc::Maps maps;
   const uint64_t cache_rows = (uint64_t)n_pages * kPage;
   if (!make_map_576(&maps.q, q_abs, (uint64_t)n_ver * B * s_q * dims->H, 3, tc::kMh) ||
-      !make_map_576(&maps.k, cache, cache_rows, 3, tc::kR) ||
-      !make_map_576(&maps.v, cache, cache_rows, 4, tc::kR))
+      !make_map_576(&maps.k0, cache, cache_rows, 3, tc::kPg, tc::kKSplit) ||
+      !make_map_576(&maps.k1, cache, cache_rows, 3, tc::kPg, tc::kQPanels - tc::kKSplit) ||
+      !make_map_576(&maps.v, cache, cache_rows, 3, tc::kR, 4))
     return MLA_ERR_CUDA;
   for (int i = 0; i < tc::kNumBoxHeights; ++i)
     if (!make_map_576(&maps.row[i], cache, cache_rows, 2, (uint32_t)(tc::kR >> i)))
@@ -392,9 +413,15 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
   tc::PlanHeader* plan = reinterpret_cast<tc::PlanHeader*>(ws + wl.off_plan);
   int* stream_off = reinterpret_cast<int*>(ws + wl.off_streams);
   int* stream_bad = reinterpret_cast<int*>(ws + wl.off_bad);
+  int* pair_stream = reinterpret_cast<int*>(ws + wl.off_pairs);
   float* partial = reinterpret_cast<float*>(ws + wl.off_partial);
+  float* partial_lse = reinterpret_cast<float*>(ws + wl.off_plse);
+  if (!make_map_out(&maps.o, o_lat + (size_t)h0 * tc::kDc, (uint64_t)n_h, (uint64_t)B * s_q,
+                    (uint64_t)dims->H * tc::kDc, 3) ||
+      !make_map_out(&maps.part, partial, (uint64_t)tc::kM * 2 * G, 1, 0, 2))
+    return MLA_ERR_CUDA;
 
-  tc::plan_kernel<<<1, 256, 0, st>>>(a, n_hb, G, plan, stream_off, stream_bad);
+  tc::plan_kernel<<<1, 256, 0, st>>>(a, n_hb, G, plan, stream_off, stream_bad, pair_stream);
   if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
 
   tc::Params p;
@@ -403,13 +430,14 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
   p.G = G;
   p.plan = plan;
   p.stream_off = stream_off;
-  p.partial = partial;
+  p.pair_stream = pair_stream;
+  p.partial_lse = partial_lse;
   p.scale_log2 = dims->scale * tc::kLog2e;
   tc::decode_tc_kernel<<<2 * G, tc::kThreads, tc::kSmemBytes, st>>>(p, maps);
   if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
 
-  tc::combine_kernel<<<dim3(n_streams, tc::kM / 8), 256, 0, st>>>(a, n_hb, plan, stream_off,
-                                                                  stream_bad, partial);
+  tc::combine_kernel<<<dim3(n_streams, tc::kM / 4), 128, 0, st>>>(
+      a, n_hb, plan, stream_off, stream_bad, partial, partial_lse);
   return launch_ok();
 }
 
