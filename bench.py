@@ -47,6 +47,24 @@ def _cache_bytes(wl, rows_per_seq):
     return int(sum(rows_per_seq)) * (wl.d_c + wl.d_r) * 2
 
 
+# ---------------------------------------------------------------- multi-rank
+def max_over_ranks(values, device, world):
+    """Element-wise max of per-rank times over all ranks: the job is as slow
+    as its slowest replica.  All ranks must call it (it is a collective)."""
+    import torch
+    if world == 1:
+        return [float(v) for v in values]
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(bytes_per_rank, world, ms_per_step):
+    """Whole-job GB/s when every rank streams its own batch (weak scaling)."""
+    return bytes_per_rank * world / (ms_per_step * 1e-3) / 1e9
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     """Samples SM clock and throttle reasons with NVML in a thread."""
@@ -236,17 +254,15 @@ def run_gpu(args):
     torch.cuda.synchronize(dev)
     ms_e2e = s2.elapsed_time(e2)
 
-    vals = torch.tensor([ms_total, ms_e2e], device=dev, dtype=torch.float64)
+    ms_total, ms_e2e = max_over_ranks([ms_total, ms_e2e], dev, world)
     if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
         dist.barrier()
-    ms_total, ms_e2e = vals.tolist()
 
     if rank == 0:
         peaks, src = _peaks()
         ms_step = ms_total / args.steps
-        value = cache_bytes * world / (ms_step * 1e-3) / 1e9
-        e2e_val = cache_bytes * world / (ms_e2e / args.steps * 1e-3) / 1e9
+        value = job_throughput(cache_bytes, world, ms_step)
+        e2e_val = job_throughput(cache_bytes, world, ms_e2e / args.steps)
         achieved = cache_bytes / (t_dec * 1e-3) / 1e9
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
