@@ -536,8 +536,11 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
     // are requested into L2 while the ring is still full, so that the stage
     // loads (and the peer's value loads of this page) hit L2.
     Walk pw = w;
-    int n_tile = 0, n_pref = 1;
-    if (has_work) walk_next(p, pw);
+    int n_tile = 0, n_pref = 2;      // the walker starts at the third tile
+    if (has_work) {
+      walk_next(p, pw);
+      walk_next(p, pw);
+    }
     for (bool more = has_work; more && ok; more = (w.u < w.u1)) {
       const StreamPos sp = stream_pos(p, w.s);
       const Tile t = describe(a, sp.b, w.k);
@@ -565,7 +568,10 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
       }
       if (!load_k(t, sp.b, 0) || !load_k(t, sp.b, 1)) { fail(ok); break; }
       if (n_tile == 0 && lane == 0) mbar_arrive(&bar->k_started);
-      for (; lane == 0 && n_pref <= n_tile + kPrefetchTiles && pw.u < pw.u1; ++n_pref) {
+      // (not before the second tile: at start every CTA's first query and
+      // score loads already fill HBM, and prefetches would only delay them)
+      for (; lane == 0 && n_tile > 0 && n_pref <= n_tile + kPrefetchTiles && pw.u < pw.u1;
+           ++n_pref) {
         const Tile tp = describe(a, stream_pos(p, pw.s).b, pw.k);
         const int rows = half_rows(tp, (int)rank);
         if (!tp.gather && rows > 0) {

@@ -31,6 +31,30 @@ struct DeviceInfo {
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
 
+// The tensor-core kernels take nearly all of an SM's shared memory.  The
+// small kernels between them ask for the same split of the unified L1/shared
+// storage, so consecutive launches never make an SM switch configuration.
+mla_status_t prefer_max_shared() {
+  const int carveout = cudaSharedmemCarveoutMaxShared;
+  const void* small[] = {
+      reinterpret_cast<const void*>(&tc::plan_kernel),
+      reinterpret_cast<const void*>(&tc::combine_kernel),
+      reinterpret_cast<const void*>(&merge_lse_kernel),
+      reinterpret_cast<const void*>(&absorb_kernel<float>),
+      reinterpret_cast<const void*>(&absorb_kernel<__nv_bfloat16>),
+      reinterpret_cast<const void*>(&decode_simt_kernel<float>),
+      reinterpret_cast<const void*>(&decode_simt_kernel<__nv_bfloat16>),
+      reinterpret_cast<const void*>(&vproj_simt_kernel<float>),
+      reinterpret_cast<const void*>(&vproj_simt_kernel<__nv_bfloat16>),
+      reinterpret_cast<const void*>(&oproj_simt_kernel<float>),
+      reinterpret_cast<const void*>(&oproj_simt_kernel<__nv_bfloat16>)};
+  for (const void* f : small)
+    if (cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, carveout) !=
+        cudaSuccess)
+      return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
 mla_status_t device_info(DeviceInfo** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
@@ -39,6 +63,7 @@ mla_status_t device_info(DeviceInfo** out) {
   if (!d.ready) {
     if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return MLA_ERR_CUDA;
+    if (prefer_max_shared() != MLA_OK) return MLA_ERR_CUDA;
     d.ready = true;
   }
   *out = &d;
@@ -447,6 +472,8 @@ mla_status_t mla_merge_lse(int32_t n_q, int32_t H, int32_t h0, int32_t n_h, int3
   if (n_q < 0 || H < 1 || h0 < 0 || n_h < 1 || h0 + n_h > H || d < 1) return MLA_ERR_INVALID_ARG;
   if (n_q == 0) return MLA_OK;
   if (!o_a || !lse_a || !o_b || !lse_b || !o || !lse) return MLA_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  if (device_info(&dev) != MLA_OK) return MLA_ERR_CUDA;
   const long long rows = (long long)n_q * n_h;
   const long long blocks = (rows + 7) / 8;
   if (blocks > INT32_MAX) return MLA_ERR_INVALID_ARG;
