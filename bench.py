@@ -60,6 +60,24 @@ def max_over_ranks(values, device, world):
     return t.tolist()
 
 
+def graph_kernel_count(graph, default):
+    """Kernel nodes in a captured torch CUDA graph (the launches of one
+    replay), or `default` if the graph cannot be inspected."""
+    try:
+        from cuda.bindings import runtime as rt
+        raw = rt.cudaGraph_t(init_value=int(graph.raw_cuda_graph()))
+        err, _, n = rt.cudaGraphGetNodes(raw, 0)
+        if err != rt.cudaError_t.cudaSuccess:
+            return default
+        err, nodes, n = rt.cudaGraphGetNodes(raw, n)
+        if err != rt.cudaError_t.cudaSuccess:
+            return default
+        kinds = [rt.cudaGraphNodeGetType(nd)[1] for nd in nodes[:n]]
+        return sum(1 for k in kinds if k == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel)
+    except Exception:
+        return default
+
+
 def job_throughput(bytes_per_rank, world, ms_per_step):
     """Whole-job GB/s when every rank streams its own batch (weak scaling)."""
     return bytes_per_rank * world / (ms_per_step * 1e-3) / 1e9
@@ -172,13 +190,16 @@ def run_gpu(args):
     # One CUDA graph per cache copy holds a whole step (6 kernels), so the
     # timed loop measures the device, not Python's launch overhead.
     def capture(fn):
-        g = torch.cuda.CUDAGraph()
+        g = torch.cuda.CUDAGraph(keep_graph=True)   # keep_graph: nodes stay countable
         with torch.cuda.graph(g):
             fn()
+        g.instantiate()
         return g
 
     g_step = [capture(lambda c=c: step(c)) for c in range(N_COPIES)]
     g_dec = [capture(lambda c=c: decode_only(c)) for c in range(N_COPIES)]
+    kernels_per_step = graph_kernel_count(g_step[0], 6)
+    kernels_per_decode = graph_kernel_count(g_dec[0], 3)
     g_abs = capture(lambda: mla.absorb_q(p.dims, p.q_nope, p.q_rope, p.q_pos, p.deltas,
                                          p.w_uk, p.q_abs))
     g_out = capture(lambda: mla.out_proj(p.dims, p.o_lat, p.w_uv, p.w_o, p.v, p.out))
@@ -280,7 +301,8 @@ def run_gpu(args):
             "breakdown_us": {"absorb_q": round(t_abs * 1e3, 2), "decode": round(t_dec * 1e3, 2),
                              "out_proj": round(t_out * 1e3, 2),
                              "how": "each call's own graph replayed back to back"},
-            "decode_only": {"us": round(t_dec * 1e3, 2), "GB_s": round(achieved, 1)},
+            "decode_only": {"us": round(t_dec * 1e3, 2), "GB_s": round(achieved, 1),
+                            "kernels": kernels_per_decode},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1),
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
@@ -289,9 +311,9 @@ def run_gpu(args):
             "clocks": clocks,
             "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": 6 * args.steps,
-            "gpu_launches_note": "per step: absorb 1, decode 3 (plan, attention, split merge), "
-                                 "W_UV 1, W_O 1",
+            "gpu_launches": kernels_per_step * args.steps,
+            "gpu_launches_note": f"{kernels_per_step} kernel nodes per step graph (absorb, "
+                                 "decode plan, attention, split merge, W_UV, W_O)",
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
