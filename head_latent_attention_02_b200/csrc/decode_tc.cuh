@@ -917,7 +917,25 @@ __global__ void plan_kernel(DecodeArgs a, int n_hb, int G, PlanHeader* plan, int
     plan->U = acc;
     plan->G = G;
     plan->n_streams = n_streams;
-    plan->C = max(kMinChunk, (acc + G - 1) / max(G, 1));
+    int C = max(kMinChunk, (acc + G - 1) / max(G, 1));
+    // When every stream has the same T tiles, a chunk that divides T (or is a
+    // multiple of it) never straddles two streams: no pair then pays a second
+    // epilogue and query reload.  Taken when it costs at most a quarter more
+    // tiles per pair than the even split.
+    const int T0 = n_streams > 0 ? stream_off[1] - stream_off[0] : 0;
+    bool uniform = T0 > 0;
+    for (int s = 1; s < n_streams && uniform; ++s) uniform = stream_off[s + 1] - stream_off[s] == T0;
+    if (uniform && G > 0) {
+      int Ca = 0;
+      if (n_streams > G) {
+        Ca = T0 * ((n_streams + G - 1) / G);
+      } else {
+        for (int parts = min(T0, G / n_streams); parts >= 1 && Ca == 0; --parts)
+          if (T0 % parts == 0) Ca = T0 / parts;
+      }
+      if (Ca >= kMinChunk && 4 * Ca <= 5 * C) C = Ca;
+    }
+    plan->C = C;
   }
   __syncthreads();
   // the stream holding each pair's first unit (walk start without a search)
