@@ -289,8 +289,10 @@ struct Bars {
   uint64_t kfull[kKStages], kempty[kKStages];
   uint64_t vfull[kVStages], vempty[kVStages];
   uint64_t q_full, q_empty;
-  uint64_t s_full[2], s_empty[2];
-  uint64_t p_full[2], p_empty[2];
+  uint64_t s_full[2], p_empty[2];
+  // softmax of tile t done (S read, P written) in both CTAs: one arrival per
+  // CTA, forwarded after the CTA's four softmax warps met on sm_local
+  uint64_t sp_done[2], sm_local[2];
   uint64_t o_done[2], o_free;       // o_done[t & 1]: P.c of tile t complete
   uint64_t mma_drain;
   uint64_t k_started;               // this CTA's first query and score loads are issued
@@ -412,8 +414,8 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
     mbar_init(&bar->q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar->s_full[i], 1);
-      mbar_init(&bar->s_empty[i], 8);
-      mbar_init(&bar->p_full[i], 8);
+      mbar_init(&bar->sp_done[i], 2);
+      mbar_init(&bar->sm_local[i], 4);
       mbar_init(&bar->p_empty[i], 1);
     }
     mbar_init(&bar->o_done[0], 1);
@@ -607,7 +609,7 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
       int prev_first = 0, prev_stream_idx = 0;
       auto issue_pv = [&](int t, int first, int stream_idx) -> bool {
         const int pb = t & 1;
-        if (!mbar_wait_cluster(&bar->p_full[pb], (t >> 1) & 1)) return false;
+        if (!mbar_wait_cluster(&bar->sp_done[pb], (t >> 1) & 1)) return false;
         if (first && stream_idx > 0 && !mbar_wait_cluster(&bar->o_free, (stream_idx - 1) & 1))
           return false;
         tc_fence_after();
@@ -649,7 +651,7 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
           ++n_q;
         }
         const int sb = it & 1;
-        if (!mbar_wait_cluster(&bar->s_empty[sb], ((it >> 1) & 1) ^ 1)) { fail(ok); break; }
+        if (!mbar_wait_cluster(&bar->sp_done[sb], ((it >> 1) & 1) ^ 1)) { fail(ok); break; }
         tc_fence_after();
         const uint32_t qa = smem_u32(sQ);
         // S (64 columns: page 0 rows in lanes 0-63, page 1 rows in lanes
@@ -778,9 +780,12 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
         tc_fence_before();
         fence_proxy_async();
         __syncwarp();
-        if (lane == 0) {
-          arrive_leader(&bar->s_empty[sb], rank);
-          arrive_leader(&bar->p_full[pb], rank);
+        if (lane == 0) mbar_arrive(&bar->sm_local[pb]);
+        // one arrival per CTA reaches the leader: the pair's MMA traffic
+        // shares the path a remote arrival takes, so fewer of them land sooner
+        if (quad == 0) {
+          if (!wait_warp(&bar->sm_local[pb], (it >> 1) & 1)) { fail(ok); break; }
+          if (lane == 0) arrive_leader(&bar->sp_done[pb], rank);
         }
         have_o = true;
         ++it;
