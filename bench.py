@@ -43,6 +43,36 @@ def _peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+DECODE_PROFILE = os.path.join(ROOT, "profiles", "decode_b16_4k.md")
+DECODE_SOURCES = ["head_latent_attention_02_b200/csrc/decode_tc.cuh",
+                  "head_latent_attention_02_b200/csrc/mla_lib.cu"]
+
+
+def _sources_sha1():
+    import hashlib
+    h = hashlib.sha1()
+    for rel in DECODE_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def decode_traffic():
+    """DRAM bytes of one decode call (plan + attention + split merge) from the
+    committed ncu summary, or None if the kernel sources changed since."""
+    try:
+        fields = {}
+        for line in open(DECODE_PROFILE):
+            if ":" in line and line.strip().startswith(("traffic_bytes", "sources_sha1")):
+                k, v = line.strip().split(":", 1)
+                fields[k.strip()] = v.strip().strip("`")
+        if fields.get("sources_sha1") != _sources_sha1():
+            return None
+        return int(fields["traffic_bytes"])
+    except Exception:
+        return None
+
+
 def _cache_bytes(wl, rows_per_seq):
     return int(sum(rows_per_seq)) * (wl.d_c + wl.d_r) * 2
 
@@ -305,7 +335,8 @@ def run_gpu(args):
                             "kernels": kernels_per_decode},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1),
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                         "frac": round(achieved / peaks["hbm_gbs"], 4),
+                         "traffic": decode_traffic(),
                          "kernel": "mla_decode (plan + decode_tc + combine)",
                          "peak_source": src},
             "clocks": clocks,
