@@ -911,25 +911,56 @@ __global__ void plan_kernel(DecodeArgs a, int n_hb, int G, PlanHeader* plan, int
     }
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int s = 0; s < n_streams; ++s) {
-      const int c = stream_off[s];
-      stream_off[s] = acc;
-      acc += c;
+  // Exclusive prefix sum of the per-stream tile counts, one block-wide pass
+  // per blockDim.x streams (warp scans, then a scan of the warp totals), and
+  // whether every stream has the same count as stream 0.
+  __shared__ int warp_tot[32];
+  __shared__ int carry;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, n_warps = blockDim.x >> 5;
+  const int T0 = n_streams > 0 ? stream_off[0] : 0;
+  bool same = true;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < n_streams; base += blockDim.x) {
+    const int s = base + threadIdx.x;
+    const int c = s < n_streams ? stream_off[s] : 0;
+    if (s < n_streams) same = same && c == T0;
+    int x = c;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, d);
+      if (lane >= d) x += y;
     }
+    if (lane == 31) warp_tot[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+      int t = lane < n_warps ? warp_tot[lane] : 0;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, t, d);
+        if (lane >= d) t += y;
+      }
+      if (lane < n_warps) warp_tot[lane] = t;
+    }
+    __syncthreads();
+    const int incl = carry + (wid > 0 ? warp_tot[wid - 1] : 0) + x;
+    if (s < n_streams) stream_off[s] = incl - c;
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) carry = incl;
+    __syncthreads();
+  }
+  const bool uniform = __syncthreads_and(same) && T0 > 0;
+  if (threadIdx.x == 0) {
+    const int acc = carry;
     stream_off[n_streams] = acc;
     plan->U = acc;
     plan->G = G;
     plan->n_streams = n_streams;
     int C = max(kMinChunk, (acc + G - 1) / max(G, 1));
-    // When every stream has the same T tiles, a chunk that divides T (or is a
-    // multiple of it) never straddles two streams: no pair then pays a second
-    // epilogue and query reload.  Taken when it costs at most a quarter more
-    // tiles per pair than the even split.
-    const int T0 = n_streams > 0 ? stream_off[1] - stream_off[0] : 0;
-    bool uniform = T0 > 0;
-    for (int s = 1; s < n_streams && uniform; ++s) uniform = stream_off[s + 1] - stream_off[s] == T0;
+    // When every stream has the same T0 tiles, a chunk that divides T0 (or is
+    // a multiple of it) never straddles two streams: no pair then pays a
+    // second epilogue and query reload.  Taken when it costs at most a
+    // quarter more tiles per pair than the even split.
     if (uniform && G > 0) {
       int Ca = 0;
       if (n_streams > G) {

@@ -115,6 +115,33 @@ def test_bf16_head_counts(H):
     _check_all(inp, p, TOL["bf16"])
 
 
+@pytest.mark.parametrize("B,rows", [(100, 128), (16, 896), (32, 1024)])
+def test_bf16_equal_length_sequences(B, rows):
+    # equal tile counts per stream: more streams than CTA pairs (each pair
+    # takes whole streams), a prime tile count (7: no aligned chunk), and
+    # streams split into equal aligned parts
+    inp = make_inputs(_bf16(B=B, d_model=256, lengths=[rows] * B), seed=5)
+    p = _gpu(inp)
+    seqs = sorted({0, B // 2, B - 1})
+    o_ref, l_ref = O.decode_absorbed_fast(inp, seqs=seqs)
+    _cmp(p.o_lat.cpu().numpy()[seqs], o_ref[seqs], TOL["bf16"], "o_lat")
+    _cmp(p.lse.cpu().numpy()[seqs], l_ref[seqs], TOL["bf16"], "lse", lse=True)
+    assert np.isfinite(p.o_lat.cpu().numpy()).all()
+
+
+def test_bf16_many_short_sequences():
+    # more streams than one planner pass covers (300 > 256) with mixed
+    # lengths, including empty-ish single rows: exercises the carried prefix
+    lengths = [int(x) for x in np.random.default_rng(7).integers(1, 300, size=300)]
+    inp = make_inputs(_bf16(B=300, H=64, d_model=256, lengths=lengths), seed=6)
+    p = _gpu(inp)
+    seqs = [0, 1, 150, 257, 299]
+    o_ref, l_ref = O.decode_absorbed_fast(inp, seqs=seqs)
+    _cmp(p.o_lat.cpu().numpy()[seqs], o_ref[seqs], TOL["bf16"], "o_lat")
+    _cmp(p.lse.cpu().numpy()[seqs], l_ref[seqs], TOL["bf16"], "lse", lse=True)
+    assert np.isfinite(p.o_lat.cpu().numpy()).all()
+
+
 def test_bf16_two_query_tokens_causal():
     inp = make_inputs(_bf16(B=2, s_q=2, lengths=[700, 130]), seed=4)
     p = _gpu(inp)
