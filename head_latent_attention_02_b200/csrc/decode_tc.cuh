@@ -438,6 +438,9 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
 
+  // Launched as a programmatic dependent of the planner: everything above
+  // overlaps it; its plan and stream offsets are read only after this wait.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   Walk w;
   const bool has_work = walk_begin(p, g, w);
   bool ok = true;
@@ -852,6 +855,7 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
   }
 
   if (warp >= 2 && warp < 6 && lane == 0) bulk_wait_all();   // epilogue stores have landed
+  asm volatile("griddepcontrol.launch_dependents;");            // the merge may be scheduled
   tc_fence_before();
   __syncthreads();
   cluster_sync();   // no CTA leaves while its peer may still touch its memory
@@ -866,6 +870,8 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
 // One CTA: per-sequence tile counts, validation, stream offsets, chunk size.
 __global__ void plan_kernel(DecodeArgs a, int n_hb, int G, PlanHeader* plan, int* stream_off,
                             int* stream_bad, int* pair_stream) {
+  // let the decode kernel start its set-up now (it waits for our results)
+  asm volatile("griddepcontrol.launch_dependents;");
   const int n_rt = a.s_q * n_hb;
   const int n_streams = a.B * n_rt;
   for (int b = threadIdx.x; b < a.B; b += blockDim.x) {
@@ -993,6 +999,9 @@ __global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a, int n_hb,
                                                       const int* stream_bad,
                                                       const float* partial,
                                                       const float* partial_lse) {
+  // a programmatic dependent of the decode kernel: its outputs are complete
+  // and visible only after this wait
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int s = blockIdx.x;
   const int m = blockIdx.y * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;

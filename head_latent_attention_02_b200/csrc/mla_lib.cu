@@ -458,11 +458,29 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
   p.pair_stream = pair_stream;
   p.partial_lse = partial_lse;
   p.scale_log2 = dims->scale * tc::kLog2e;
-  tc::decode_tc_kernel<<<2 * G, tc::kThreads, tc::kSmemBytes, st>>>(p, maps);
-  if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  // The attention and merge kernels are programmatic dependents of the
+  // kernel before them: each may start its set-up early and waits on device
+  // (griddepcontrol.wait) before it reads its predecessor's results.
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * G);
+  cfg.blockDim = dim3(tc::kThreads);
+  cfg.dynamicSmemBytes = tc::kSmemBytes;
+  cfg.stream = st;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, tc::decode_tc_kernel, p, maps) != cudaSuccess) return MLA_ERR_CUDA;
 
-  tc::combine_kernel<<<dim3(n_streams, tc::kM / 4), 128, 0, st>>>(
-      a, n_hb, plan, stream_off, stream_bad, partial, partial_lse);
+  cfg.gridDim = dim3(n_streams, tc::kM / 4);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  if (cudaLaunchKernelEx(&cfg, tc::combine_kernel, a, n_hb, static_cast<const tc::PlanHeader*>(plan),
+                         static_cast<const int*>(stream_off), static_cast<const int*>(stream_bad),
+                         static_cast<const float*>(partial),
+                         static_cast<const float*>(partial_lse)) != cudaSuccess)
+    return MLA_ERR_CUDA;
   return launch_ok();
 }
 
