@@ -37,13 +37,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
-// Arrive on a barrier in another CTA of the cluster (address from mapa),
-// releasing this thread's prior writes at cluster scope.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
-               ::"r"(cluster_addr) : "memory");
-}
-
 // try_wait with a suspend-time hint: a waiting thread sleeps until the phase
 // completes (or ~1 ms passes) instead of spinning on issue slots that the
 // warps sharing its scheduler need.
@@ -109,21 +102,7 @@ __device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
   return out;
 }
 
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};"
-               ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
-}
-
 // ------------------------------------------------------------------ TMA
-__device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, uint64_t* bar,
-                                            int32_t x, int32_t y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cta.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];"
-      ::"r"(smem_u32(smem_dst)), "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, uint64_t* bar,
                                             int32_t x, int32_t y, int32_t z) {
   asm volatile(
@@ -178,9 +157,6 @@ __device__ __forceinline__ void fence_proxy_async() {
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                ::"r"(smem_u32(dst_smem)), "r"(ncols) : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
@@ -360,23 +336,9 @@ __device__ __forceinline__ void tma_load_3d_pair(void* smem_dst, const void* tma
       : "memory");
 }
 
-__device__ __forceinline__ void tma_load_4d_pair(void* smem_dst, const void* tmap,
-                                                 uint32_t bar_cluster, int32_t x, int32_t y,
-                                                 int32_t z, int32_t w) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5}], [%6];"
-      ::"r"(smem_u32(smem_dst)), "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar_cluster)
-      : "memory");
-}
-
 __device__ __forceinline__ void mbar_arrive_cluster_addr(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
                ::"r"(cluster_addr) : "memory");
 }
 
-// Named barrier among `count` threads (ids 1..15; 0 is __syncthreads).
-__device__ __forceinline__ void named_bar(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
 }  // namespace mla
