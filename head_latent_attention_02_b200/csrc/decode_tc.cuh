@@ -27,16 +27,20 @@
 // request covers long contiguous row runs: a score stage is one box of 64
 // cache rows x 5 or 4 64-column panels (640/512-byte runs), a value stage
 // one box of 32 rows x this CTA's four latent panels (512-byte runs, 16 KB),
-// Q one box of 64 rows x 9 panels.  Partial pages and gathered rows use per-panel boxes of
-// power-of-two heights, and rows without data come from boxes placed past the
-// end of the cache, which the hardware fills with zeros.
+// Q one box of 64 rows x 9 panels.  Partial pages and gathered rows use
+// per-panel boxes of power-of-two heights, and rows without data come from
+// boxes placed past the end of the cache, which the hardware fills with
+// zeros.  The own-page rows of the next two tiles are prefetched into L2.
 //
 // Roles per CTA (224 threads): warp 0 streams Q and the score stages, warp 6
-// the value stages (TMA), warp 1 of CTA 0 issues every MMA of the pair,
-// warps 2-5 own one TMEM lane each for softmax and the epilogue.  Work is split over CTA pairs
-// as contiguous runs of (sequence, head block, tile) units; a pair writes
-// the final result of a sequence it covers entirely, else a normalised
-// partial (o, lse) that the combine kernel merges.
+// the value stages (TMA), warp 1 of CTA 0 issues every MMA of the pair from
+// per-tile flags precomputed in shared memory, warps 2-5 own one TMEM lane
+// each for softmax and the epilogue (each CTA forwards one softmax-done
+// arrival per tile to the issuer).  Work is split over CTA pairs as
+// contiguous runs of (sequence, head block, tile) units -- runs that never
+// straddle two sequences when all have the same length; a pair writes the
+// final result of a sequence it covers entirely, else a normalised partial
+// (o, lse) that the combine kernel merges.
 #pragma once
 #include <cuda.h>
 
