@@ -226,8 +226,20 @@ mla_status_t launch_wgemm(wg::Params p, const void* w, uint64_t w_rows, uint64_t
     if (x_bf16 && !make_map_panels(&tx, x_bf16, x_cols, (uint64_t)p.n_total, (uint32_t)p.n_pad,
                                    (uint32_t)p.P))
       return MLA_ERR_CUDA;
-    wg::wgemm_kernel<<<grid, wg::kThreads, smem, st>>>(p, tw, tx);
-    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    // The split-K output product is a programmatic dependent of the value
+    // launch before it: its W_O stream starts at once, and only the threads
+    // that read v or add into `out` wait for the value launch on device.
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(wg::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = pdl;
+    cfg.numAttrs = split_k ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, wg::wgemm_kernel, p, tw, tx) != cudaSuccess) return MLA_ERR_CUDA;
   }
   return MLA_OK;
 }

@@ -118,6 +118,9 @@ wgemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorM
   const int u0 = min(U, (int)blockIdx.x * p.chunk);
   const int u1 = min(U, u0 + p.chunk);
 
+  // A launch that follows may start streaming its weights now; whatever it
+  // reads of this launch's results waits for completion (griddepcontrol.wait)
+  asm volatile("griddepcontrol.launch_dependents;");
   if (p.zero) {
     for (long long i = (long long)blockIdx.x * kThreads + threadIdx.x; i < p.zero_n;
          i += (long long)gridDim.x * kThreads)
@@ -203,6 +206,7 @@ wgemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorM
   } else if (warp < 6) {
     // ------------------------------------------------------------ epilogue
     const int quad = warp & 3;
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // `out` was zeroed by the value launch
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
     int seg = 0;
     for (int u = u0; u < u1; ++u) {
@@ -262,6 +266,9 @@ wgemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorM
     const int cw = warp - 6, pair = cw >> 1;
     const int t = (cw & 1) * 32 + lane;
     const float* xf = static_cast<const float*>(p.x);
+    // the activations are the previous launch's results (the output product
+    // is launched as its programmatic dependent; a no-op otherwise)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int per_panel = p.n_pad * 8;              // 16-byte chunks per panel
     const int total = per_panel * p.P;
     for (int u = u0, i = 0; u < u1; ++u, ++i) {
