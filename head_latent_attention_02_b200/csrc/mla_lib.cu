@@ -375,7 +375,11 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
   if (B == 0) return MLA_OK;
   if (!q_abs || !cache || !block_table || !segs || !q_pos || !o_lat || !lse)
     return MLA_ERR_INVALID_ARG;
+  // cache rows, logical rows and q_abs rows are 32-bit indices on the device
   if (n_pages * kPage + 2 * kPage > INT32_MAX) return MLA_ERR_UNSUPPORTED;
+  if ((long long)max_pages * kPage > INT32_MAX ||
+      (long long)n_ver * B * s_q * dims->H > INT32_MAX)
+    return MLA_ERR_UNSUPPORTED;
   const size_t es = elem_size(dims);
   if (!aligned(cache, 256) || !aligned(q_abs, 16) || !aligned(o_lat, 16) || !aligned(lse, 4))
     return MLA_ERR_INVALID_ARG;

@@ -158,7 +158,9 @@ mla_status_t mla_absorb_q(const mla_dims_t* dims, int32_t n_q, const void* q_nop
  * Rows past the end of a segment in its last page, and pages no table
  * references, may hold anything (NaN included) without affecting results.
  * Errors: INVALID_ARG (null/size/alignment), UNSUPPORTED (page_size != 64,
- * n_ver > 8), WORKSPACE (ws_bytes too small). */
+ * n_ver > 8, or n_pages * page_size, max_pages * page_size or
+ * n_ver * B * s_q * H beyond 2^31 - 1: device indices are 32-bit),
+ * WORKSPACE (ws_bytes too small). */
 mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const void* q_abs,
                         int32_t n_ver, int32_t h0, int32_t n_h, const void* cache,
                         int64_t n_pages, const int32_t* block_table, int32_t max_pages,

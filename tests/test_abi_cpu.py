@@ -67,6 +67,14 @@ def test_decode_rejects_bad_dims(L):
     assert _decode(_dims(), n_ver=9) == 2
 
 
+def test_decode_rejects_sizes_past_32_bit_indices(L):
+    # logical rows (max_pages x 64) and q_abs rows (n_ver x B x s_q x H) are
+    # 32-bit on the device: refused before anything is launched
+    assert _decode(_dims(), max_pages=1 << 26) == 2
+    assert _decode(_dims(), B=1 << 22, s_q=2, n_ver=2) == 2
+    assert _decode(_dims(), n_pages=1 << 25) == 2
+
+
 def test_decode_rejects_misaligned_cache(L):
     d = _dims()
     rc = mla.lib().mla_decode(ctypes.byref(d), 1, 1, FAKE, 1, 0, 128, FAKE + 16, 4, FAKE, 4,
