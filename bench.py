@@ -192,25 +192,32 @@ def run_gpu(args):
         dist.barrier()
     mla.lib()
 
-    wl = WORKLOADS[WORKLOAD]
+    wl = WORKLOADS[args.workload]
     inp = make_inputs(wl, seed=rank, poison=False)
-    p = runner.upload(inp, device=dev)
+    o_off = lse_off = None
+    if wl.n_local:
+        # the Local heads' offline (MLA-Off) partial is an input of the step:
+        # synthetic normalised rows and log-sum-exp values
+        g = np.random.default_rng([rank, 99])
+        o_off = g.standard_normal((inp.n_q, wl.H, wl.d_c)).astype(np.float32) * 0.1
+        lse_off = (g.standard_normal((inp.n_q, wl.H)) + 8.0).astype(np.float32)
+    p = runner.upload(inp, device=dev, head_order=inp.head_order, o_off=o_off, lse_off=lse_off)
     caches = [p.cache] + [p.cache.clone() for _ in range(N_COPIES - 1)]
     stream = torch.cuda.current_stream(dev)
-    cache_bytes = _cache_bytes(wl, inp.n_rows)
+    # cache rows the step reads: every sequence's rows, plus the protected
+    # rows the Local heads re-read
+    n_read = int(sum(inp.n_rows)) + (int(np.sum(inp.n_gather)) if inp.n_gather is not None else 0)
+    cache_bytes = n_read * (wl.d_c + wl.d_r) * 2
 
     def step(i, s=None):
         # s=None: the binding launches on torch's current stream (the capture
         # stream while a graph is being recorded)
         p.cache = caches[i % N_COPIES]
-        mla.absorb_q(p.dims, p.q_nope, p.q_rope, p.q_pos, p.deltas, p.w_uk, p.q_abs, s)
-        mla.decode(p.dims, p.B, p.s_q, p.q_abs, p.n_ver, 0, p.H, p.cache, p.block_table,
-                   p.segs, p.q_pos, p.o_lat, p.lse, p.workspace, stream=s)
-        mla.out_proj(p.dims, p.o_lat, p.w_uv, p.w_o, p.v, p.out, s)
+        runner.run_step(p, stream=s)
 
     def decode_only(i):
-        mla.decode(p.dims, p.B, p.s_q, p.q_abs, p.n_ver, 0, p.H, caches[i % N_COPIES],
-                   p.block_table, p.segs, p.q_pos, p.o_lat, p.lse, p.workspace)
+        p.cache = caches[i % N_COPIES]
+        runner.run_decode(p)
 
     for i in range(args.warmup):
         step(i, stream)
@@ -320,12 +327,17 @@ def run_gpu(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) latents/queries, N(0,1/fan_in) weights)",
-            "config": {"workload": WORKLOAD, "B": wl.B, "H": wl.H, "cached_rows": 4096,
+            "config": {"workload": args.workload, "B": wl.B, "H": wl.H,
+                       "cached_rows_total": int(sum(inp.n_rows)),
+                       "rows_per_sequence": (int(inp.n_rows[0]) if len(set(inp.n_rows)) == 1
+                                             else f"{min(inp.n_rows)}..{max(inp.n_rows)}"),
                        "d_c": wl.d_c, "d_r": wl.d_r, "d_n": wl.d_n, "d_v": wl.d_v,
                        "d_model": wl.d_model, "page": 64, "s_q": wl.s_q,
+                       "n_local_heads": wl.n_local,
                        "cache_bytes_per_step": cache_bytes,
-                       "l2": f"cache rotates over {N_COPIES} copies ({N_COPIES * cache_bytes / 1e6:.0f} MB)"
-                             " and each step streams W_O (235 MB): both exceed the 126 MB L2",
+                       "l2": f"cache rotates over {N_COPIES} copies "
+                             f"({N_COPIES * cache_bytes / 1e6:.0f} MB) and each step streams "
+                             f"W_O ({wl.d_model * wl.H * wl.d_v * 2 / 1e6:.0f} MB)",
                        "parallelism": f"replica x{world} (independent batches)"},
             "timing": "CUDA graph per step (6 kernels), CUDA events around the K replays",
             "breakdown_us": {"absorb_q": round(t_abs * 1e3, 2), "decode": round(t_dec * 1e3, 2),
@@ -336,8 +348,9 @@ def run_gpu(args):
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1),
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(achieved / peaks["hbm_gbs"], 4),
-                         "traffic": decode_traffic(),
-                         "kernel": "mla_decode (plan + decode_tc + combine)",
+                         "traffic": decode_traffic() if args.workload == WORKLOAD else None,
+                         "kernel": "decode calls of the step (plan + decode_tc + combine"
+                                   + (", twice, + merge_lse)" if wl.n_local else ")"),
                          "peak_source": src},
             "clocks": clocks,
             "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
@@ -346,7 +359,7 @@ def run_gpu(args):
             "gpu_launches_note": f"{kernels_per_step} kernel nodes per step graph (absorb, "
                                  "decode plan, attention, split merge, W_UV, W_O)",
         }
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD:
             line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -429,6 +442,9 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="bf16_b16_4k (default, the headline), bf16_varlen_b64, redknot_56_8, "
+                         "bf16_long_256k")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -113,6 +113,16 @@ def run_step(p: DeviceProblem, stream=None, out_proj: bool = True):
     """One pass of the hot path on ``stream``; results land in p.o_lat,
     p.lse, p.v and p.out."""
     mla.absorb_q(p.dims, p.q_nope, p.q_rope, p.q_pos, p.deltas, p.w_uk, p.q_abs, stream)
+    run_decode(p, stream)
+    if out_proj:
+        mla.out_proj(p.dims, p.o_lat, p.w_uv, p.w_o, p.v, p.out if p.w_o is not None else None,
+                     stream)
+
+
+def run_decode(p: DeviceProblem, stream=None):
+    """The attention part of a step (q_abs must be current): one decode call,
+    or for Local/Global head splits the Global decode, the Local gathered
+    decode and the offline/online merge."""
     if p.n_local:
         # Global heads: online over every row (prefix and relocated document)
         mla.decode(p.dims, p.B, p.s_q, p.q_abs, p.n_ver, p.n_local, p.H - p.n_local, p.cache,
@@ -127,6 +137,3 @@ def run_step(p: DeviceProblem, stream=None, out_proj: bool = True):
         mla.decode(p.dims, p.B, p.s_q, p.q_abs, p.n_ver, 0, p.H, p.cache, p.block_table, p.segs,
                    p.q_pos, p.o_lat, p.lse, p.workspace, gather_rows=p.gather_rows,
                    n_gather=p.n_gather, stream=stream)
-    if out_proj:
-        mla.out_proj(p.dims, p.o_lat, p.w_uv, p.w_o, p.v, p.out if p.w_o is not None else None,
-                     stream)
