@@ -82,6 +82,7 @@ constexpr int kThreads = 224;
 constexpr int kTmemCols = 512;
 constexpr int kColO = 0, kColS = 256;
 constexpr int kMinChunk = 2;
+constexpr int kPlanThreads = 1024;       // planner block (one CTA)
 constexpr int kPrefetchTiles = 2;        // tiles of own-page rows requested into L2 ahead
 constexpr int kFlagTiles = 256;          // per-tile issue flags precomputed in shared memory
 constexpr int kNumBoxHeights = 6;        // 32, 16, 8, 4, 2, 1 rows
@@ -140,9 +141,13 @@ __device__ __forceinline__ int seg_tiles(int len) {
   return (np + 1) / 2;
 }
 
+// kGather: the call attends gathered rows (gather_rows != null).  The kernels
+// are instantiated per mode, so the page-mode instantiation carries no code
+// for gathered rows.
+template <bool kGather>
 __device__ __forceinline__ Tile describe(const DecodeArgs& a, int b, int k) {
   Tile t;
-  t.gather = a.gather_rows != nullptr;
+  t.gather = kGather;
   t.ver = 0;
   t.g0 = 0;
   t.n_rows = 0;
@@ -150,7 +155,7 @@ __device__ __forceinline__ Tile describe(const DecodeArgs& a, int b, int k) {
   t.nv0 = t.nv1 = 0;
   t.kpos0 = t.kpos1 = 0;
   const mla_seg_t* sg = a.segs + (size_t)b * a.max_segs;
-  if (t.gather) {
+  if constexpr (kGather) {
     const int ng = a.n_gather[b];
     t.g0 = k * kT;
     t.n_rows = min(kT, ng - t.g0);
@@ -196,9 +201,10 @@ __device__ __forceinline__ Tile describe(const DecodeArgs& a, int b, int k) {
 // (no block-table read: the MMA issuer only needs to know when the query
 // panel changes).  0 if the tile lies in no segment, as in describe(): the
 // loader and the issuer must take the same query-reload decisions.
+template <bool kGather>
 __device__ __forceinline__ int tile_version(const DecodeArgs& a, int b, int k) {
   const mla_seg_t* sg = a.segs + (size_t)b * a.max_segs;
-  if (a.gather_rows) {
+  if constexpr (kGather) {
     const int r0 = a.gather_rows[(size_t)b * a.max_gather + k * kT];
     for (int s = 0; s < a.max_segs; ++s)
       if (r0 >= sg[s].row_begin && r0 < sg[s].row_end) return sg[s].q_version;
@@ -278,14 +284,16 @@ __device__ __forceinline__ StreamPos stream_pos(const Params& p, int s) {
 // Issue flags of unit u of a pair's run starting at u0: bit 0, the unit opens
 // a stream; bit 1, it needs another query panel (new stream or relocation
 // version).  The same decisions as the query loader's.
+template <bool kGather>
 __device__ __forceinline__ uint32_t unit_flags(const Params& p, int u, int u0, int s_lo) {
   const int n_streams = p.plan->n_streams;
   const int s = stream_of(p.stream_off, n_streams, u, s_lo);
-  const int ver = tile_version(p.a, stream_pos(p, s).b, u - p.stream_off[s]);
+  const int ver = tile_version<kGather>(p.a, stream_pos(p, s).b, u - p.stream_off[s]);
   if (u == u0) return 3u;
   const int sp = stream_of(p.stream_off, n_streams, u - 1, s_lo);
   if (sp != s) return 3u;
-  return tile_version(p.a, stream_pos(p, sp).b, u - 1 - p.stream_off[sp]) != ver ? 2u : 0u;
+  return tile_version<kGather>(p.a, stream_pos(p, sp).b, u - 1 - p.stream_off[sp]) != ver ? 2u
+                                                                                       : 0u;
 }
 
 // ----------------------------------------------------------------- barriers
@@ -346,27 +354,70 @@ __device__ __forceinline__ void load_rows(uint8_t* dst, const Maps& mp, uint32_t
   }
 }
 
+// Gathered rows i0 + 32 k (k < N; those at or past n are absent) of sequence
+// b: physical cache row (y_oob when absent or unlocatable) and request
+// position (INT32_MAX likewise).  Every index, segment and block-table load of
+// the N rows is issued before any result is used, so a lane pays about one
+// dependent-load latency per tile rather than one per row and panel.  The
+// planner has already checked that every gathered row of a live stream lies
+// in a segment; a bad page id records MLA_ERR_BAD_INDEX and reads as zeros.
+// Not inlined: only gathered tiles call it, and the loader loop of page tiles
+// stays as compact as it is without it.
+template <int N>
+__device__ __noinline__ void locate_gathered(const DecodeArgs& a, int b, int i0, int n,
+                                                long long y_oob, long long* phys, int* kpos) {
+  const mla_seg_t* sg = a.segs + (size_t)b * a.max_segs;
+  int row[N], seg[N], page[N];
+  bool in[N];
+#pragma unroll
+  for (int k = 0; k < N; ++k) {
+    row[k] = i0 + 32 * k < n ? a.gather_rows[(size_t)b * a.max_gather + i0 + 32 * k] : 0;
+    seg[k] = -1;
+  }
+  for (int s = 0; s < a.max_segs; ++s) {
+    const int rb = sg[s].row_begin, re = sg[s].row_end;
+#pragma unroll
+    for (int k = 0; k < N; ++k)
+      if (seg[k] < 0 && row[k] >= rb && row[k] < re) seg[k] = s;
+  }
+#pragma unroll
+  for (int k = 0; k < N; ++k) {
+    const bool present = i0 + 32 * k < n;
+    in[k] = present && seg[k] >= 0 && row[k] / kPage < a.max_pages;
+    page[k] = in[k] ? a.block_table[(size_t)b * a.max_pages + row[k] / kPage] : -1;
+    if (present && !in[k]) set_status(MLA_ERR_BAD_INDEX);
+  }
+#pragma unroll
+  for (int k = 0; k < N; ++k) {
+    phys[k] = y_oob;
+    kpos[k] = INT32_MAX;
+    if (in[k] && page[k] >= 0 && page[k] < a.n_pages) {
+      phys[k] = (long long)page[k] * kPage + row[k] % kPage;
+      kpos[k] = sg[seg[k]].key_pos_base + (row[k] - sg[seg[k]].row_begin);
+    } else if (in[k]) {
+      set_status(MLA_ERR_BAD_INDEX);
+    }
+  }
+}
+
 // Visibility of the 64 tile rows [64 half, +64) of tile t for a query at q_pos
 // qp, as a bitmask (bit i: row 64 half + i exists and key_pos <= qp).  Page
 // rows have consecutive key positions, so the mask is a prefix; gathered rows
-// are located one per lane and combined by ballot.
+// are located two per lane and combined by ballot.
 __device__ __noinline__ uint64_t gather_visible(const DecodeArgs& a, const Tile& t, int b, int half,
                                                int qp, int lane) {
-  const int nvh = half_rows(t, half);
-  const int i0 = t.g0 + kPg * half + lane;
-  int kp0 = INT32_MAX, kp1 = INT32_MAX;
-  long long ph;
-  int vv;
-  if (lane < nvh && !locate_row(a, b, i0, &ph, &kp0, &vv)) kp0 = INT32_MAX;
-  if (lane + 32 < nvh && !locate_row(a, b, i0 + 32, &ph, &kp1, &vv)) kp1 = INT32_MAX;
-  const uint32_t lo = __ballot_sync(0xffffffffu, kp0 <= qp);
-  const uint32_t hi = __ballot_sync(0xffffffffu, kp1 <= qp);
+  long long ph[2];
+  int kp[2];
+  locate_gathered<2>(a, b, t.g0 + kPg * half + lane, t.g0 + t.n_rows, 0, ph, kp);
+  const uint32_t lo = __ballot_sync(0xffffffffu, kp[0] <= qp);
+  const uint32_t hi = __ballot_sync(0xffffffffu, kp[1] <= qp);
   return (uint64_t)lo | ((uint64_t)hi << 32);
 }
 
+template <bool kGather>
 __device__ __forceinline__ uint64_t visible_rows(const DecodeArgs& a, const Tile& t, int b,
                                                  int half, int qp, int lane) {
-  if (t.gather) return gather_visible(a, t, b, half, qp, lane);
+  if constexpr (kGather) return gather_visible(a, t, b, half, qp, lane);
   const int n = min(half_rows(t, half), max(0, qp - half_kpos(t, half) + 1));
   return n >= 64 ? ~0ull : ((1ull << n) - 1ull);
 }
@@ -386,6 +437,7 @@ __device__ __noinline__ void scale_o(uint32_t taddr, float f) {
 }
 
 // ----------------------------------------------------------------- kernel
+template <bool kGather>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -451,7 +503,7 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
   const int n_tiles = has_work ? w.u1 - w.u : 0;
   if (warp == 1 && rank == 0 && n_tiles <= kFlagTiles) {
     for (int i = lane; i < n_tiles; i += 32)
-      bar->tflags[i] = (uint8_t)unit_flags(p, w.u + i, w.u, w.s);
+      bar->tflags[i] = (uint8_t)unit_flags<kGather>(p, w.u + i, w.u, w.s);
     __syncwarp();
   }
 
@@ -469,16 +521,17 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
       prefetch_tmap(&mp.v);
       for (int i = 0; i < kNumBoxHeights; ++i) prefetch_tmap(&mp.row[i]);
     }
-    // rows [r0, r0 + n) of one panel from gathered rows gi, gi+1, ... of
-    // sequence b (one box per row; rows that cannot be located read as zero)
-    auto gather_panel = [&](uint8_t* dst, uint32_t fb, int b, int gi, int n, int x) {
-      for (int i = lane; i < n; i += 32) {
-        long long phys;
-        int kp, vv;
-        if (!locate_row(a, b, gi + i, &phys, &kp, &vv)) phys = y_oob;
-        tma_load_2d_pair(dst + i * 128, &mp.row[kNumBoxHeights - 1], fb, x, (int)phys);
-      }
+    // rows [0, n) of one panel, row 32 k + lane from physical row ph[k] (one
+    // box per row; rows that could not be located are past the cache: zeros)
+    auto gather_panel = [&](uint8_t* dst, uint32_t fb, const long long* ph, int n, int x) {
+      for (int k = 0; 32 * k + lane < n; ++k)
+        tma_load_2d_pair(dst + (32 * k + lane) * 128, &mp.row[kNumBoxHeights - 1], fb, x,
+                         (int)ph[k]);
     };
+    // physical rows of the current gathered tile: the score loader's rows
+    // 64 rank + lane + 32 k (k < 2), the value loader's lane + 32 k (k < 4)
+    long long gph[4];
+    int gkp[4];
     // score stage j of tile t: all 64 rows of this CTA's page, panels
     // [5 j, 5 j + 5) (stage 0) or [5, 9) (stage 1), in slot j
     auto load_k = [&](const Tile& t, int b, int j) -> bool {
@@ -489,16 +542,16 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
       if (rank == 0 && lane == 0)
         mbar_arrive_expect_tx(&bar->kfull[j], 2 * (j ? kKStage1 : kKStage0));
       const int rows = half_rows(t, (int)rank);
-      if (t.gather) {
+      if constexpr (kGather) {
         for (int pn = p0; pn < p1; ++pn)
-          gather_panel(dst + (pn - p0) * kKPanel, fb, b, t.g0 + kPg * (int)rank, rows, 64 * pn);
+          gather_panel(dst + (pn - p0) * kKPanel, fb, gph, rows, 64 * pn);
       }
       if (lane == 0) {
-        if (!t.gather && rows == kPg) {
+        if (!kGather && rows == kPg) {
           tma_load_3d_pair(dst, j ? &mp.k1 : &mp.k0, fb, 0, (int)half_phys(t, (int)rank), p0);
         } else {
           for (int pn = p0; pn < p1; ++pn) {
-            if (!t.gather)
+            if (!kGather)
               load_rows(dst + (pn - p0) * kKPanel, mp, fb, 64 * pn, half_phys(t, (int)rank), 0, rows);
             load_rows(dst + (pn - p0) * kKPanel, mp, fb, 64 * pn, y_oob, rows, kPg - rows);
           }
@@ -519,18 +572,17 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
         if (rank == 0 && lane == 0) mbar_arrive_expect_tx(&bar->vfull[slot], 2 * kVStage);
         const int hi = kc >> 1, r0 = kR * (kc & 1);
         const int rows = max(0, min(kR, half_rows(t, hi) - r0));
-        if (t.gather) {
+        if constexpr (kGather) {
           for (int q = 0; q < 4; ++q)
-            gather_panel(dst + q * kSPanel, fb, b, t.g0 + kR * kc, rows,
-                         256 * (int)rank + 64 * q);
+            gather_panel(dst + q * kSPanel, fb, gph + kc, rows, 256 * (int)rank + 64 * q);
         }
         if (lane == 0) {
-          if (!t.gather && rows == kR) {
+          if (!kGather && rows == kR) {
             tma_load_3d_pair(dst, &mp.v, fb, 0, (int)(half_phys(t, hi) + r0), 4 * (int)rank);
           } else {
             for (int q = 0; q < 4; ++q) {
               const int x = 256 * (int)rank + 64 * q;
-              if (!t.gather) load_rows(dst + q * kSPanel, mp, fb, x, half_phys(t, hi) + r0, 0, rows);
+              if (!kGather) load_rows(dst + q * kSPanel, mp, fb, x, half_phys(t, hi) + r0, 0, rows);
               load_rows(dst + q * kSPanel, mp, fb, x, y_oob, rows, kR - rows);
             }
           }
@@ -552,11 +604,12 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
     }
     for (bool more = has_work; more && ok; more = (w.u < w.u1)) {
       const StreamPos sp = stream_pos(p, w.s);
-      const Tile t = describe(a, sp.b, w.k);
+      const Tile t = describe<kGather>(a, sp.b, w.k);
       if (vwarp) {
         // the first value loads queue behind the query and score loads, which
         // the first MMAs need long before any value stage
         if (n_tile++ == 0 && !wait_warp(&bar->k_started, 0)) { fail(ok); break; }
+        if constexpr (kGather) locate_gathered<4>(a, sp.b, t.g0 + lane, t.g0 + t.n_rows, y_oob, gph, gkp);
         if (!load_v(t, sp.b)) { fail(ok); break; }
         walk_next(p, w);
         continue;
@@ -575,15 +628,18 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
         cur_s = w.s;
         cur_v = t.ver;
       }
+      if constexpr (kGather)
+        locate_gathered<2>(a, sp.b, t.g0 + kPg * (int)rank + lane, t.g0 + t.n_rows, y_oob, gph,
+                           gkp);
       if (!load_k(t, sp.b, 0) || !load_k(t, sp.b, 1)) { fail(ok); break; }
       if (n_tile == 0 && lane == 0) mbar_arrive(&bar->k_started);
       // (not before the second tile: at start every CTA's first query and
       // score loads already fill HBM, and prefetches would only delay them)
       for (; lane == 0 && n_tile > 0 && n_pref <= n_tile + kPrefetchTiles && pw.u < pw.u1;
            ++n_pref) {
-        const Tile tp = describe(a, stream_pos(p, pw.s).b, pw.k);
+        const Tile tp = describe<kGather>(a, stream_pos(p, pw.s).b, pw.k);
         const int rows = half_rows(tp, (int)rank);
-        if (!tp.gather && rows > 0) {
+        if (!kGather && rows > 0) {
           const int y = (int)half_phys(tp, (int)rank);
           tma_prefetch_l2_3d(&mp.k0, 0, y, 0);
           tma_prefetch_l2_3d(&mp.k1, 0, y, kKSplit);
@@ -647,7 +703,8 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
       };
       // per-tile flags: from shared memory, or computed here for long runs
       auto flags_of = [&](int i) -> uint32_t {
-        return n_tiles <= kFlagTiles ? bar->tflags[i] : unit_flags(p, w.u + i, w.u, w.s);
+        return n_tiles <= kFlagTiles ? bar->tflags[i]
+                                     : unit_flags<kGather>(p, w.u + i, w.u, w.s);
       };
       uint32_t f = n_tiles > 0 ? flags_of(0) : 0u;
       for (; it < n_tiles && ok; ++it) {
@@ -717,9 +774,9 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
       float m_run = -INFINITY, l_run = 0.f;
       bool have_o = false;
       while (ok && w.u < w.u1 && w.s == s) {
-        const Tile tl = describe(a, sp.b, w.k);
+        const Tile tl = describe<kGather>(a, sp.b, w.k);
         const int sb = it & 1;
-        const uint64_t vis = visible_rows(a, tl, sp.b, half, qp, lane);
+        const uint64_t vis = visible_rows<kGather>(a, tl, sp.b, half, qp, lane);
         if (!wait_warp(&bar->s_full[sb], (it >> 1) & 1)) { fail(ok); break; }
         tc_fence_after();
         const uint32_t s_col = trow + kColS + sb * 64;
@@ -872,6 +929,7 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
 
 // ----------------------------------------------------------------- planner
 // One CTA: per-sequence tile counts, validation, stream offsets, chunk size.
+template <bool kGather>
 __global__ void plan_kernel(DecodeArgs a, int n_hb, int G, PlanHeader* plan, int* stream_off,
                             int* stream_bad, int* pair_stream) {
   // let the decode kernel start its set-up now (it waits for our results)
@@ -894,22 +952,10 @@ __global__ void plan_kernel(DecodeArgs a, int n_hb, int G, PlanHeader* plan, int
       prev_end = re;
       tiles += seg_tiles(re - rb);
     }
-    if (a.gather_rows && !bad) {
+    if (kGather && !bad) {
       const int ng = a.n_gather[b];
       if (ng < 0 || ng > a.max_gather) bad = true;
       tiles = bad ? 0 : (ng + kT - 1) / kT;
-      // the gathered rows of one tile must share one relocation version
-      for (int k = 0; !bad && k < tiles; ++k) {
-        int v0 = -1;
-        for (int i = k * kT; i < min(ng, k * kT + kT); ++i) {
-          const int r = a.gather_rows[(size_t)b * a.max_gather + i];
-          int v = -1;
-          for (int s = 0; s < a.max_segs; ++s)
-            if (r >= sg[s].row_begin && r < sg[s].row_end) { v = sg[s].q_version; break; }
-          if (v < 0 || (v0 >= 0 && v != v0)) { bad = true; break; }
-          v0 = v;
-        }
-      }
     }
     if (bad) {
       set_status(MLA_ERR_BAD_INDEX);
@@ -921,6 +967,39 @@ __global__ void plan_kernel(DecodeArgs a, int n_hb, int G, PlanHeader* plan, int
     }
   }
   __syncthreads();
+  if constexpr (kGather) {
+    // Every gathered row must lie in a segment, and the rows of one tile
+    // (entries [128 k, 128 k + 128)) in segments of one relocation version.
+    // One thread per entry, all sequences at once; a failing sequence is
+    // marked 2 in its first stream's flag, then every stream of it is
+    // emptied and flagged.
+    const long long n_entries = (long long)a.B * a.max_gather;
+    for (long long f = threadIdx.x; f < n_entries; f += blockDim.x) {
+      const int b = (int)(f / a.max_gather), i = (int)(f % a.max_gather);
+      const int ng = a.n_gather[b];
+      if (ng < 0 || ng > a.max_gather || i >= ng) continue;
+      const int32_t* gr = a.gather_rows + (size_t)b * a.max_gather;
+      const int r = gr[i], r0 = gr[i - i % kT];
+      const mla_seg_t* sg = a.segs + (size_t)b * a.max_segs;
+      int v = -1, v0 = -1;
+      for (int s = 0; s < a.max_segs; ++s) {
+        const int rb = sg[s].row_begin, re = sg[s].row_end, q = sg[s].q_version;
+        if (v < 0 && r >= rb && r < re) v = q;
+        if (v0 < 0 && r0 >= rb && r0 < re) v0 = q;
+      }
+      if (v < 0 || v != v0) stream_bad[b * n_rt] = 2;
+    }
+    __syncthreads();
+    for (int b = threadIdx.x; b < a.B; b += blockDim.x) {
+      if (stream_bad[b * n_rt] != 2) continue;
+      set_status(MLA_ERR_BAD_INDEX);
+      for (int r = 0; r < n_rt; ++r) {
+        stream_off[b * n_rt + r] = 0;
+        stream_bad[b * n_rt + r] = 1;
+      }
+    }
+    __syncthreads();
+  }
   // Exclusive prefix sum of the per-stream tile counts, one block-wide pass
   // per blockDim.x streams (warp scans, then a scan of the warp totals), and
   // whether every stream has the same count as stream 0.

@@ -37,7 +37,8 @@ std::mutex g_mu;
 mla_status_t prefer_max_shared() {
   const int carveout = cudaSharedmemCarveoutMaxShared;
   const void* small[] = {
-      reinterpret_cast<const void*>(&tc::plan_kernel),
+      reinterpret_cast<const void*>(&tc::plan_kernel<false>),
+      reinterpret_cast<const void*>(&tc::plan_kernel<true>),
       reinterpret_cast<const void*>(&tc::combine_kernel),
       reinterpret_cast<const void*>(&merge_lse_kernel),
       reinterpret_cast<const void*>(&absorb_kernel<float>),
@@ -445,11 +446,17 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
       return MLA_ERR_CUDA;
 
   if (!dev->tc_attr_set) {
-    if (cudaFuncSetAttribute(tc::decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(tc::decode_tc_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             tc::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(tc::decode_tc_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                              tc::kSmemBytes) != cudaSuccess)
       return MLA_ERR_CUDA;
     dev->tc_attr_set = true;
   }
+  // page mode and gathered-row mode are separate instantiations
+  const bool gather = gather_rows != nullptr;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   tc::PlanHeader* plan = reinterpret_cast<tc::PlanHeader*>(ws + wl.off_plan);
   int* stream_off = reinterpret_cast<int*>(ws + wl.off_streams);
@@ -462,7 +469,12 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
       !make_map_out(&maps.part, partial, (uint64_t)tc::kM * 2 * G, 1, 0, 2))
     return MLA_ERR_CUDA;
 
-  tc::plan_kernel<<<1, 256, 0, st>>>(a, n_hb, G, plan, stream_off, stream_bad, pair_stream);
+  if (gather)
+    tc::plan_kernel<true><<<1, tc::kPlanThreads, 0, st>>>(a, n_hb, G, plan, stream_off,
+                                                          stream_bad, pair_stream);
+  else
+    tc::plan_kernel<false><<<1, tc::kPlanThreads, 0, st>>>(a, n_hb, G, plan, stream_off,
+                                                           stream_bad, pair_stream);
   if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
 
   tc::Params p;
@@ -487,7 +499,9 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
   cfg.stream = st;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, tc::decode_tc_kernel, p, maps) != cudaSuccess) return MLA_ERR_CUDA;
+  if ((gather ? cudaLaunchKernelEx(&cfg, tc::decode_tc_kernel<true>, p, maps)
+              : cudaLaunchKernelEx(&cfg, tc::decode_tc_kernel<false>, p, maps)) != cudaSuccess)
+    return MLA_ERR_CUDA;
 
   cfg.gridDim = dim3(n_streams, tc::kM / 4);
   cfg.blockDim = dim3(128);

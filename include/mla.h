@@ -146,7 +146,11 @@ mla_status_t mla_absorb_q(const mla_dims_t* dims, int32_t n_q, const void* q_nop
  *   gather_rows   NULL, or [B, max_gather] logical rows to attend instead of
  *                 all segment rows ([RK]: protected token rows recomputed
  *                 online); n_gather [B] gives how many entries are used.
- *                 Every gathered row must lie in a segment.
+ *                 Every gathered row must lie in a segment, and the rows of
+ *                 each group of entries [128 k, 128 k + 128) in segments of
+ *                 one q_version (they share one query panel); a sequence
+ *                 that breaks either rule records BAD_INDEX and gets NaN
+ *                 o_lat and lse.
  *   q_pos         [B*s_q] request positions (int32)
  *   o_lat         [B*s_q, H, d_c] out (float): heads outside [h0, h0+n_h)
  *                 are not written

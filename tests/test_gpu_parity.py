@@ -57,6 +57,15 @@ def _gpu(inp, **kw):
     return p
 
 
+def _gpu_status(inp, code):
+    p = runner.upload(inp)
+    runner.run_step(p, out_proj=False)
+    torch.cuda.synchronize()
+    assert mla.get_status() == code
+    assert mla.get_status() == 0
+    return p
+
+
 def _oracle(inp, heads=None):
     o_lat, lse = O.decode_absorbed_fast(inp, heads=heads)
     return o_lat, lse
@@ -203,6 +212,34 @@ def test_empty_and_single_row_gathers():
     # one gathered row: the output is that row's latent exactly (weight 1)
     c5 = inp.pool[inp.block_table[0, 0], 5, :wl.d_c]
     assert np.array_equal(o[0], np.broadcast_to(c5, o[0].shape))
+
+
+def test_gathered_rows_validated_per_sequence():
+    # RedKnot layout: prefix rows 0-127 (version 0), document rows 128-383
+    # (version 1); 130 gathered document rows per sequence, i.e. two tiles
+    wl = Workload("gv", "bf16", B=3, H=128, d_model=256, prefix=128, doc=256, protected=130)
+    inp = make_inputs(wl, seed=9)
+    g = inp.gather_rows
+    g[0, 128:130] = [3, 4]     # second tile wholly in the prefix: valid
+    g[1, 5] = 7                # a prefix row inside a document tile: rejected
+    g[2, 129] = 5000           # a row outside every segment: rejected
+    p = _gpu_status(inp, 6)
+    o, l = p.o_lat.cpu().numpy(), p.lse.cpu().numpy()
+    assert np.isnan(o[1:]).all() and np.isnan(l[1:]).all()
+    o_ref, l_ref = O.decode_absorbed_fast(inp, seqs=[0])
+    _cmp(o[0], o_ref[0], TOL["bf16"], "o_lat")
+    _cmp(l[0], l_ref[0], TOL["bf16"], "lse", lse=True)
+
+
+def test_gathered_rows_many_sequences():
+    # 12 x 300 gathered entries: more than one planner pass over the entries,
+    # three tiles per sequence (the last one ragged)
+    wl = Workload("gm", "bf16", B=12, H=64, d_model=256, prefix=64, doc=1024, protected=300)
+    inp = make_inputs(wl, seed=10)
+    p = _gpu(inp)
+    o_ref, l_ref = O.decode_absorbed_fast(inp)
+    _cmp(p.o_lat.cpu().numpy(), o_ref, TOL["bf16"], "o_lat")
+    _cmp(p.lse.cpu().numpy(), l_ref, TOL["bf16"], "lse", lse=True)
 
 
 def test_query_before_every_row_is_empty():
