@@ -26,6 +26,10 @@ blocking, fusion or reordering beyond what the definitions state:
   offline (MLA-Off) partial plus protected rows recomputed online, Global
   heads online, merged before one shared output projection.
 
+Upstream of the decode, ``cache_rows`` and ``append_rows`` state how new
+tokens enter the paged cache (the latent as is, the rotary key rotated at its
+cache position, each logical row in its block-table page and slot).
+
 Readings where the pages are silent (each one is listed with its reason in
 the design notes): softmax scale 1/sqrt(d_n + d_r); RoPE on adjacent pairs
 (2i, 2i+1) with angle pos * base^(-2i/d_r); cached rotary keys stored already
@@ -192,6 +196,41 @@ def gather_cache(pool: np.ndarray, block_table_b: np.ndarray, rows: np.ndarray,
     """Cached rows [T, d_c + d_r] of one sequence, read through its block table."""
     pages = np.asarray(block_table_b)[rows // page]
     return np.asarray(pool[pages, rows % page], np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Cache writer (upstream of the decode) -- tutorial, "Position Rotations
+# Complicate the Absorption" (the decoupled rotary key is stored beside the
+# latent); RedKnot-MLA abstract (a document is cached at canonical position
+# zero and relocated on the query side)
+# ---------------------------------------------------------------------------
+
+def cache_rows(c, k_rope_raw, cache_pos, base: float) -> np.ndarray:
+    """Rows as the cache stores them, [T, d_c + d_r]: the latent c_t as it is
+    and the rotary key rotated at its cache position.
+
+    A row's cache position is its request position minus the relocation
+    offset it will be served with: a prefix row is cached at its request
+    position, a document cached on its own at 0, 1, 2, ...
+    """
+    c = np.asarray(c, np.float64)
+    k = rope_rotate(k_rope_raw, np.asarray(cache_pos, np.float64), base)
+    return np.concatenate([c, k], axis=-1)
+
+
+def append_rows(pool: np.ndarray, block_table_b: np.ndarray, row0: int, rows: np.ndarray,
+                page: int = 64) -> np.ndarray:
+    """Store ``rows`` as logical rows row0, row0 + 1, ... of one sequence.
+
+    Logical row r lives in page block_table_b[r // page] at slot r % page.
+    Returns a new fp64 pool; every slot not written keeps its old contents.
+    """
+    out = np.array(pool, dtype=np.float64, copy=True)
+    bt = np.asarray(block_table_b)
+    for i, row in enumerate(np.asarray(rows, np.float64)):
+        r = int(row0) + i
+        out[int(bt[r // page]), r % page] = row
+    return out
 
 
 # ---------------------------------------------------------------------------

@@ -23,6 +23,9 @@ PINS = [
     P.test_merge_of_any_split_equals_unsplit,
     P.test_merge_with_empty_is_identity,
     P.test_out_proj_fold_identity,
+    P.test_written_cache_serves_textbook_rope_attention,
+    P.test_cache_rows_at_position_zero_store_the_raw_key,
+    P.test_append_rows_lands_in_its_slots_only,
 ]
 
 
@@ -99,7 +102,35 @@ def _out_proj_T(o_lat, w_uv, w_o):
     return v, v.reshape(v.shape[0], -1) @ np.asarray(w_o, np.float64).T
 
 
-_ORIG = {k: getattr(O, k) for k in ("attend_direct", "merge_lse", "softmax_lse")}
+def _writer_position_plus_one(c, k_rope_raw, cache_pos, base):
+    return _ORIG["cache_rows"](c, k_rope_raw, np.asarray(cache_pos) + 1, base)
+
+
+def _writer_unrotated(c, k_rope_raw, cache_pos, base):
+    return np.concatenate([np.asarray(c, np.float64), np.asarray(k_rope_raw, np.float64)], -1)
+
+
+def _writer_request_rotation_sign(c, k_rope_raw, cache_pos, base):
+    return _ORIG["cache_rows"](c, k_rope_raw, -np.asarray(cache_pos), base)
+
+
+def _append_slot_shift(pool, block_table_b, row0, rows, page=64):
+    out = np.array(pool, dtype=np.float64, copy=True)
+    for i, row in enumerate(np.asarray(rows, np.float64)):
+        r = int(row0) + i
+        out[int(block_table_b[r // page]), (r + 1) % page] = row
+    return out
+
+
+def _append_page_of_next_row(pool, block_table_b, row0, rows, page=64):
+    out = np.array(pool, dtype=np.float64, copy=True)
+    for i, row in enumerate(np.asarray(rows, np.float64)):
+        r = int(row0) + i
+        out[int(block_table_b[(r + 1) // page]), r % page] = row
+    return out
+
+
+_ORIG = {k: getattr(O, k) for k in ("attend_direct", "merge_lse", "softmax_lse", "cache_rows")}
 
 MUTANTS = {
     "rope_sign": ("rope_rotate", _rope_sign),
@@ -115,6 +146,11 @@ MUTANTS = {
     "merge_weights_swapped": ("merge_lse", _merge_swapped),
     "lse_without_max": ("softmax_lse", _softmax_no_max),
     "out_proj_transposed": ("out_proj", _out_proj_T),
+    "writer_position_plus_one": ("cache_rows", _writer_position_plus_one),
+    "writer_unrotated": ("cache_rows", _writer_unrotated),
+    "writer_rotation_sign": ("cache_rows", _writer_request_rotation_sign),
+    "append_slot_shift": ("append_rows", _append_slot_shift),
+    "append_page_of_next_row": ("append_rows", _append_page_of_next_row),
 }
 
 

@@ -281,3 +281,80 @@ def test_out_proj_fold_identity():
     v1, _ = O.out_proj(np.array(g["weighted_latent"])[None, None, :],
                        np.array(g["u_v"])[None], np.eye(4))
     assert np.allclose(v1[0, 0], g["value_out"], rtol=0, atol=1e-15)
+
+
+# ------------------------------------------------------------- cache writer
+
+def _textbook_head(q_nope, q_rope, p, u_k, c, k_raw, req_pos, scale, base):
+    """One head and one query from the definitions, with Python complex
+    numbers: every visible row (request position <= p) scores
+    scale * (q_nope . U_K c_t + <R(p) q_rope, R(P_t) k_t>), where the rotary
+    dot product of two real vectors is the real part of sum_i z_q,i conj(z_k,i)
+    over the feature pairs.  Returns (sum_t a_t c_t, lse)."""
+    d_r = len(q_rope)
+    s = []
+    for t in range(len(c)):
+        if req_pos[t] > p:
+            continue
+        content = float(np.dot(q_nope, np.asarray(u_k, np.float64) @ c[t]))
+        rot = 0.0
+        for i in range(d_r // 2):
+            th = base ** (-2.0 * i / d_r)
+            zq = complex(q_rope[2 * i], q_rope[2 * i + 1]) * cmath.exp(1j * p * th)
+            zk = complex(k_raw[t][2 * i], k_raw[t][2 * i + 1]) * cmath.exp(1j * req_pos[t] * th)
+            rot += (zq * zk.conjugate()).real
+        s.append((t, scale * (content + rot)))
+    m = max(v for _, v in s)
+    tot = sum(math.exp(v - m) for _, v in s)
+    o = sum(math.exp(v - m) / tot * c[t] for t, v in s)
+    return o, m + math.log(tot)
+
+
+def test_written_cache_serves_textbook_rope_attention():
+    # prefix rows are cached at their request positions; a document is cached
+    # on its own at canonical positions 0, 1, ... and served right behind the
+    # prefix (relocation offset = prefix length)
+    wl = Workload("w", "f32", B=1, H=2, d_c=8, d_r=8, d_n=4, d_v=4, d_model=8,
+                  prefix=64, doc=37)
+    inp = make_inputs(wl, seed=11)
+    rows, kpos, ver = O.sequence_rows(inp.segs[0])
+    assert list(rows) == list(range(101))
+    rng = np.random.default_rng(12)
+    c = rng.standard_normal((101, wl.d_c))
+    k_raw = rng.standard_normal((101, wl.d_r))
+    cache_pos = kpos - np.asarray(inp.deltas)[ver]
+    assert list(cache_pos[:64]) == list(range(64)) and list(cache_pos[64:]) == list(range(37))
+    inp.pool = O.append_rows(inp.pool, inp.block_table[0], 0,
+                             O.cache_rows(c, k_raw, cache_pos, wl.rope_base))
+    o_d, l_d, _ = O.decode(inp)
+    o_a, l_a = O.decode_absorbed_fast(inp)
+    p = int(inp.q_pos[0])
+    for h in range(wl.H):
+        o_ref, l_ref = _textbook_head(inp.q_nope[0, h], inp.q_rope[0, h], p, inp.w_uk[h], c,
+                                      k_raw, kpos, wl.scale, wl.rope_base)
+        for o, l in ((o_d, l_d), (o_a, l_a)):
+            assert np.allclose(o[0, h], o_ref, rtol=0, atol=1e-10)
+            assert abs(l[0, h] - l_ref) < 1e-10
+
+
+def test_cache_rows_at_position_zero_store_the_raw_key():
+    rng = np.random.default_rng(13)
+    c, k = rng.standard_normal((3, 8)), rng.standard_normal((3, 6))
+    got = O.cache_rows(c, k, [0, 0, 0], 10000.0)
+    assert np.array_equal(got[:, :8], c) and np.array_equal(got[:, 8:], k)
+
+
+def test_append_rows_lands_in_its_slots_only():
+    pool = np.full((6, 64, 3), np.nan)
+    bt = np.array([4, 1, 5, 0])
+    rows = np.arange(300, dtype=np.float64).reshape(100, 3)
+    out = O.append_rows(pool, bt, 50, rows)          # logical rows 50 .. 149
+    # logical rows 50-63 are slots 50-63 of page 4, rows 64-127 all of page 1,
+    # rows 128-149 slots 0-21 of page 5; nothing else changes
+    assert np.array_equal(out[4, 50:], rows[0:14])
+    assert np.array_equal(out[1], rows[14:78])
+    assert np.array_equal(out[5, :22], rows[78:100])
+    untouched = np.ones((6, 64), bool)
+    untouched[4, 50:] = untouched[1] = untouched[5, :22] = False
+    assert np.isnan(out[untouched]).all()
+    assert np.isnan(pool).all()                      # the input pool is not modified
