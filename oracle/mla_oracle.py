@@ -26,6 +26,10 @@ blocking, fusion or reordering beyond what the definitions state:
   offline (MLA-Off) partial plus protected rows recomputed online, Global
   heads online, merged before one shared output projection.
 
+"QK-Normed MLA" abstract: post-projection QK RMSNorm made compatible with
+the latent path (``decode_qknorm``; the explicit form and the absorbed form
+with one cached inverse-RMS scalar per token).
+
 Upstream of the decode, ``cache_rows`` and ``append_rows`` state how new
 tokens enter the paged cache (the latent as is, the rotary key rotated at its
 cache position, each logical row in its block-table page and slot).
@@ -367,6 +371,98 @@ def decode_absorbed_fast(inp, heads=None, seqs=None, rows_override=None):
                                   p - int(inp.deltas[v]), wl.rope_base)    # [n_h, d_r]
                 s[:, sel] += q_r @ k_rope[sel].T                         # rotary term
             s = np.where((kpos <= p)[None, :], wl.scale * s, NEG_INF)
+            a, ls = softmax_lse(s)
+            o_lat[qi] = a @ c
+            lse[qi] = ls
+    return o_lat, lse
+
+
+# ---------------------------------------------------------------------------
+# QK-normed MLA -- "QK-Normed MLA" abstract: post-projection RMSNorm of the
+# queries and keys; the static key-side weight folds into the absorbed query
+# and the dynamic key statistic is one inverse-RMS scalar per token and KV
+# group, so the latent decode path survives
+# ---------------------------------------------------------------------------
+
+QK_NORM_EPS = 1e-6
+
+
+def rms_norm(x, weight, eps: float = QK_NORM_EPS) -> np.ndarray:
+    """x / sqrt(mean(x^2) + eps) * weight over the last axis."""
+    x = np.asarray(x, np.float64)
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps) * np.asarray(weight, np.float64)
+
+
+def key_inv_rms(c, w_uk, eps: float = QK_NORM_EPS) -> np.ndarray:
+    """The dynamic key statistic, one per token: 1 / rms of the token's content
+    keys of every head of the group, concatenated (H * d_n values).
+
+    c [T, d_c]; w_uk [H, d_n, d_c] -> [T].  Computable when the row is
+    written, from the latent alone.
+    """
+    k = np.einsum("hnc,tc->thn", np.asarray(w_uk, np.float64), np.asarray(c, np.float64))
+    k = k.reshape(k.shape[0], -1)
+    return 1.0 / np.sqrt(np.mean(k * k, axis=-1) + eps)
+
+
+def qknorm_scores_direct(q_nope, q_rope, q_pos, w_uk, c, k_rope, key_shift, g_q, g_k,
+                         scale, base, eps: float = QK_NORM_EPS) -> np.ndarray:
+    """Scaled scores [H, T] of one query token with explicit post-projection
+    QK RMSNorm: the content query of all heads (H * d_n values) and each
+    token's content keys of all heads are normalised with weights g_q, g_k;
+    the rotary path is left as it is.  Keys are expanded (U_K c_t) and the
+    cached rotary keys restored to their request positions, as in
+    ``attend_direct``.  q_nope [H, d_n]; q_rope [H, d_r]; w_uk [H, d_n, d_c];
+    c [T, d_c]; k_rope [T, d_r]; key_shift [T]; g_q, g_k [H * d_n].
+    """
+    H, d_n = np.asarray(q_nope).shape
+    q_hat = rms_norm(np.asarray(q_nope, np.float64).reshape(-1), g_q, eps).reshape(H, d_n)
+    k = np.einsum("hnc,tc->thn", np.asarray(w_uk, np.float64), np.asarray(c, np.float64))
+    k_hat = rms_norm(k.reshape(k.shape[0], -1), g_k, eps).reshape(k.shape)
+    k_r = rope_rotate(k_rope, key_shift, base)
+    q_r = rope_rotate(q_rope, q_pos, base)
+    return scale * (np.einsum("hn,thn->ht", q_hat, k_hat) + q_r @ k_r.T)
+
+
+def qknorm_scores_absorbed(q_nope, q_rope, q_pos, w_uk, c, k_rope, key_shift, g_q, g_k,
+                           scale, base, eps: float = QK_NORM_EPS) -> np.ndarray:
+    """The same scores [H, T] through the latent path: the query is normalised
+    and multiplied by the key weight, then absorbed, U_K^T (g_k * q_hat); the
+    content score against the cached latent is multiplied by the token's
+    inverse key RMS; the rotary query is relocated per row as in
+    ``attend_absorbed``.
+    """
+    H, d_n = np.asarray(q_nope).shape
+    q_hat = rms_norm(np.asarray(q_nope, np.float64).reshape(-1), g_q, eps).reshape(H, d_n)
+    q_w = q_hat * np.asarray(g_k, np.float64).reshape(H, d_n)
+    q_lat = np.einsum("hn,hnc->hc", q_w, np.asarray(w_uk, np.float64))      # [H, d_c]
+    c = np.asarray(c, np.float64)
+    content = (q_lat @ c.T) * key_inv_rms(c, w_uk, eps)[None, :]
+    rel = np.asarray(q_pos, np.float64) - np.asarray(key_shift, np.float64)    # [T]
+    q_r = rope_rotate(np.asarray(q_rope, np.float64)[:, None, :], rel[None, :], base)  # [H, T, d_r]
+    rotary = np.einsum("htd,td->ht", q_r, np.asarray(k_rope, np.float64))
+    return scale * (content + rotary)
+
+
+def decode_qknorm(inp, g_q, g_k, form: str = "absorbed", eps: float = QK_NORM_EPS, seqs=None):
+    """QK-normed attention of every query token over its sequence (all heads
+    form one KV group).  Masking, softmax and the weighted latent are those of
+    the plain decode.  Returns o_lat [n_q, H, d_c], lse [n_q, H]."""
+    wl = inp.wl
+    scores = qknorm_scores_absorbed if form == "absorbed" else qknorm_scores_direct
+    o_lat = np.full((inp.n_q, wl.H, wl.d_c), np.nan)
+    lse = np.full((inp.n_q, wl.H), np.nan)
+    for b in (range(wl.B) if seqs is None else seqs):
+        rows, kpos, ver = sequence_rows(inp.segs[b])
+        cache = gather_cache(inp.pool, inp.block_table[b], rows)
+        c, k_rope = cache[:, :wl.d_c], cache[:, wl.d_c:]
+        shift = np.asarray(inp.deltas, np.int64)[ver]
+        for j in range(wl.s_q):
+            qi = b * wl.s_q + j
+            p = int(inp.q_pos[qi])
+            s = scores(inp.q_nope[qi], inp.q_rope[qi], p, inp.w_uk, c, k_rope, shift,
+                       g_q, g_k, wl.scale, wl.rope_base, eps)
+            s = np.where((kpos <= p)[None, :], s, NEG_INF)
             a, ls = softmax_lse(s)
             o_lat[qi] = a @ c
             lse[qi] = ls

@@ -26,6 +26,10 @@ PINS = [
     P.test_written_cache_serves_textbook_rope_attention,
     P.test_cache_rows_at_position_zero_store_the_raw_key,
     P.test_append_rows_lands_in_its_slots_only,
+    lambda: P.test_qknorm_absorbed_equals_explicit(dict(s_q=2, lengths=(13, 70))),
+    P.test_qknorm_matches_torch_rms_norm_and_sdpa,
+    P.test_qknorm_is_scale_invariant_in_query_and_latent,
+    P.test_qknorm_with_unit_rms_inputs_is_plain_attention,
 ]
 
 
@@ -130,7 +134,48 @@ def _append_page_of_next_row(pool, block_table_b, row0, rows, page=64):
     return out
 
 
-_ORIG = {k: getattr(O, k) for k in ("attend_direct", "merge_lse", "softmax_lse", "cache_rows")}
+def _qk_absorbed_rope_scaled(q_nope, q_rope, q_pos, w_uk, c, k_rope, key_shift, g_q, g_k,
+                             scale, base, eps=O.QK_NORM_EPS):
+    # the per-token key statistic applied to the whole score, rotary term too
+    s = _ORIG["qknorm_scores_absorbed"](q_nope, q_rope, q_pos, w_uk, c, k_rope, key_shift,
+                                        g_q, g_k, scale, base, eps)
+    inv = O.key_inv_rms(c, w_uk, eps)
+    content = _ORIG["qknorm_scores_absorbed"](q_nope, np.zeros_like(q_rope), q_pos, w_uk, c,
+                                              k_rope, key_shift, g_q, g_k, scale, base, eps)
+    return content + (s - content) * inv[None, :]
+
+
+def _qk_absorbed_key_weight_dropped(q_nope, q_rope, q_pos, w_uk, c, k_rope, key_shift, g_q,
+                                    g_k, scale, base, eps=O.QK_NORM_EPS):
+    return _ORIG["qknorm_scores_absorbed"](q_nope, q_rope, q_pos, w_uk, c, k_rope, key_shift,
+                                           g_q, np.ones_like(np.asarray(g_k, np.float64)),
+                                           scale, base, eps)
+
+
+def _key_inv_rms_first_head(c, w_uk, eps=O.QK_NORM_EPS):
+    return _ORIG["key_inv_rms"](c, np.asarray(w_uk)[:1], eps)
+
+
+def _rms_norm_eps_outside(x, weight, eps=O.QK_NORM_EPS):
+    x = np.asarray(x, np.float64)
+    return x / (np.sqrt(np.mean(x * x, axis=-1, keepdims=True)) + eps) * np.asarray(weight)
+
+
+def _qk_direct_no_query_norm(q_nope, q_rope, q_pos, w_uk, c, k_rope, key_shift, g_q, g_k,
+                             scale, base, eps=O.QK_NORM_EPS):
+    # the query weight applied but the query never divided by its RMS
+    H, d_n = np.asarray(q_nope).shape
+    q_w = np.asarray(q_nope, np.float64) * np.asarray(g_q, np.float64).reshape(H, d_n)
+    k = np.einsum("hnc,tc->thn", np.asarray(w_uk, np.float64), np.asarray(c, np.float64))
+    k_hat = O.rms_norm(k.reshape(k.shape[0], -1), g_k, eps).reshape(k.shape)
+    q_r = O.rope_rotate(q_rope, q_pos, base)
+    k_r = O.rope_rotate(k_rope, key_shift, base)
+    return scale * (np.einsum("hn,thn->ht", q_w, k_hat) + q_r @ k_r.T)
+
+
+_ORIG = {k: getattr(O, k) for k in ("attend_direct", "merge_lse", "softmax_lse", "cache_rows",
+                                    "qknorm_scores_absorbed", "qknorm_scores_direct",
+                                    "key_inv_rms")}
 
 MUTANTS = {
     "rope_sign": ("rope_rotate", _rope_sign),
@@ -151,6 +196,11 @@ MUTANTS = {
     "writer_rotation_sign": ("cache_rows", _writer_request_rotation_sign),
     "append_slot_shift": ("append_rows", _append_slot_shift),
     "append_page_of_next_row": ("append_rows", _append_page_of_next_row),
+    "qknorm_rope_scaled": ("qknorm_scores_absorbed", _qk_absorbed_rope_scaled),
+    "qknorm_key_weight_dropped": ("qknorm_scores_absorbed", _qk_absorbed_key_weight_dropped),
+    "qknorm_stat_one_head": ("key_inv_rms", _key_inv_rms_first_head),
+    "qknorm_eps_outside_sqrt": ("rms_norm", _rms_norm_eps_outside),
+    "qknorm_query_not_normalised": ("qknorm_scores_direct", _qk_direct_no_query_norm),
 }
 
 

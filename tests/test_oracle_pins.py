@@ -358,3 +358,98 @@ def test_append_rows_lands_in_its_slots_only():
     untouched[4, 50:] = untouched[1] = untouched[5, :22] = False
     assert np.isnan(out[untouched]).all()
     assert np.isnan(pool).all()                      # the input pool is not modified
+
+
+# ------------------------------------------------------------- QK-normed MLA
+
+def _qk_weights(inp, seed=21):
+    g = np.random.default_rng(seed)
+    n = inp.wl.H * inp.wl.d_n
+    return 1.0 + 0.2 * g.standard_normal(n), 1.0 + 0.2 * g.standard_normal(n)
+
+
+@pytest.mark.parametrize("kw", [dict(s_q=2, lengths=(13, 70)),
+                                dict(B=1, s_q=1, lengths=None, prefix=64, doc=45)])
+def test_qknorm_absorbed_equals_explicit(kw):
+    # "exactly equivalent to explicit post-projection QK RMSNorm in exact
+    # arithmetic": the latent path with one inverse-RMS scalar per token
+    inp = _tiny(**kw)
+    g_q, g_k = _qk_weights(inp)
+    o_a, l_a = O.decode_qknorm(inp, g_q, g_k, "absorbed")
+    o_d, l_d = O.decode_qknorm(inp, g_q, g_k, "direct")
+    assert np.allclose(o_a, o_d, rtol=0, atol=1e-12)
+    assert np.allclose(l_a, l_d, rtol=0, atol=1e-12)
+
+
+def test_qknorm_matches_torch_rms_norm_and_sdpa():
+    """Keys expanded explicitly, normalised by torch's rms_norm over all heads'
+    content keys of a token, rotary parts by complex multiplication, then
+    torch's scaled_dot_product_attention with the latent as values."""
+    inp = _tiny(s_q=2, lengths=(13, 70))
+    wl = inp.wl
+    g_q, g_k = _qk_weights(inp)
+    eps = O.QK_NORM_EPS
+    T = torch.from_numpy
+    outs = [O.decode_qknorm(inp, g_q, g_k, form) for form in ("absorbed", "direct")]
+    for b in range(wl.B):
+        rows = int(inp.n_rows[b])
+        r = np.arange(rows)
+        cache = inp.pool[inp.block_table[b, r // 64], r % 64].astype(np.float64)
+        c, kr = cache[:, :wl.d_c], cache[:, wl.d_c:]
+        k_all = np.stack([c @ inp.w_uk[h].astype(np.float64).T for h in range(wl.H)], 1)
+        k_hat = torch.nn.functional.rms_norm(T(k_all.reshape(rows, -1)), (wl.H * wl.d_n,),
+                                             T(g_k), eps).numpy().reshape(rows, wl.H, wl.d_n)
+        for j in range(wl.s_q):
+            qi = b * wl.s_q + j
+            qp = int(inp.q_pos[qi])
+            q_hat = torch.nn.functional.rms_norm(
+                T(inp.q_nope[qi].astype(np.float64).reshape(-1)), (wl.H * wl.d_n,), T(g_q),
+                eps).numpy().reshape(wl.H, wl.d_n)
+            mask = torch.tensor(r[None, :] <= qp)
+            for h in range(wl.H):
+                q = np.concatenate([q_hat[h], _rope_complex(inp.q_rope[qi, h], qp, wl.rope_base)])
+                k = np.concatenate([k_hat[:, h], kr], 1)
+                ref = torch.nn.functional.scaled_dot_product_attention(
+                    T(q)[None, None], T(k)[None], T(c)[None], attn_mask=mask[None],
+                    scale=wl.scale)[0, 0].numpy()
+                for o, _ in outs:
+                    assert np.allclose(o[qi, h], ref, rtol=0, atol=1e-12)
+
+
+def test_qknorm_is_scale_invariant_in_query_and_latent():
+    # with eps = 0 the normalised content keys ignore a common scale of the
+    # latent (so o_lat scales with it), and the normalised query ignores a
+    # scale of q_nope
+    inp = _tiny(s_q=2, lengths=(13, 70))
+    g_q, g_k = _qk_weights(inp)
+    o1, l1 = O.decode_qknorm(inp, g_q, g_k, eps=0.0)
+    big = copy.deepcopy(inp)
+    big.pool = inp.pool.astype(np.float64)
+    big.pool[:, :, :inp.wl.d_c] *= 3.5
+    big.q_nope = inp.q_nope * 0.25
+    o2, l2 = O.decode_qknorm(big, g_q, g_k, eps=0.0)
+    assert np.allclose(o2, 3.5 * o1, rtol=0, atol=1e-11)
+    assert np.allclose(l2, l1, rtol=0, atol=1e-11)
+
+
+def test_qknorm_with_unit_rms_inputs_is_plain_attention():
+    # unit weights, eps = 0, every token's content keys (all heads) and every
+    # query's content part already of RMS 1: the norms are identities
+    inp = _tiny(s_q=2, lengths=(13, 70))
+    wl = inp.wl
+    pool = inp.pool.astype(np.float64)
+    for pg in range(pool.shape[0]):
+        for sl in range(pool.shape[1]):
+            c = pool[pg, sl, :wl.d_c]
+            if np.isnan(c).any():
+                continue
+            k = np.concatenate([inp.w_uk[h].astype(np.float64) @ c for h in range(wl.H)])
+            pool[pg, sl, :wl.d_c] = c / math.sqrt(float(np.mean(k * k)))
+    inp.pool = pool
+    qn = inp.q_nope.astype(np.float64)
+    inp.q_nope = qn / np.sqrt(np.mean(qn.reshape(qn.shape[0], -1) ** 2, -1))[:, None, None]
+    ones = np.ones(wl.H * wl.d_n)
+    o_n, l_n = O.decode_qknorm(inp, ones, ones, eps=0.0)
+    o_p, l_p = O.decode_absorbed_fast(inp)
+    assert np.allclose(o_n, o_p, rtol=0, atol=1e-11)
+    assert np.allclose(l_n, l_p, rtol=0, atol=1e-11)
