@@ -30,6 +30,9 @@ blocking, fusion or reordering beyond what the definitions state:
 the latent path (``decode_qknorm``; the explicit form and the absorbed form
 with one cached inverse-RMS scalar per token).
 
+QuantMLA abstract: a low-bit latent cache (symmetric per-channel codes,
+packed; ``dequantize_pool`` gives the cache the low-bit attention reads).
+
 Upstream of the decode, ``cache_rows`` and ``append_rows`` state how new
 tokens enter the paged cache (the latent as is, the rotary key rotated at its
 cache position, each logical row in its block-table page and slot).
@@ -469,6 +472,71 @@ def decode_qknorm(inp, g_q, g_k, form: str = "absorbed", eps: float = QK_NORM_EP
     return o_lat, lse
 
 
+# ---------------------------------------------------------------------------
+# Low-bit latent cache -- QuantMLA abstract: the content and rotary caches
+# stored as low-bit integers (INT4 and INT4, or INT2 content with an INT4
+# rotary key), unpacked and dequantised inside the attention.  The learned,
+# offline-fused transforms of the abstract are not modelled: the scales are
+# inputs.
+# ---------------------------------------------------------------------------
+
+def quantize_symmetric(x, scale, bits: int) -> np.ndarray:
+    """Signed codes round(x / scale), ties to even, clamped to
+    [-2^(bits-1), 2^(bits-1) - 1]; ``scale`` broadcasts over the last axis
+    (one static scale per channel).  Returns int64 codes."""
+    lo, hi = -(1 << (bits - 1)), (1 << (bits - 1)) - 1
+    q = np.round(np.asarray(x, np.float64) / np.asarray(scale, np.float64))
+    return np.clip(q, lo, hi).astype(np.int64)
+
+
+def dequantize(codes, scale) -> np.ndarray:
+    """The value a code stands for: code * its channel's scale."""
+    return np.asarray(codes, np.float64) * np.asarray(scale, np.float64)
+
+
+def pack_codes(codes, bits: int) -> np.ndarray:
+    """Pack signed codes along the last axis into bytes, 8 / bits codes per
+    byte, the first code in the lowest bits, each as a bits-wide two's
+    complement field."""
+    codes = np.asarray(codes, np.int64)
+    per = 8 // bits
+    n = codes.shape[-1]
+    assert n % per == 0
+    fields = (codes & ((1 << bits) - 1)).reshape(codes.shape[:-1] + (n // per, per))
+    out = np.zeros(fields.shape[:-1], np.int64)
+    for k in range(per):
+        out |= fields[..., k] << (bits * k)
+    return out.astype(np.uint8)
+
+
+def unpack_codes(packed, bits: int) -> np.ndarray:
+    """Inverse of ``pack_codes``: signed codes, 8 / bits per byte."""
+    b = np.asarray(packed, np.int64)
+    per = 8 // bits
+    mask, sign = (1 << bits) - 1, 1 << (bits - 1)
+    fields = np.stack([(b >> (bits * k)) & mask for k in range(per)], axis=-1)
+    codes = np.where(fields >= sign, fields - (1 << bits), fields)
+    return codes.reshape(b.shape[:-1] + (b.shape[-1] * per,))
+
+
+def quantized_row_bytes(d_c: int, d_r: int, bits_c: int, bits_r: int) -> int:
+    """Bytes of one packed cache row (content codes, then rotary codes)."""
+    return (d_c * bits_c + d_r * bits_r) // 8
+
+
+def dequantize_pool(pool, d_c: int, scale_c, scale_r, bits_c: int, bits_r: int) -> np.ndarray:
+    """The cache the low-bit attention reads: every stored row quantised with
+    its per-channel scales (content and rotary separately) and dequantised.
+    NaN rows (never referenced) stay NaN."""
+    pool = np.asarray(pool, np.float64)
+    out = np.array(pool, copy=True)
+    used = ~np.isnan(pool).any(axis=-1)
+    rows = pool[used]
+    out[used, :d_c] = dequantize(quantize_symmetric(rows[:, :d_c], scale_c, bits_c), scale_c)
+    out[used, d_c:] = dequantize(quantize_symmetric(rows[:, d_c:], scale_r, bits_r), scale_r)
+    return out
+
+
 def out_proj(o_lat, w_uv, w_o):
     """Value up-projection per head, then the shared output projection.
 
@@ -481,3 +549,21 @@ def out_proj(o_lat, w_uv, w_o):
     v = np.einsum("hdc,qhc->qhd", np.asarray(w_uv, np.float64), o_lat)
     out = v.reshape(v.shape[0], -1) @ np.asarray(w_o, np.float64).T
     return v, out
+
+
+def fold_value_into_output(w_uv, w_o) -> np.ndarray:
+    """Each head's value up-projection folded into its slice of the output
+    projection (tutorial, "Move the Value Expansion After the Weighted Sum"):
+    W_fold[:, h*d_c:(h+1)*d_c] = W_O[:, h*d_v:(h+1)*d_v] W_UV[h].
+    w_uv [H, d_v, d_c]; w_o [d_model, H*d_v] -> [d_model, H*d_c]."""
+    w_uv = np.asarray(w_uv, np.float64)
+    w_o = np.asarray(w_o, np.float64)
+    H, d_v, _ = w_uv.shape
+    return np.concatenate([w_o[:, h * d_v:(h + 1) * d_v] @ w_uv[h] for h in range(H)], axis=1)
+
+
+def out_proj_folded(o_lat, w_fold) -> np.ndarray:
+    """out = W_fold concat_h(o_lat_h): one product from the weighted latents."""
+    o_lat = np.asarray(o_lat, np.float64)
+    return o_lat.reshape(o_lat.shape[0], -1) @ np.asarray(w_fold, np.float64).T
+

@@ -30,6 +30,11 @@ PINS = [
     P.test_qknorm_matches_torch_rms_norm_and_sdpa,
     P.test_qknorm_is_scale_invariant_in_query_and_latent,
     P.test_qknorm_with_unit_rms_inputs_is_plain_attention,
+    P.test_packed_code_bytes_worked_by_hand,
+    lambda: P.test_pack_unpack_round_trip_every_byte(4),
+    lambda: P.test_quantization_error_bound_and_saturation(4),
+    P.test_quantization_ties_go_to_the_even_code,
+    lambda: P.test_grid_exact_cache_passes_through_unchanged(4),
 ]
 
 
@@ -173,6 +178,39 @@ def _qk_direct_no_query_norm(q_nope, q_rope, q_pos, w_uk, c, k_rope, key_shift, 
     return scale * (np.einsum("hn,thn->ht", q_w, k_hat) + q_r @ k_r.T)
 
 
+def _quantize_truncating(x, scale, bits):
+    lo, hi = -(1 << (bits - 1)), (1 << (bits - 1)) - 1
+    q = np.trunc(np.asarray(x, np.float64) / np.asarray(scale, np.float64))
+    return np.clip(q, lo, hi).astype(np.int64)
+
+
+def _quantize_symmetric_range(x, scale, bits):
+    hi = (1 << (bits - 1)) - 1
+    q = np.round(np.asarray(x, np.float64) / np.asarray(scale, np.float64))
+    return np.clip(q, -hi, hi).astype(np.int64)
+
+
+def _pack_high_first(codes, bits):
+    codes = np.asarray(codes, np.int64)
+    per = 8 // bits
+    fields = (codes & ((1 << bits) - 1)).reshape(codes.shape[:-1] + (-1, per))
+    out = np.zeros(fields.shape[:-1], np.int64)
+    for k in range(per):
+        out |= fields[..., k] << (bits * (per - 1 - k))
+    return out.astype(np.uint8)
+
+
+def _unpack_unsigned(packed, bits):
+    b = np.asarray(packed, np.int64)
+    per = 8 // bits
+    fields = np.stack([(b >> (bits * k)) & ((1 << bits) - 1) for k in range(per)], axis=-1)
+    return fields.reshape(b.shape[:-1] + (b.shape[-1] * per,))
+
+
+def _dequantize_divides(codes, scale):
+    return np.asarray(codes, np.float64) / np.asarray(scale, np.float64)
+
+
 _ORIG = {k: getattr(O, k) for k in ("attend_direct", "merge_lse", "softmax_lse", "cache_rows",
                                     "qknorm_scores_absorbed", "qknorm_scores_direct",
                                     "key_inv_rms")}
@@ -201,6 +239,11 @@ MUTANTS = {
     "qknorm_stat_one_head": ("key_inv_rms", _key_inv_rms_first_head),
     "qknorm_eps_outside_sqrt": ("rms_norm", _rms_norm_eps_outside),
     "qknorm_query_not_normalised": ("qknorm_scores_direct", _qk_direct_no_query_norm),
+    "quantize_truncates": ("quantize_symmetric", _quantize_truncating),
+    "quantize_symmetric_range": ("quantize_symmetric", _quantize_symmetric_range),
+    "pack_first_code_high": ("pack_codes", _pack_high_first),
+    "unpack_without_sign": ("unpack_codes", _unpack_unsigned),
+    "dequantize_divides": ("dequantize", _dequantize_divides),
 }
 
 

@@ -7,6 +7,7 @@ that a dropped term, a wrong sign or index, or a transposed operand fails.
 CPU only.
 """
 import cmath
+import itertools
 import copy
 import json
 import math
@@ -277,6 +278,16 @@ def test_out_proj_fold_identity():
     v, out = O.out_proj(o, w_uv, w_o)
     folded = sum(o[:, h] @ (w_o[:, h * d_v:(h + 1) * d_v] @ w_uv[h]).T for h in range(H))
     assert np.allclose(out, folded, rtol=0, atol=1e-12)
+    w_fold = O.fold_value_into_output(w_uv, w_o)
+    assert w_fold.shape == (d_model, H * d_c)
+    assert np.allclose(O.out_proj_folded(o, w_fold), out, rtol=0, atol=1e-12)
+    # by hand: W_UV = [[1, 2], [3, 4]], W_O = [[5, 6]] fold to [5+18, 10+24] =
+    # [23, 34]; o = [1, 1] gives 57 both ways (W_UV o = [3, 7]; 15 + 42)
+    wf = O.fold_value_into_output(np.array([[[1.0, 2.0], [3.0, 4.0]]]), np.array([[5.0, 6.0]]))
+    assert wf.tolist() == [[23.0, 34.0]]
+    assert O.out_proj_folded(np.array([[[1.0, 1.0]]]), wf).tolist() == [[57.0]]
+    assert O.out_proj(np.array([[[1.0, 1.0]]]), np.array([[[1.0, 2.0], [3.0, 4.0]]]),
+                      np.array([[5.0, 6.0]]))[1].tolist() == [[57.0]]
     g = GOLD["value"]
     v1, _ = O.out_proj(np.array(g["weighted_latent"])[None, None, :],
                        np.array(g["u_v"])[None], np.eye(4))
@@ -453,3 +464,69 @@ def test_qknorm_with_unit_rms_inputs_is_plain_attention():
     o_p, l_p = O.decode_absorbed_fast(inp)
     assert np.allclose(o_n, o_p, rtol=0, atol=1e-11)
     assert np.allclose(l_n, l_p, rtol=0, atol=1e-11)
+
+
+# ------------------------------------------------------------- low-bit cache
+
+def test_packed_code_bytes_worked_by_hand():
+    # INT4, first code in the low nibble: 1 -> 0x1 and -2 -> 0xE make 0xE1;
+    # 7 -> 0x7 and -8 -> 0x8 make 0x87.  INT2, fields from the low bits up:
+    # 1 -> 01, -2 -> 10, 0 -> 00, -1 -> 11 make 0b11001001 = 0xC9.
+    assert O.pack_codes(np.array([1, -2, 7, -8]), 4).tolist() == [0xE1, 0x87]
+    assert O.pack_codes(np.array([1, -2, 0, -1]), 2).tolist() == [0xC9]
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_pack_unpack_round_trip_every_byte(bits):
+    lo, hi = -(1 << (bits - 1)), (1 << (bits - 1)) - 1
+    per = 8 // bits
+    codes = np.array(list(itertools.product(range(lo, hi + 1), repeat=per))).reshape(-1)
+    packed = O.pack_codes(codes, bits)
+    assert sorted(packed.tolist()) == list(range(256))     # each byte value once
+    assert np.array_equal(O.unpack_codes(packed, bits), codes)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_quantization_error_bound_and_saturation(bits):
+    lo, hi = -(1 << (bits - 1)), (1 << (bits - 1)) - 1
+    scale = np.array([0.5, 0.25, 2.0])
+    x = np.random.default_rng(bits).uniform(lo, hi, (1000, 3)) * scale
+    err = np.abs(O.dequantize(O.quantize_symmetric(x, scale, bits), scale) - x)
+    assert (err <= scale / 2 + 1e-15).all()
+    far = np.array([[100.0, -100.0, 1e9]]) * scale
+    assert O.quantize_symmetric(far, scale, bits).tolist() == [[hi, lo, hi]]
+
+
+def test_quantization_ties_go_to_the_even_code():
+    s = np.array([1.0])
+    x = np.array([[0.5], [1.5], [2.5], [-0.5], [-1.5], [6.5]])
+    assert O.quantize_symmetric(x, s, 4)[:, 0].tolist() == [0, 2, 2, 0, -2, 6]
+
+
+@pytest.mark.parametrize("bits_c", [2, 4])
+def test_grid_exact_cache_passes_through_unchanged(bits_c):
+    # a cache whose values are already code * channel scale is stored
+    # exactly, so the low-bit attention equals the plain one on it
+    inp = _tiny(s_q=2, lengths=(13, 70))
+    wl = inp.wl
+    g = np.random.default_rng(31)
+    sc, sr = g.uniform(0.2, 0.6, wl.d_c), g.uniform(0.2, 0.6, wl.d_r)
+    pool = inp.pool.astype(np.float64)
+    used = ~np.isnan(pool).any(-1)
+    n = int(used.sum())
+    pool[used, :wl.d_c] = g.integers(-(1 << (bits_c - 1)), 1 << (bits_c - 1), (n, wl.d_c)) * sc
+    pool[used, wl.d_c:] = g.integers(-8, 8, (n, wl.d_r)) * sr
+    deq = O.dequantize_pool(pool, wl.d_c, sc, sr, bits_c, 4)
+    assert np.array_equal(deq, pool, equal_nan=True)
+    inp.pool = pool
+    o1, l1 = O.decode_absorbed_fast(inp)
+    inp.pool = deq
+    o2, l2 = O.decode_absorbed_fast(inp)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_quantized_row_bytes():
+    # 512 content + 64 rotary values: 1152 bytes in bf16, 288 at INT4/INT4
+    # (4x), 160 at INT2 content with an INT4 rotary key (7.2x)
+    assert O.quantized_row_bytes(512, 64, 4, 4) == 288
+    assert O.quantized_row_bytes(512, 64, 2, 4) == 160
