@@ -530,3 +530,33 @@ def test_quantized_row_bytes():
     # (4x), 160 at INT2 content with an INT4 rotary key (7.2x)
     assert O.quantized_row_bytes(512, 64, 4, 4) == 288
     assert O.quantized_row_bytes(512, 64, 2, 4) == 160
+
+
+# ------------------------------------- absorbed vs direct on the named configs
+
+def test_absorbed_equals_direct_on_named_configs():
+    # the absorbed form gives the large configs their full coverage; the
+    # direct (expanded-key) form checks it on seeded samples of them
+    from head_latent_attention_02_b200.workloads import WORKLOADS
+    inp = make_inputs(WORKLOADS["tiny_f32"], seed=0)
+    d_lat, d_lse, _ = O.decode(inp)
+    f_lat, f_lse = O.decode_absorbed_fast(inp)
+    assert np.allclose(f_lat, d_lat, rtol=1e-10, atol=1e-12)
+    assert np.allclose(f_lse, d_lse, rtol=1e-10, atol=1e-12)
+    # B=16 x 4096 rows: sequences 0 and 15, heads 0 and 127
+    inp = make_inputs(WORKLOADS["bf16_b16_4k"], seed=0, with_weights=True)
+    seqs, heads = [0, 15], [0, 127]
+    d_lat, d_lse, _ = O.decode(inp, heads=heads, seqs=seqs)
+    f_lat, f_lse = O.decode_absorbed_fast(inp, heads=heads, seqs=seqs)
+    rows = np.array(seqs)
+    assert np.allclose(f_lat[rows], d_lat[rows], rtol=1e-10, atol=1e-12)
+    assert np.allclose(f_lse[rows], d_lse[rows], rtol=1e-10, atol=1e-12)
+    # RedKnot: a head over all 24 576 rows (prefix + relocated document) and
+    # a head over the 256 gathered protected rows
+    inp = make_inputs(WORKLOADS["redknot_56_8"], seed=0)
+    rows_all = {0: list(range(int(inp.n_rows[0])))}
+    for ov in (rows_all, None):
+        d_lat, d_lse, _ = O.decode(inp, heads=[3], rows_override=ov)
+        f_lat, f_lse = O.decode_absorbed_fast(inp, heads=[3], rows_override=ov)
+        assert np.allclose(f_lat, d_lat, rtol=1e-10, atol=1e-12)
+        assert np.allclose(f_lse, d_lse, rtol=1e-10, atol=1e-12)
