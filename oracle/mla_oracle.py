@@ -68,6 +68,14 @@ def mha_cache_bytes(L: int, T: int, B: int, heads: int, d_k: int, d_v: int, b: i
     return L * T * B * heads * (d_k + d_v) * b
 
 
+def head_row_ceiling(local_heads: int, global_heads: int, reusable_layers: int,
+                     total_layers: int) -> float:
+    """RedKnot-MLA abstract, analytic logical head-row ceiling: the share of
+    (layer, head) rows that can come from the offline path -- the Local
+    heads' share of the heads times the reusable layers' share of the layers."""
+    return local_heads / (local_heads + global_heads) * reusable_layers / total_layers
+
+
 # ---------------------------------------------------------------------------
 # Content path -- tutorial, "The Direct Form" and "Move the Key Projection"
 # ---------------------------------------------------------------------------

@@ -560,3 +560,15 @@ def test_absorbed_equals_direct_on_named_configs():
         f_lat, f_lse = O.decode_absorbed_fast(inp, heads=[3], rows_override=ov)
         assert np.allclose(f_lat, d_lat, rtol=1e-10, atol=1e-12)
         assert np.allclose(f_lse, d_lse, rtol=1e-10, atol=1e-12)
+
+
+def test_redknot_head_row_ceilings():
+    # informational: the printed percentages follow from the printed layer
+    # and head counts with the inferred layer totals
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "redknot_head_rows.json")))
+    for pr in g["profiles"]:
+        c = O.head_row_ceiling(pr["local_heads"], pr["global_heads"], pr["reusable_layers"],
+                               pr["total_layers"])
+        assert round(100 * c, 2) == pr["ceiling_percent"], pr["name"]
+    # the 56/8 split of the RedKnot config is the Flash profile's
+    assert O.head_row_ceiling(56, 8, 1, 1) == 0.875
