@@ -77,6 +77,36 @@ def _cache_bytes(wl, rows_per_seq):
     return int(sum(rows_per_seq)) * (wl.d_c + wl.d_r) * 2
 
 
+def decode_flops(wl, n_rows, n_gather=None):
+    """Attention FLOPs of one step's decode calls: 2 * s_q * heads * rows *
+    (d_c + d_r + d_c) -- the score over the 576-wide row and the weighted sum
+    over the latent.  Global heads (all heads without a Local/Global split)
+    attend every row of their sequence; Local heads attend the gathered rows."""
+    per_row = 2 * wl.s_q * (2 * wl.d_c + wl.d_r)
+    rows = int(np.sum(n_rows))
+    if not wl.n_local:
+        return per_row * wl.H * rows
+    gathered = int(np.sum(n_gather)) if n_gather is not None else 0
+    return per_row * ((wl.H - wl.n_local) * rows + wl.n_local * gathered)
+
+
+def decode_roofline(flops, cache_bytes, t_dec_ms, peaks, src, traffic, kernel):
+    """Roofline object of the decode call: against HBM (cache bytes / time)
+    unless its arithmetic intensity is above the measured ridge (bf16 peak /
+    HBM copy rate), then against the bf16 tensor peak (FLOPs / time)."""
+    t = t_dec_ms * 1e-3
+    intensity = flops / cache_bytes
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if intensity > ridge:
+        achieved, peak, unit, bound = flops / t / 1e12, peaks["bf16_tflops"], "TFLOP/s", "tensor"
+    else:
+        achieved, peak, unit, bound = cache_bytes / t / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
+    return {"bound": bound, "achieved": round(achieved, 1), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": kernel,
+            "peak_source": src, "flop_per_byte": round(intensity, 1),
+            "ridge_flop_per_byte": round(ridge, 1)}
+
+
 # ---------------------------------------------------------------- multi-rank
 def max_over_ranks(values, device, world):
     """Element-wise max of per-rank times over all ranks: the job is as slow
@@ -345,13 +375,11 @@ def run_gpu(args):
                              "how": "each call's own graph replayed back to back"},
             "decode_only": {"us": round(t_dec * 1e3, 2), "GB_s": round(achieved, 1),
                             "kernels": kernels_per_decode},
-            "roofline": {"bound": "hbm", "achieved": round(achieved, 1),
-                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(achieved / peaks["hbm_gbs"], 4),
-                         "traffic": decode_traffic() if args.workload == WORKLOAD else None,
-                         "kernel": "decode calls of the step (plan + decode_tc + combine"
-                                   + (", twice, + merge_lse)" if wl.n_local else ")"),
-                         "peak_source": src},
+            "roofline": decode_roofline(
+                decode_flops(wl, inp.n_rows, inp.n_gather), cache_bytes, t_dec, peaks, src,
+                decode_traffic() if args.workload == WORKLOAD else None,
+                "decode calls of the step (plan + decode_tc + combine"
+                + (", twice, + merge_lse)" if wl.n_local else ")")),
             "clocks": clocks,
             "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},

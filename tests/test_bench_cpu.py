@@ -32,3 +32,27 @@ def test_reference_arm_prints_one_contract_line():
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_decode_flops_and_roofline_bound():
+    # FLOPs per step: 2 * s_q * heads * rows * (512 + 64 + 512); the 256K
+    # two-token case sits above the measured ridge (bf16 peak / HBM copy
+    # rate) and is reported against the tensor peak, the others against HBM
+    sys.path.insert(0, ROOT)
+    import bench
+    from head_latent_attention_02_b200.workloads import WORKLOADS
+    peaks = {"hbm_gbs": 6543.4, "bf16_tflops": 1623.7}
+    cases = [("bf16_b16_4k", [4096] * 16, None, 18_253_611_008, "hbm"),
+             ("bf16_long_256k", [262144] * 2, None, 292_057_776_128, "tensor"),
+             ("redknot_56_8", [24576], [256], 2 * 1088 * (8 * 24576 + 56 * 256), "hbm")]
+    for name, rows, ng, flops, bound in cases:
+        wl = WORKLOADS[name]
+        assert bench.decode_flops(wl, rows, ng) == flops
+        cb = (sum(rows) + (sum(ng) if ng else 0)) * 1152
+        r = bench.decode_roofline(flops, cb, 0.05, peaks, "measured", None, "k")
+        assert r["bound"] == bound
+        if bound == "hbm":
+            assert r["unit"] == "GB/s" and r["achieved"] == round(cb / 0.05e-3 / 1e9, 1)
+        else:
+            assert r["unit"] == "TFLOP/s" and r["achieved"] == round(flops / 0.05e-3 / 1e12, 1)
+        assert r["frac"] == round(r["achieved"] / r["peak"], 4)
