@@ -572,3 +572,40 @@ def test_redknot_head_row_ceilings():
         assert round(100 * c, 2) == pr["ceiling_percent"], pr["name"]
     # the 56/8 split of the RedKnot config is the Flash profile's
     assert O.head_row_ceiling(56, 8, 1, 1) == 0.875
+
+
+def test_channel_scales_fold_into_query_and_output():
+    # with one scale per channel, attention over the dequantised cache equals
+    # attention over the raw integer codes with the scales folded into the
+    # absorbed query (content and rotary parts) and into the weighted latent
+    inp = _tiny(s_q=2, lengths=(13, 70))
+    wl = inp.wl
+    g = np.random.default_rng(41)
+    sc, sr = g.uniform(0.2, 0.6, wl.d_c), g.uniform(0.2, 0.6, wl.d_r)
+    pool = inp.pool.astype(np.float64)
+    used = ~np.isnan(pool).any(-1)
+    codes = np.full_like(pool, np.nan)
+    codes[used, :wl.d_c] = O.quantize_symmetric(pool[used, :wl.d_c], sc, 4)
+    codes[used, wl.d_c:] = O.quantize_symmetric(pool[used, wl.d_c:], sr, 4)
+    deq = np.full_like(pool, np.nan)
+    deq[used, :wl.d_c] = codes[used, :wl.d_c] * sc
+    deq[used, wl.d_c:] = codes[used, wl.d_c:] * sr
+    inp.pool = deq
+    o_ref, l_ref = O.decode_absorbed_fast(inp)
+    # integer codes are exact in bf16 (|code| <= 8)
+    assert np.array_equal(codes[used], np.round(codes[used])) and np.abs(codes[used]).max() <= 8
+    for b in range(wl.B):
+        rows, kpos, ver = O.sequence_rows(inp.segs[b])
+        cc = O.gather_cache(codes, inp.block_table[b], rows)
+        for j in range(wl.s_q):
+            qi = b * wl.s_q + j
+            p = int(inp.q_pos[qi])
+            q_lat = np.einsum("hn,hnc->hc", inp.q_nope[qi].astype(np.float64),
+                              inp.w_uk.astype(np.float64)) * sc          # scale into the query
+            q_r = O.rope_rotate(inp.q_rope[qi].astype(np.float64), p, wl.rope_base) * sr
+            s = wl.scale * (q_lat @ cc[:, :wl.d_c].T + q_r @ cc[:, wl.d_c:].T)
+            s = np.where((kpos <= p)[None, :], s, -np.inf)
+            a, lse = O.softmax_lse(s)
+            o = (a @ cc[:, :wl.d_c]) * sc                                  # scale after the sum
+            assert np.allclose(o, o_ref[qi], rtol=0, atol=1e-12)
+            assert np.allclose(lse, l_ref[qi], rtol=0, atol=1e-12)
