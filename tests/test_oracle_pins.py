@@ -609,3 +609,28 @@ def test_channel_scales_fold_into_query_and_output():
             o = (a @ cc[:, :wl.d_c]) * sc                                  # scale after the sum
             assert np.allclose(o, o_ref[qi], rtol=0, atol=1e-12)
             assert np.allclose(lse, l_ref[qi], rtol=0, atol=1e-12)
+
+
+def test_qknorm_one_factor_per_column_with_prescaled_rotary_keys():
+    # if the cache writer stores rms_t * k_rope_t, the QK-normed score is one
+    # 576-wide product against the stored row times the token's inverse RMS:
+    # scale * inv_t * (q_w . c_t + q_r . (rms_t k_rope_t))
+    inp = _tiny(B=1, s_q=1, lengths=None, prefix=64, doc=45)
+    wl = inp.wl
+    g_q, g_k = _qk_weights(inp)
+    rows, kpos, ver = O.sequence_rows(inp.segs[0])
+    cache = O.gather_cache(inp.pool, inp.block_table[0], rows)
+    c, k_rope = cache[:, :wl.d_c], cache[:, wl.d_c:]
+    shift = np.asarray(inp.deltas, np.int64)[ver]
+    p = int(inp.q_pos[0])
+    ref = O.qknorm_scores_absorbed(inp.q_nope[0], inp.q_rope[0], p, inp.w_uk, c, k_rope, shift,
+                                   g_q, g_k, wl.scale, wl.rope_base)
+    inv = O.key_inv_rms(c, inp.w_uk)
+    stored = np.concatenate([c, k_rope / inv[:, None]], 1)          # rms_t * k_rope_t
+    q_hat = O.rms_norm(inp.q_nope[0].astype(np.float64).reshape(-1), g_q).reshape(wl.H, wl.d_n)
+    q_lat = np.einsum("hn,hnc->hc", q_hat * g_k.reshape(wl.H, wl.d_n), inp.w_uk.astype(np.float64))
+    q_r = O.rope_rotate(inp.q_rope[0].astype(np.float64)[:, None, :],
+                        (p - shift)[None, :], wl.rope_base)           # [H, T, d_r]
+    s = wl.scale * inv[None, :] * (q_lat @ stored[:, :wl.d_c].T
+                                   + np.einsum("htd,td->ht", q_r, stored[:, wl.d_c:]))
+    assert np.allclose(s, ref, rtol=0, atol=1e-11)
