@@ -1,46 +1,49 @@
-// decode_tc.cuh -- absorbed MLA decode on sm_100a tensor cores (CTA pairs).
+// decode_tc.cuh -- absorbed MLA decode on sm_100a tensor cores.
 //
 // What it computes (Day 27 tutorial "Multi-Head Latent Attention", sections
 // "Move the Key Projection Into the Query", "Position Rotations Complicate
 // the Absorption", "Move the Value Expansion After the Weighted Sum"): for
-// 128 query rows (one query token x up to 128 heads) and every cached row t,
-//     S[m, t] = scale * (q_abs[m, :512] . c_t + q_abs[m, 512:] . k_rope_t)
-//     P = online-softmax(S masked by key_pos(t) <= q_pos),  O[m, :] = sum_t P[m,t] c_t
+// the (up to) 128 head rows of one query token and every cached row t,
+//     S[h, t] = scale * (q_abs[h, :512] . c_t + q_abs[h, 512:] . k_rope_t)
+//     P = online-softmax(S masked by key_pos(t) <= q_pos),  O[h, :] = sum_t P[h,t] c_t
 // reading each 576-element latent row [c_t | k_rope_t] from HBM once.
 //
-// Decomposition.  A cluster of two CTAs on two SMs shares one tcgen05 MMA
-// (cta_group::2): CTA r holds the query rows of heads [64r, 64r + 64) and the
-// cache rows of page 2k + r of a 128-row tile; the pair computes the full
-// 128 x 128 score tile (N=128 MMAs accumulated over two column stages of the
-// pages), each CTA receiving its 64 head rows in TMEM (tokens 0-63 in lanes
-// 0-63, tokens 64-127 in lanes 64-127 of the same columns).  The softmax of
-// a head row is shared by lanes t and t + 64 (the row max is combined
-// through shared memory).  P . c runs as M=128 x N=256 pair MMAs; in MMA nb
-// CTA r supplies latent columns [256 r + 128 nb, +128) for all 128 rows
-// (re-read through L2), so each CTA's value columns are one contiguous half
-// and O for its 64 heads lies in 256 TMEM columns with latent [0, 256) in
-// lanes 0-63 and [256, 512) in lanes 64-127.  No scores or probabilities
-// cross between the SMs: only the MMA operands do, inside the pair
-// instruction.
+// Decomposition.  Every tensor-core product runs with 128 rows per SM, the
+// shape at which tcgen05 reaches its full rate (64 rows per SM run at half
+// rate), and the two products live on the two CTAs of a cluster:
+//   - the score CTA (rank 0) holds the 128 heads' absorbed queries: the 512
+//     latent columns in tensor memory (the A operand of the score MMAs, copied
+//     in by tcgen05.cp) and the 64 rotary columns in shared memory.  It
+//     streams each 128-row tile of cache rows through a ring of 64-column
+//     panels and computes S = Q . [c | k_rope]^T as M=128 x N=128 MMAs into a
+//     double-buffered accumulator.  Its softmax threads own one head row each
+//     (lane = head; two warps split a row's 128 columns and exchange only
+//     the row max).  They store P in bf16, with the per-row rescale factors,
+//     straight into the value CTA's shared memory, then make those writes
+//     visible to its tensor core with a cluster-scope async-proxy fence and
+//     a release arrival on its barrier.
+//   - the value CTA (rank 1) holds O = P . c for the 128 heads in all 512
+//     tensor-memory columns.  It streams the same tile's latent columns again
+//     (an L2 hit: the score CTA fetched them moments before) one page at a
+//     time and issues M=128 x N=256 MMAs with P as the A operand.  Its four
+//     epilogue warps apply the occasional rescale of O and write the result.
+// Work is split over clusters as contiguous runs of (sequence, query token,
+// head block, tile) units; a cluster writes the final result of a stream it
+// covers entirely, else a normalised partial (o, lse) that the combine kernel
+// merges.
 //
-// Loads.  Full rows are fetched with multi-dimensional TMA boxes so that each
-// request covers long contiguous row runs: a score stage is one box of 64
-// cache rows x 5 or 4 64-column panels (640/512-byte runs), a value stage
-// one box of 32 rows x this CTA's four latent panels (512-byte runs, 16 KB),
-// Q one box of 64 rows x 9 panels.  Partial pages and gathered rows use
-// per-panel boxes of power-of-two heights, and rows without data come from
-// boxes placed past the end of the cache, which the hardware fills with
-// zeros.  The own-page rows of the next two tiles are prefetched into L2.
+// Loads.  The score MMA needs both pages of a tile in each 64-column panel
+// (N = 128 rows; 64-row MMAs issue no faster than 128-row ones), so a score
+// stage is three such panels.  When the two pages sit next to each other in
+// the pool the stage is one 3-D box; otherwise each page-panel is its own box,
+// which the TMA unit serves at about half the rate (a fixed cost per box).
+// A value slot is one page's 8 latent panels (one 3-D box).  Rows without
+// data (past a sequence's end, behind a bad page id) come from boxes placed
+// past the end of the cache, which the hardware fills with zeros, so NaN in
+// unused rows never reaches a product.  Gathered rows (attended through a
+// gather list) arrive as four-row gather boxes.
 //
-// Roles per CTA (224 threads): warp 0 streams Q and the score stages, warp 6
-// the value stages (TMA), warp 1 of CTA 0 issues every MMA of the pair from
-// per-tile flags precomputed in shared memory, warps 2-5 own one TMEM lane
-// each for softmax and the epilogue (each CTA forwards one softmax-done
-// arrival per tile to the issuer).  Work is split over CTA pairs as
-// contiguous runs of (sequence, head block, tile) units -- runs that never
-// straddle two sequences when all have the same length; a pair writes the
-// final result of a sequence it covers entirely, else a normalised partial
-// (o, lse) that the combine kernel merges.
+// Every wait is bounded and records MLA_ERR_TIMEOUT when it gives up.
 #pragma once
 #include <cuda.h>
 
@@ -51,65 +54,75 @@ namespace mla {
 namespace tc {
 
 constexpr int kDc = 512, kDr = 64, kRow = kDc + kDr;
-constexpr int kM = 128;                  // query rows of the pair
-constexpr int kMh = 64;                  // query rows per CTA
-constexpr int kT = 128;                  // cache rows per tile (two pages)
+constexpr int kM = 128;                  // head rows of a stream (MMA M)
+constexpr int kT = 128;                  // cache rows per tile (two pages; score MMA N)
 constexpr int kPg = 64;                  // rows per page
-constexpr int kR = 32;                   // cache rows per value stage
-constexpr int kQPanels = 9;              // 8 latent + 1 rotary 64-column panels
-constexpr int kQPanel = kMh * 128;       // 64 rows x 128 B = 8 KB
-constexpr int kSPanel = kR * 128;        // 32 rows x 128 B = 4 KB
-constexpr int kKPanel = kPg * 128;       // 64 rows x 128 B = 8 KB
-// Score stages split a page's rows by columns: stage 0 holds panels 0-4 and
-// stage 1 panels 5-8 of all 64 rows, so each score MMA spans the page (N=128
-// for the pair) and the two stages of a tile alternate between fixed slots.
-constexpr int kKSplit = 5;                              // panels in stage 0
-constexpr int kKStage0 = kKSplit * kKPanel;             // 40 KB
-constexpr int kKStage1 = (kQPanels - kKSplit) * kKPanel;  // 32 KB
-constexpr int kVStage = 4 * kSPanel;          // 16 KB: 32 rows x this CTA's 4 latent panels
-constexpr int kKStages = 2, kVStages = 3;
-constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQPanels * kQPanel;
-constexpr int kOffV = kOffK + kKStage0 + kKStage1;
-constexpr int kOffP = kOffV + kVStages * kVStage;
-constexpr int kPBuf = 2 * kQPanel;       // 64 rows x 128 tokens bf16 (two 64-token panels)
-constexpr int kOffMisc = kOffP + 2 * kPBuf;
-constexpr int kMiscBytes = 1536;
-constexpr int kOffBar = kOffMisc + kMiscBytes;
-constexpr int kBarBytes = 512;
+constexpr int kPanels = 9;               // 64-column panels of a row: 8 latent + 1 rotary
+constexpr int kSlot = kT * 128;          // score panel: 128 rows x 128 B = 16 KB
+constexpr int kStagePanels = 3;          // score ring stage: three panels (one 3-D box when
+constexpr int kStage = kStagePanels * kSlot;   //   both pages of the tile are adjacent)
+constexpr int kNStages = 4;              // score-side ring stages (192 KB)
+constexpr int kVPage = 8 * kPg * 128;    // value slot: one page's 8 latent panels = 64 KB
+constexpr int kNV = 2;                   // value-side ring slots
+constexpr int kPBuf = 2 * kM * 128;      // P: 128 rows x 128 tokens bf16, two 64-token panels
+constexpr int kHdrFlag = 512;            // header after P: rescale factor per row (512 B),
+constexpr int kMsgStride = 33 * 1024;    //   then one flag word per softmax warp
+constexpr int kEndBytes = 1536;          // per stream end: row sums of both halves, row max
+constexpr int kStageWarp = 32 * 128;     // epilogue staging: 32 rows x 32 floats per warp
+// score CTA
+constexpr int kOffRing = 0;
+constexpr int kOffQr = kOffRing + kNStages * kStage;           // rotary query panel
+constexpr int kOffMax = kOffQr + kSlot;                        // row-max exchange [2][2][128]
+constexpr int kEndScore = kOffMax + 2 * 2 * kM * 4;
+// value CTA
+constexpr int kOffVal = 0;
+constexpr int kOffMsg = kOffVal + kNV * kVPage;                // two incoming P messages
+constexpr int kOffEnd = kOffMsg + 2 * kMsgStride;
+constexpr int kOffStage = kOffEnd + 2 * kEndBytes;
+constexpr int kEndValue = kOffStage + 4 * kStageWarp;
+// unit descriptors, then barriers, at the same offsets in both CTAs (commits
+// multicast to both)
+constexpr int kOffDesc = kEndScore > kEndValue ? kEndScore : kEndValue;
+constexpr int kOffBar = kOffDesc + 64 * 32;
+constexpr int kBarBytes = 1024;
 constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;   // + alignment slack
-constexpr int kThreads = 224;
+// warp 0 loads, warp 1 issues MMAs; score CTA: warps 2-9 run the softmax (two
+// per TMEM lane quarter, one 64-column half of the tile each); value CTA:
+// warps 2-5 rescale O and write it out, warps 6-9 have no role; warp 10 of
+// both computes the unit descriptors
+constexpr int kThreads = 352;
+constexpr int kProducerWarp = 10;
+constexpr int kSoftWarps = 8;
 constexpr int kTmemCols = 512;
-constexpr int kColO = 0, kColS = 256;
+constexpr int kColQ = 0, kColS = 256;    // score CTA: Q latent (256 columns), S double buffer
 constexpr int kMinChunk = 2;
 constexpr int kPlanThreads = 1024;       // planner block (one CTA)
-constexpr int kPrefetchTiles = 2;        // tiles of own-page rows requested into L2 ahead
-constexpr int kFlagTiles = 256;          // per-tile issue flags precomputed in shared memory
 constexpr int kNumBoxHeights = 6;        // 32, 16, 8, 4, 2, 1 rows
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: lazy rescale margin
-constexpr int kStoreCols = 32;           // fp32 columns per output store box (128 B)
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kOffMsg % 1024 == 0 && kMsgStride % 1024 == 0 && kSlot % 1024 == 0 &&
+              kVPage % 1024 == 0 && kPBuf + kHdrFlag + 4 * kSoftWarps <= kMsgStride,
+              "swizzle alignment and message size");
 
 struct PlanHeader {
   int U, C, G, n_streams;
 };
 
-// TMA descriptors (all 64 columns wide, 128-byte swizzle):
-//   q   3-D (col, q_abs row, panel): 64 rows x 9 panels of one head block
-//   k0  3-D (col, cache row, panel): 64 rows x panels 0-4 (score stage 0)
-//   k1  3-D (col, cache row, panel): 64 rows x panels 5-8 (score stage 1)
-//   v   3-D (col, cache row, panel): 32 rows x 4 panels (one latent half)
-//   row 2-D (col, cache row): boxes of 32 >> i rows (i = 0..5) for partial
-//       pages, gathered rows and zero rows past the end of the cache
-// and two fp32 store maps (32 columns x 32 rows, 128-byte swizzle):
-//   o   3-D (col, head - h0, query row) over o_lat: heads past n_h are
-//       clipped by the map, so a store never reaches another head range
-//   part 2-D (col, slot row) over the split partials [2G x 128, 512]
+// TMA descriptors (64 columns wide, 128-byte swizzle):
+//   q3   3-D (col, q_abs row, panel), box {64, 128, 3}: three panels of a head block
+//   qr   2-D (col, q_abs row), box {64, 128}: the rotary panel of a head block
+//   k3   3-D (col, cache row, panel), box {64, 128, 3}: three panels of two
+//        physically adjacent pages (one score stage)
+//   kp   2-D (col, cache row), box {64, 64}: one panel of a page
+//   row  2-D (col, cache row), boxes of 32 >> i rows (i = 0..5) for partial
+//        pages and zero rows past the end of the cache
+//   vp   3-D (col, cache row, panel), box {64, 64, 8}: a page's latent panels
+//   g4   2-D (col, cache row), box {64, 1}: four-row gathers
 struct Maps {
-  CUtensorMap q, k0, k1, v;
+  CUtensorMap q3, qr, k3, kp;
   CUtensorMap row[kNumBoxHeights];
-  CUtensorMap o, part;
+  CUtensorMap vp, g4;
 };
 
 struct Params {
@@ -118,8 +131,9 @@ struct Params {
   int G;
   const PlanHeader* plan;
   const int* stream_off;
-  const int* pair_stream;  // stream holding the first unit of each pair's run
-  float* partial_lse;     // [2G x 128] (the rows live behind the part map)
+  const int* pair_stream;  // stream holding the first unit of each cluster's run
+  float* partial;          // [2G x 128, 512] normalised split partials
+  float* partial_lse;      // [2G x 128]
   float scale_log2;
 };
 
@@ -281,80 +295,7 @@ __device__ __forceinline__ StreamPos stream_pos(const Params& p, int s) {
   return r;
 }
 
-// Issue flags of unit u of a pair's run starting at u0: bit 0, the unit opens
-// a stream; bit 1, it needs another query panel (new stream or relocation
-// version).  The same decisions as the query loader's.
-template <bool kGather>
-__device__ __forceinline__ uint32_t unit_flags(const Params& p, int u, int u0, int s_lo) {
-  const int n_streams = p.plan->n_streams;
-  const int s = stream_of(p.stream_off, n_streams, u, s_lo);
-  const int ver = tile_version<kGather>(p.a, stream_pos(p, s).b, u - p.stream_off[s]);
-  if (u == u0) return 3u;
-  const int sp = stream_of(p.stream_off, n_streams, u - 1, s_lo);
-  if (sp != s) return 3u;
-  return tile_version<kGather>(p.a, stream_pos(p, sp).b, u - 1 - p.stream_off[sp]) != ver ? 2u
-                                                                                       : 0u;
-}
-
-// ----------------------------------------------------------------- barriers
-struct Bars {
-  uint64_t kfull[kKStages], kempty[kKStages];
-  uint64_t vfull[kVStages], vempty[kVStages];
-  uint64_t q_full, q_empty;
-  uint64_t s_full[2], p_empty[2];
-  // softmax of tile t done (S read, P written) in both CTAs: one arrival per
-  // CTA, forwarded after the CTA's four softmax warps met on sm_local
-  uint64_t sp_done[2], sm_local[2];
-  uint64_t o_done[2], o_free;       // o_done[t & 1]: P.c of tile t complete
-  uint64_t mma_drain;
-  uint64_t k_started;               // this CTA's first query and score loads are issued
-  uint64_t row_sync[2], l_sync;     // the 128 softmax threads of one CTA
-  uint32_t tmem_base;
-  uint8_t tflags[kFlagTiles];       // unit_flags of the pair's tiles (runs <= kFlagTiles)
-};
-static_assert(sizeof(Bars) <= kBarBytes, "barrier block too large");
-
-__device__ __forceinline__ void fail(bool& ok) {
-  if (ok) set_status(MLA_ERR_TIMEOUT);
-  ok = false;
-}
-
-// Bounded waits whose outcome is the same for every lane of the warp, so a
-// timeout makes the whole warp leave together.
-__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity));
-}
-__device__ __forceinline__ bool wait_warp_cluster(uint64_t* bar, uint32_t parity) {
-  return __all_sync(0xffffffffu, mbar_wait_cluster(bar, parity));
-}
-
-// Arrive on a barrier of the pair's rank-0 CTA (local or remote).
-__device__ __forceinline__ void arrive_leader(uint64_t* bar, uint32_t rank) {
-  if (rank == 0) mbar_arrive(bar);
-  else mbar_arrive_cluster_addr(mapa(smem_u32(bar), 0));
-}
-
-// Fill smem rows [r0, r0 + n) (pitch 128 B, n <= 64) of one 64-column panel
-// from cache rows starting at y, as power-of-two boxes.  A y at or past the end of
-// the cache (oob) makes the hardware fill the rows with zeros, so rows
-// without data read as 0 in the P.c product without any generic-proxy store.
-__device__ __forceinline__ void load_rows(uint8_t* dst, const Maps& mp, uint32_t bar, int x,
-                                          long long y, int r0, int n) {
-  int r = r0;
-  for (; n - (r - r0) > kR; r += kR)   // n <= 64: at most one leading full box
-    tma_load_2d_pair(dst + r * 128, &mp.row[0], bar, x, (int)(y + (r - r0)));
-  n -= r - r0;
-#pragma unroll 1
-  for (int hb = 0; hb < kNumBoxHeights; ++hb) {
-    const int h = kR >> hb;
-    if (n & h) {
-      tma_load_2d_pair(dst + r * 128, &mp.row[hb], bar, x, (int)(y + (r - r0)));
-      r += h;
-    }
-  }
-}
-
-// Gathered rows i0 + 32 k (k < N; those at or past n are absent) of sequence
+// Gathered rows i0 + kStride k (k < N; those at or past n are absent) of sequence
 // b: physical cache row (y_oob when absent or unlocatable) and request
 // position (INT32_MAX likewise).  Every index, segment and block-table load of
 // the N rows is issued before any result is used, so a lane pays about one
@@ -363,7 +304,7 @@ __device__ __forceinline__ void load_rows(uint8_t* dst, const Maps& mp, uint32_t
 // in a segment; a bad page id records MLA_ERR_BAD_INDEX and reads as zeros.
 // Not inlined: only gathered tiles call it, and the loader loop of page tiles
 // stays as compact as it is without it.
-template <int N>
+template <int N, int kStride>
 __device__ __noinline__ void locate_gathered(const DecodeArgs& a, int b, int i0, int n,
                                                 long long y_oob, long long* phys, int* kpos) {
   const mla_seg_t* sg = a.segs + (size_t)b * a.max_segs;
@@ -371,7 +312,7 @@ __device__ __noinline__ void locate_gathered(const DecodeArgs& a, int b, int i0,
   bool in[N];
 #pragma unroll
   for (int k = 0; k < N; ++k) {
-    row[k] = i0 + 32 * k < n ? a.gather_rows[(size_t)b * a.max_gather + i0 + 32 * k] : 0;
+    row[k] = i0 + kStride * k < n ? a.gather_rows[(size_t)b * a.max_gather + i0 + kStride * k] : 0;
     seg[k] = -1;
   }
   for (int s = 0; s < a.max_segs; ++s) {
@@ -382,7 +323,7 @@ __device__ __noinline__ void locate_gathered(const DecodeArgs& a, int b, int i0,
   }
 #pragma unroll
   for (int k = 0; k < N; ++k) {
-    const bool present = i0 + 32 * k < n;
+    const bool present = i0 + kStride * k < n;
     in[k] = present && seg[k] >= 0 && row[k] / kPage < a.max_pages;
     page[k] = in[k] ? a.block_table[(size_t)b * a.max_pages + row[k] / kPage] : -1;
     if (present && !in[k]) set_status(MLA_ERR_BAD_INDEX);
@@ -400,32 +341,121 @@ __device__ __noinline__ void locate_gathered(const DecodeArgs& a, int b, int i0,
   }
 }
 
-// Visibility of the 64 tile rows [64 half, +64) of tile t for a query at q_pos
-// qp, as a bitmask (bit i: row 64 half + i exists and key_pos <= qp).  Page
-// rows have consecutive key positions, so the mask is a prefix; gathered rows
-// are located two per lane and combined by ballot.
-__device__ __noinline__ uint64_t gather_visible(const DecodeArgs& a, const Tile& t, int b, int half,
-                                               int qp, int lane) {
-  long long ph[2];
-  int kp[2];
-  locate_gathered<2>(a, b, t.g0 + kPg * half + lane, t.g0 + t.n_rows, 0, ph, kp);
-  const uint32_t lo = __ballot_sync(0xffffffffu, kp[0] <= qp);
-  const uint32_t hi = __ballot_sync(0xffffffffu, kp[1] <= qp);
-  return (uint64_t)lo | ((uint64_t)hi << 32);
+// ----------------------------------------------------------------- unit descriptors
+// Everything a role needs about one unit (stream, tile) of a cluster's run,
+// computed ahead of time by the producer warp so that no role waits on a chain
+// of global loads (stream offsets, segments, block table, query position) in
+// its per-tile loop.
+constexpr uint32_t kFirst = 1, kLast = 2, kNewQ = 4, kWhole = 8, kSlot1 = 16;
+struct Desc {
+  int s, k;            // stream, tile within the stream
+  int phys0, phys1;    // page mode: physical row of each page's row 0
+  int kpos0, kpos1;    // page mode: request position of each page's row 0
+  int qp;              // the stream's query position
+  uint8_t nv0, nv1;    // page mode: valid rows of each page; gather mode: nv0 = rows in the tile
+  uint8_t ver;         // relocation version (selects the query panel)
+  uint8_t flags;       // kFirst / kLast: first / last tile of its stream in this run;
+                       // kNewQ: needs another query panel; kWhole: the run covers the
+                       // whole stream; kSlot1: the partial goes to the run's second slot
+};
+static_assert(sizeof(Desc) == 32, "descriptor size");
+constexpr int kDescRing = 64;            // entries, filled in batches of 32 (one per lane)
+
+// ----------------------------------------------------------------- barriers
+struct Bars {
+  // score CTA
+  uint64_t ring_full[kNStages], ring_empty[kNStages];
+  uint64_t qr_full, qr_empty, q_drain;
+  uint64_t s_full[2], s_empty[2];
+  uint64_t end_empty[2];              // stream-end message slot free (4 remote arrivals)
+  uint64_t row_sync[2][4];            // per lane quarter: both halves published the row max
+  // both CTAs: P.c of tile t complete (in the score CTA: P buffer t & 1 free)
+  uint64_t pv[2];
+  // value CTA
+  uint64_t v_full[kNV], v_empty[kNV];
+  uint64_t p_full[2];                 // P message of tile t landed (8 arrivals + bytes)
+  uint64_t o_ok[2];                   // tile t may start its P.c (rescale or epilogue done)
+  uint64_t end_full[2];               // stream-end message landed (8 arrivals + bytes)
+  // both CTAs: descriptor batches
+  uint64_t d_full[2], d_empty[2];
+  uint64_t mma_drain;
+  uint32_t tmem_base;
+  int n_units;                        // units in this cluster's run
+};
+static_assert(sizeof(Bars) <= kBarBytes, "barrier block too large");
+
+__device__ __forceinline__ void fail(bool& ok) {
+  if (ok) set_status(MLA_ERR_TIMEOUT);
+  ok = false;
 }
 
+// Bounded waits whose outcome is the same for every lane of the warp, so a
+// timeout makes the whole warp leave together.
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+}
+__device__ __forceinline__ bool wait_warp_cluster(uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_wait_cluster(bar, parity));
+}
+
+// Descriptor ring: unit `it` is entry it % 64.  A consumer waits for the batch
+// holding it when it reaches the batch's first entry (batch 0 was waited for
+// before the loop) and releases the batch after its last entry.
+__device__ __forceinline__ bool desc_wait(Bars* bar, int it, bool warp_wide) {
+  if (it == 0 || (it & 31) != 0) return true;
+  const int bt = it >> 5;
+  return warp_wide ? wait_warp(&bar->d_full[bt & 1], (bt >> 1) & 1)
+                   : mbar_wait(&bar->d_full[bt & 1], (bt >> 1) & 1);
+}
+__device__ __forceinline__ void desc_done(Bars* bar, int it, int n, bool arrive) {
+  if (arrive && ((it & 31) == 31 || it == n - 1)) mbar_arrive(&bar->d_empty[(it >> 5) & 1]);
+}
+
+// Fill smem rows [r0, r0 + n) (pitch 128 B, n <= 64) of one 64-column panel
+// from cache rows starting at y, as power-of-two boxes.  A y at or past the
+// end of the cache makes the hardware fill the rows with zeros.
+__device__ __forceinline__ void load_rows(uint8_t* dst, const Maps& mp, uint64_t* bar, int x,
+                                          long long y, int r0, int n) {
+  int r = r0;
+  for (; n - (r - r0) > 32; r += 32)     // n <= 64: at most one leading full box
+    tma_load_2d(dst + r * 128, &mp.row[0], bar, x, (int)(y + (r - r0)));
+  n -= r - r0;
+#pragma unroll 1
+  for (int hb = 0; hb < kNumBoxHeights; ++hb) {
+    const int h = 32 >> hb;
+    if (n & h) {
+      tma_load_2d(dst + r * 128, &mp.row[hb], bar, x, (int)(y + (r - r0)));
+      r += h;
+    }
+  }
+}
+
+// Visibility of 64 tile rows [64 hf, 64 hf + 64) for the unit's query (bit i:
+// row 64 hf + i exists and key_pos <= qp).  Page rows have consecutive key
+// positions, so each page's mask is a prefix; gathered rows are located one
+// per lane and combined by ballot.
 template <bool kGather>
-__device__ __forceinline__ uint64_t visible_rows(const DecodeArgs& a, const Tile& t, int b,
-                                                 int half, int qp, int lane) {
-  if constexpr (kGather) return gather_visible(a, t, b, half, qp, lane);
-  const int n = min(half_rows(t, half), max(0, qp - half_kpos(t, half) + 1));
-  return n >= 64 ? ~0ull : ((1ull << n) - 1ull);
+__device__ __forceinline__ uint64_t visibility(const DecodeArgs& a, const Desc& d, int b, int hf,
+                                               int lane) {
+  if constexpr (kGather) {
+    long long ph[2];
+    int kp[2];
+    const int g0 = d.k * kT;
+    locate_gathered<2, 32>(a, b, g0 + kPg * hf + lane, g0 + d.nv0, 0, ph, kp);
+    const uint32_t lo = __ballot_sync(0xffffffffu, kp[0] <= d.qp);
+    const uint32_t hi = __ballot_sync(0xffffffffu, kp[1] <= d.qp);
+    return (uint64_t)lo | ((uint64_t)hi << 32);
+  } else {
+    const int nv = hf ? d.nv1 : d.nv0, kp = hf ? d.kpos1 : d.kpos0;
+    const int n = max(0, min(nv, d.qp - kp + 1));
+    return n >= 64 ? ~0ull : ((1ull << n) - 1ull);
+  }
 }
 
-// Rescale this warp's 32 TMEM lanes of O (256 columns) by f.
+// Rescale this warp's 32 lanes of O (all 512 columns) by f.
 __device__ __noinline__ void scale_o(uint32_t taddr, float f) {
 #pragma unroll 1
-  for (int c = 0; c < 256; c += 32) {
+  for (int c = 0; c < 512; c += 32) {
     float ov[32];
     tmem_ld32(taddr + c, ov);
     tmem_wait_ld();
@@ -436,6 +466,73 @@ __device__ __noinline__ void scale_o(uint32_t taddr, float f) {
   tmem_wait_st();
 }
 
+// Producer: the descriptors of units u0 + base + lane (lane < cnt), one per
+// lane, with the loads of the whole batch in flight together.  `cs` is the
+// stream of the batch's first unit; `ps` / `pv` are the stream and version of
+// the unit before the batch (-1 for none); all three carry to the next batch.
+template <bool kGather>
+__device__ __forceinline__ Desc produce(const Params& p, int u0, int u1, int base, int cnt,
+                                        int& cs, int& ps, int& pv, int lane) {
+  const DecodeArgs& a = p.a;
+  const int n_streams = p.plan->n_streams;
+  const int u = u0 + base + lane;
+  const bool live = lane < cnt;
+  // The stream holding u is the last stream whose offset is <= u.  Windows of
+  // 32 offsets from cs on (overlapping by one); a lane is resolved once the
+  // offset after its candidate is > u.
+  int s = -1, off = 0, off_next = 0;
+  for (int ws = cs, guard = 0; guard < (1 << 16); ws += 31, ++guard) {
+    const int o = ws + lane <= n_streams ? p.stream_off[ws + lane] : INT_MAX;
+    int le = 0;
+#pragma unroll 8
+    for (int j = 0; j < 32; ++j) le += (__shfl_sync(0xffffffffu, o, j) <= u) ? 1 : 0;
+    const int jm = max(le - 1, 0);
+    const int o_j = __shfl_sync(0xffffffffu, o, jm);
+    const int o_n = __shfl_sync(0xffffffffu, o, min(jm + 1, 31));
+    if (live && s < 0 && jm < 31 && o_n > u) {
+      s = ws + jm;
+      off = o_j;
+      off_next = o_n;
+    }
+    if (__all_sync(0xffffffffu, !live || s >= 0)) break;
+  }
+  Desc d;
+  d.s = max(s, 0);
+  d.k = u - off;
+  const StreamPos sp = stream_pos(p, d.s);
+  const int qi = sp.b * a.s_q + sp.j;
+  d.qp = live ? a.q_pos[qi] : 0;
+  Tile t = {};
+  if (live) t = describe<kGather>(a, sp.b, d.k);
+  d.phys0 = (int)t.phys0;
+  d.phys1 = (int)t.phys1;
+  d.kpos0 = t.kpos0;
+  d.kpos1 = t.kpos1;
+  d.nv0 = (uint8_t)(kGather ? t.n_rows : t.nv0);
+  d.nv1 = (uint8_t)t.nv1;
+  d.ver = (uint8_t)t.ver;
+  const int T = off_next - off;
+  uint32_t f = 0;
+  if (u == u0 || d.k == 0) f |= kFirst;
+  if (u == u1 - 1 || d.k == T - 1) f |= kLast;
+  int s_prev = __shfl_up_sync(0xffffffffu, d.s, 1);
+  int v_prev = __shfl_up_sync(0xffffffffu, (int)d.ver, 1);
+  if (lane == 0) {
+    s_prev = ps;
+    v_prev = pv;
+  }
+  if (d.s != s_prev || (int)d.ver != v_prev) f |= kNewQ;
+  if (off >= u0 && off + T <= u1) f |= kWhole;
+  if (off > u0) f |= kSlot1;
+  d.flags = (uint8_t)f;
+  // carry to the next batch: the last live unit's stream and version
+  const int last = max(cnt - 1, 0);
+  cs = __shfl_sync(0xffffffffu, d.s, last);
+  ps = cs;
+  pv = __shfl_sync(0xffffffffu, (int)d.ver, last);
+  return d;
+}
+
 // ----------------------------------------------------------------- kernel
 template <bool kGather>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -443,487 +540,538 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem + kOffQ;
-  uint8_t* sK = smem + kOffK;
-  uint8_t* sV = smem + kOffV;
-  uint8_t* sP = smem + kOffP;
-  float* sMax = reinterpret_cast<float*>(smem + kOffMisc);         // [2][128]
-  float* sL = sMax + 2 * kM;                                       // [128]
   Bars* bar = reinterpret_cast<Bars*>(smem + kOffBar);
-
+  Desc* ring_d = reinterpret_cast<Desc*>(smem + kOffDesc);
   const DecodeArgs& a = p.a;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
+  const uint32_t rank = cluster_ctarank();   // 0: scores and softmax; 1: P.c and output
   const int g = blockIdx.x >> 1;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kKStages; ++i) {
-      mbar_init(&bar->kfull[i], 1);    // rank 0 arms both CTAs' bytes
-      mbar_init(&bar->kempty[i], 1);
+    for (int i = 0; i < kNStages; ++i) {
+      mbar_init(&bar->ring_full[i], 1);
+      mbar_init(&bar->ring_empty[i], 1);
     }
-    for (int i = 0; i < kVStages; ++i) {
-      mbar_init(&bar->vfull[i], 1);
-      mbar_init(&bar->vempty[i], 1);
+    for (int i = 0; i < kNV; ++i) {
+      mbar_init(&bar->v_full[i], 1);
+      mbar_init(&bar->v_empty[i], 1);
     }
-    mbar_init(&bar->q_full, 1);
-    mbar_init(&bar->q_empty, 1);
+    mbar_init(&bar->qr_full, 1);
+    mbar_init(&bar->qr_empty, 1);
+    mbar_init(&bar->q_drain, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar->s_full[i], 1);
-      mbar_init(&bar->sp_done[i], 2);
-      mbar_init(&bar->sm_local[i], 4);
-      mbar_init(&bar->p_empty[i], 1);
+      mbar_init(&bar->s_empty[i], kSoftWarps);
+      mbar_init(&bar->end_empty[i], 4);
+      for (int q = 0; q < 4; ++q) mbar_init(&bar->row_sync[i][q], 2);
+      mbar_init(&bar->pv[i], 1);
+      mbar_init(&bar->p_full[i], kSoftWarps);
+      mbar_init(&bar->o_ok[i], 4);
+      mbar_init(&bar->end_full[i], kSoftWarps);
+      mbar_init(&bar->d_full[i], 1);
+      // consumers of each descriptor batch: loader, MMA issuer, and the eight
+      // softmax warps (score CTA) or four epilogue warps (value CTA)
+      mbar_init(&bar->d_empty[i], rank == 0 ? 2 + kSoftWarps : 2 + 4);
     }
-    mbar_init(&bar->o_done[0], 1);
-    mbar_init(&bar->o_done[1], 1);
-    mbar_init(&bar->o_free, 8);
     mbar_init(&bar->mma_drain, 1);
-    mbar_init(&bar->k_started, 1);
-    mbar_init(&bar->row_sync[0], kM);
-    mbar_init(&bar->row_sync[1], kM);
-    mbar_init(&bar->l_sync, kM);
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc_pair(&bar->tmem_base, kTmemCols);
-    tmem_relinquish_pair();
+    tmem_alloc(&bar->tmem_base, kTmemCols);
+    tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
-  cluster_sync();     // both CTAs' barriers and TMEM exist before any cross-CTA use
+  cluster_sync();     // both CTAs' barriers exist before any cross-CTA use
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
 
   // Launched as a programmatic dependent of the planner: everything above
   // overlaps it; its plan and stream offsets are read only after this wait.
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  Walk w;
-  const bool has_work = walk_begin(p, g, w);
   bool ok = true;
-  const int n_tiles = has_work ? w.u1 - w.u : 0;
-  if (warp == 1 && rank == 0 && n_tiles <= kFlagTiles) {
-    for (int i = lane; i < n_tiles; i += 32)
-      bar->tflags[i] = (uint8_t)unit_flags<kGather>(p, w.u + i, w.u, w.s);
-    __syncwarp();
-  }
+  const long long y_oob = a.n_pages * kPg;   // first row past the cache: reads as zeros
+  const uint32_t peer = mapa(smem_u32(smem), rank ^ 1u);   // the other CTA's shared memory
+  // roles with a per-unit loop (the other warps of the value CTA have none)
+  const bool consumer = warp < (rank == 0 ? 2 + kSoftWarps : 6);
 
-  if (warp == 0 || warp == 6) {
-    // ------------------------------------------------------------ loads
-    // Every stage lands the same byte count in each CTA, all by TMA (rows
-    // without data come from out-of-bounds boxes, which read as zero), so
-    // rank 0 arms each stage with both CTAs' bytes and rank 1 never signals.
-    const long long y_oob = a.n_pages * kPg;   // first row past the cache
-    int nk = 0, nv = 0, n_qload = 0, cur_s = -1, cur_v = -1;
-    if (lane == 0) {
-      prefetch_tmap(&mp.q);
-      prefetch_tmap(&mp.k0);
-      prefetch_tmap(&mp.k1);
-      prefetch_tmap(&mp.v);
-      for (int i = 0; i < kNumBoxHeights; ++i) prefetch_tmap(&mp.row[i]);
-    }
-    // rows [0, n) of one panel, row 32 k + lane from physical row ph[k] (one
-    // box per row; rows that could not be located are past the cache: zeros)
-    auto gather_panel = [&](uint8_t* dst, uint32_t fb, const long long* ph, int n, int x) {
-      for (int k = 0; 32 * k + lane < n; ++k)
-        tma_load_2d_pair(dst + (32 * k + lane) * 128, &mp.row[kNumBoxHeights - 1], fb, x,
-                         (int)ph[k]);
-    };
-    // physical rows of the current gathered tile: the score loader's rows
-    // 64 rank + lane + 32 k (k < 2), the value loader's lane + 32 k (k < 4)
-    long long gph[4];
-    int gkp[4];
-    // score stage j of tile t: all 64 rows of this CTA's page, panels
-    // [5 j, 5 j + 5) (stage 0) or [5, 9) (stage 1), in slot j
-    auto load_k = [&](const Tile& t, int b, int j) -> bool {
-      if (!wait_warp(&bar->kempty[j], ((nk / kKStages) & 1) ^ 1)) return false;
-      uint8_t* dst = sK + (j ? kKStage0 : 0);
-      const int p0 = j ? kKSplit : 0, p1 = j ? kQPanels : kKSplit;
-      const uint32_t fb = mapa(smem_u32(&bar->kfull[j]), 0);
-      if (rank == 0 && lane == 0)
-        mbar_arrive_expect_tx(&bar->kfull[j], 2 * (j ? kKStage1 : kKStage0));
-      const int rows = half_rows(t, (int)rank);
-      if constexpr (kGather) {
-        for (int pn = p0; pn < p1; ++pn)
-          gather_panel(dst + (pn - p0) * kKPanel, fb, gph, rows, 64 * pn);
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ descriptors
+    Walk w;
+    const bool has_work = walk_begin(p, g, w);
+    const int u0 = w.u, u1 = has_work ? w.u1 : w.u;
+    const int n = u1 - u0;
+    int cs = has_work ? w.s : 0, ps = -1, pv = -1;
+    for (int bt = 0; bt == 0 || 32 * bt < n; ++bt) {
+      if (!wait_warp(&bar->d_empty[bt & 1], ((bt >> 1) & 1) ^ 1)) { fail(ok); break; }
+      const int base = 32 * bt, cnt = min(32, n - base);
+      if (cnt > 0) {
+        const Desc d = produce<kGather>(p, u0, u1, base, cnt, cs, ps, pv, lane);
+        if (lane < cnt) ring_d[(base + lane) % kDescRing] = d;
       }
+      if (bt == 0 && lane == 0) bar->n_units = n;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->d_full[bt & 1]);
+    }
+  } else if (consumer) {
+    // the run's length is published with the first batch
+    if (!wait_warp(&bar->d_full[0], 0)) fail(ok);
+  }
+  const int n_units = (ok && consumer) ? bar->n_units : 0;
+
+  if (rank == 0) {
+    // ================================================================ score CTA
+    uint8_t* ring = smem + kOffRing;
+    uint8_t* sQr = smem + kOffQr;
+    if (warp == 0) {
+      // ------------------------------------------------------------ loads
       if (lane == 0) {
-        if (!kGather && rows == kPg) {
-          tma_load_3d_pair(dst, j ? &mp.k1 : &mp.k0, fb, 0, (int)half_phys(t, (int)rank), p0);
-        } else {
-          for (int pn = p0; pn < p1; ++pn) {
-            if (!kGather)
-              load_rows(dst + (pn - p0) * kKPanel, mp, fb, 64 * pn, half_phys(t, (int)rank), 0, rows);
-            load_rows(dst + (pn - p0) * kKPanel, mp, fb, 64 * pn, y_oob, rows, kPg - rows);
-          }
-        }
+        prefetch_tmap(&mp.q3);
+        prefetch_tmap(&mp.qr);
+        prefetch_tmap(&mp.k3);
+        prefetch_tmap(&mp.kp);
+        if (kGather) prefetch_tmap(&mp.g4);
       }
-      __syncwarp();
-      ++nk;
-      return true;
-    };
-    // value stage kc of tile t: tile rows [32 kc, +32), this CTA's latent
-    // columns [256 rank, +256) (4 panels)
-    auto load_v = [&](const Tile& t, int b) -> bool {
-      for (int kc = 0; kc < 4; ++kc) {
-        const int slot = nv % kVStages;
-        if (!wait_warp(&bar->vempty[slot], ((nv / kVStages) & 1) ^ 1)) return false;
-        uint8_t* dst = sV + slot * kVStage;
-        const uint32_t fb = mapa(smem_u32(&bar->vfull[slot]), 0);
-        if (rank == 0 && lane == 0) mbar_arrive_expect_tx(&bar->vfull[slot], 2 * kVStage);
-        const int hi = kc >> 1, r0 = kR * (kc & 1);
-        const int rows = max(0, min(kR, half_rows(t, hi) - r0));
-        if constexpr (kGather) {
-          for (int q = 0; q < 4; ++q)
-            gather_panel(dst + q * kSPanel, fb, gph + kc, rows, 256 * (int)rank + 64 * q);
-        }
-        if (lane == 0) {
-          if (!kGather && rows == kR) {
-            tma_load_3d_pair(dst, &mp.v, fb, 0, (int)(half_phys(t, hi) + r0), 4 * (int)rank);
-          } else {
-            for (int q = 0; q < 4; ++q) {
-              const int x = 256 * (int)rank + 64 * q;
-              if (!kGather) load_rows(dst + q * kSPanel, mp, fb, x, half_phys(t, hi) + r0, 0, rows);
-              load_rows(dst + q * kSPanel, mp, fb, x, y_oob, rows, kR - rows);
+      int nst = 0, nq = 0;
+      for (int it = 0; it < n_units && ok; ++it) {
+        if (!desc_wait(bar, it, true)) { fail(ok); break; }
+        const Desc d = ring_d[it % kDescRing];
+        const StreamPos sp = stream_pos(p, d.s);
+        if (d.flags & kNewQ) {
+          // the head block's absorbed queries: the rotary panel into its own
+          // buffer, the 8 latent panels through the ring as three stages
+          // (panels 0-2, 3-5, 6-8; the copy to tensor memory skips panel 8)
+          const int qrow = (d.ver * a.n_q + sp.b * a.s_q + sp.j) * a.H + a.h0 + sp.hb * kM;
+          if (!wait_warp(&bar->qr_empty, (nq & 1) ^ 1)) { fail(ok); break; }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&bar->qr_full, kSlot);
+            tma_load_2d(sQr, &mp.qr, &bar->qr_full, kDc, qrow);
+          }
+          for (int st = 0; st < 3 && ok; ++st, ++nst) {
+            const int slot = nst % kNStages;
+            if (!wait_warp(&bar->ring_empty[slot], ((nst / kNStages) & 1) ^ 1)) { fail(ok); break; }
+            if (lane == 0) {
+              mbar_arrive_expect_tx(&bar->ring_full[slot], kStage);
+              tma_load_3d(ring + slot * kStage, &mp.q3, &bar->ring_full[slot], 0, qrow, 3 * st);
             }
           }
+          if (!ok) break;
+          ++nq;
         }
-        __syncwarp();
-        ++nv;
-      }
-      return true;
-    };
-    const bool vwarp = (warp == 6);
-    // L2 prefetch walker: the own-page rows of the next kPrefetchTiles tiles
-    // are requested into L2 while the ring is still full, so that the stage
-    // loads (and the peer's value loads of this page) hit L2.
-    Walk pw = w;
-    int n_tile = 0, n_pref = 2;      // the walker starts at the third tile
-    if (has_work) {
-      walk_next(p, pw);
-      walk_next(p, pw);
-    }
-    for (bool more = has_work; more && ok; more = (w.u < w.u1)) {
-      const StreamPos sp = stream_pos(p, w.s);
-      const Tile t = describe<kGather>(a, sp.b, w.k);
-      if (vwarp) {
-        // the first value loads queue behind the query and score loads, which
-        // the first MMAs need long before any value stage
-        if (n_tile++ == 0 && !wait_warp(&bar->k_started, 0)) { fail(ok); break; }
-        if constexpr (kGather) locate_gathered<4>(a, sp.b, t.g0 + lane, t.g0 + t.n_rows, y_oob, gph, gkp);
-        if (!load_v(t, sp.b)) { fail(ok); break; }
-        walk_next(p, w);
-        continue;
-      }
-      if (w.s != cur_s || t.ver != cur_v) {
-        if (n_qload > 0 && !wait_warp(&bar->q_empty, (n_qload - 1) & 1)) { fail(ok); break; }
-        if (lane == 0) {
-          const int qi = sp.b * a.s_q + sp.j;
-          const int y = (t.ver * a.n_q + qi) * a.H + a.h0 + sp.hb * kM + kMh * (int)rank;
-          const uint32_t qb = mapa(smem_u32(&bar->q_full), 0);
-          if (rank == 0) mbar_arrive_expect_tx(&bar->q_full, 2 * kQPanels * kQPanel);
-          tma_load_3d_pair(sQ, &mp.q, qb, 0, y, 0);
+        long long gph[4];
+        int gkp[4];
+        if constexpr (kGather)
+          locate_gathered<4, 1>(a, sp.b, d.k * kT + 4 * lane, d.k * kT + d.nv0, y_oob, gph, gkp);
+        // both pages full and next to each other in the pool: one box per stage
+        const bool adjacent = !kGather && d.nv0 == kPg && d.nv1 == kPg && d.phys1 == d.phys0 + kPg;
+        for (int st = 0; st < 3 && ok; ++st, ++nst) {
+          const int slot = nst % kNStages;
+          if (!wait_warp(&bar->ring_empty[slot], ((nst / kNStages) & 1) ^ 1)) { fail(ok); break; }
+          uint8_t* dst = ring + slot * kStage;
+          uint64_t* fb = &bar->ring_full[slot];
+          if (lane == 0) mbar_arrive_expect_tx(fb, kStage);
+          __syncwarp();
+          if constexpr (kGather) {
+#pragma unroll
+            for (int pn = 0; pn < kStagePanels; ++pn)
+              tma_gather4(dst + pn * kSlot + 4 * lane * 128, &mp.g4, fb, 64 * (3 * st + pn),
+                          (int)gph[0], (int)gph[1], (int)gph[2], (int)gph[3]);
+          } else if (adjacent) {
+            if (lane == 0) tma_load_3d(dst, &mp.k3, fb, 0, d.phys0, 3 * st);
+          } else if (lane < 2) {
+            const int rows = lane ? d.nv1 : d.nv0;
+            const long long ph = lane ? d.phys1 : d.phys0;
+            for (int pn = 0; pn < kStagePanels; ++pn) {
+              uint8_t* hd = dst + pn * kSlot + lane * (kPg * 128);
+              const int x = 64 * (3 * st + pn);
+              if (rows == kPg) {
+                tma_load_2d(hd, &mp.kp, fb, x, (int)ph);
+              } else {
+                load_rows(hd, mp, fb, x, ph, 0, rows);
+                load_rows(hd, mp, fb, x, y_oob, rows, kPg - rows);
+              }
+            }
+          }
+          __syncwarp();
         }
-        __syncwarp();
-        ++n_qload;
-        cur_s = w.s;
-        cur_v = t.ver;
+        desc_done(bar, it, n_units, lane == 0);
       }
-      if constexpr (kGather)
-        locate_gathered<2>(a, sp.b, t.g0 + kPg * (int)rank + lane, t.g0 + t.n_rows, y_oob, gph,
-                           gkp);
-      if (!load_k(t, sp.b, 0) || !load_k(t, sp.b, 1)) { fail(ok); break; }
-      if (n_tile == 0 && lane == 0) mbar_arrive(&bar->k_started);
-      // (not before the second tile: at start every CTA's first query and
-      // score loads already fill HBM, and prefetches would only delay them)
-      for (; lane == 0 && n_tile > 0 && n_pref <= n_tile + kPrefetchTiles && pw.u < pw.u1;
-           ++n_pref) {
-        const Tile tp = describe<kGather>(a, stream_pos(p, pw.s).b, pw.k);
-        const int rows = half_rows(tp, (int)rank);
-        if (!kGather && rows > 0) {
-          const int y = (int)half_phys(tp, (int)rank);
-          tma_prefetch_l2_3d(&mp.k0, 0, y, 0);
-          tma_prefetch_l2_3d(&mp.k1, 0, y, kKSplit);
-        }
-        walk_next(p, pw);
+      // drain: every load issued here has landed before the CTA exits
+      for (int dd = 1; dd <= kNStages && dd <= nst && ok; ++dd) {
+        const int n = nst - dd;
+        if (!wait_warp(&bar->ring_full[n % kNStages], (n / kNStages) & 1)) fail(ok);
       }
-      __syncwarp();
-      ++n_tile;
-      walk_next(p, w);
-    }
-    // drain: every load issued here has landed before the CTA exits (the
-    // stage barriers live in rank 0, which waits on them for both CTAs)
-    if (rank == 0) {
-      for (int d = 1; d <= kKStages && d <= nk && ok; ++d) {
-        const int n = nk - d;
-        if (!wait_warp(&bar->kfull[n % kKStages], (n / kKStages) & 1)) fail(ok);
-      }
-      for (int d = 1; d <= kVStages && d <= nv && ok; ++d) {
-        const int n = nv - d;
-        if (!wait_warp(&bar->vfull[n % kVStages], (n / kVStages) & 1)) fail(ok);
-      }
-      if (ok && !vwarp && n_qload > 0 && !wait_warp(&bar->q_full, (n_qload - 1) & 1)) fail(ok);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA (rank 0)
-    if (rank == 0 && lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(kM, 2 * kPg, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(kM, 256, false, true);
-      int it = 0, nk = 0, nv = 0, n_q = 0, n_streams = 0;
-      int prev_first = 0, prev_stream_idx = 0;
-      auto issue_pv = [&](int t, int first, int stream_idx) -> bool {
-        const int pb = t & 1;
-        if (!mbar_wait_cluster(&bar->sp_done[pb], (t >> 1) & 1)) return false;
-        if (first && stream_idx > 0 && !mbar_wait_cluster(&bar->o_free, (stream_idx - 1) & 1))
-          return false;
-        tc_fence_after();
-        const uint32_t pa = smem_u32(sP + pb * kPBuf);
-        for (int kc = 0; kc < 4; ++kc) {
-          const int slot = nv % kVStages;
-          if (!mbar_wait(&bar->vfull[slot], (nv / kVStages) & 1)) return false;
+      if (ok && nq > 0 && !wait_warp(&bar->qr_full, (nq - 1) & 1)) fail(ok);
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA
+      if (lane == 0) {
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(kM, kT, false, false);
+        const uint32_t ring0 = smem_u32(ring), qr0 = smem_u32(sQr);
+        int nst = 0, nq = 0;
+        for (int it = 0; it < n_units && ok; ++it) {
+          if (!desc_wait(bar, it, false)) { fail(ok); break; }
+          const uint32_t flags = ring_d[it % kDescRing].flags;
+          desc_done(bar, it, n_units, true);
+          if (flags & kNewQ) {
+            if (nq > 0) {   // the earlier score MMAs are done reading Q and its rotary panel
+              mma_commit(&bar->qr_empty);
+              mma_commit(&bar->q_drain);
+              if (!mbar_wait(&bar->q_drain, (nq - 1) & 1)) { fail(ok); break; }
+            }
+            if (!mbar_wait(&bar->qr_full, nq & 1)) { fail(ok); break; }
+            for (int st = 0; st < 3 && ok; ++st, ++nst) {
+              const int slot = nst % kNStages;
+              if (!mbar_wait(&bar->ring_full[slot], (nst / kNStages) & 1)) { fail(ok); break; }
+              tc_fence_after();
+              for (int pn = 0; pn < kStagePanels && 3 * st + pn < 8; ++pn)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                  tmem_cp_128x256b(tmem + kColQ + 32 * (3 * st + pn) + 8 * ks,
+                                   smem_desc_sw128(ring0 + slot * kStage + pn * kSlot + ks * 32, 16, 1024));
+              mma_commit(&bar->ring_empty[slot]);
+            }
+            if (!ok) break;
+            ++nq;
+          }
+          const int sb = it & 1;
+          if (!mbar_wait(&bar->s_empty[sb], ((it >> 1) & 1) ^ 1)) { fail(ok); break; }
           tc_fence_after();
-          const uint32_t vb = smem_u32(sV + slot * kVStage);
+          const uint32_t dt = tmem + kColS + 128 * sb;
+          for (int st = 0; st < 3 && ok; ++st, ++nst) {
+            const int slot = nst % kNStages;
+            if (!mbar_wait(&bar->ring_full[slot], (nst / kNStages) & 1)) { fail(ok); break; }
+            tc_fence_after();
 #pragma unroll
-          for (int nb = 0; nb < 2; ++nb) {
+            for (int pn = 0; pn < kStagePanels; ++pn) {
+              const int panel = 3 * st + pn;
+              const uint32_t kb = ring0 + slot * kStage + pn * kSlot;
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const int ks = 2 * kc + j;     // 16-row step of the 128-row tile
-              const uint64_t ad =
-                  smem_desc_sw128(pa + (ks >> 2) * kQPanel + (ks & 3) * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(vb + nb * 2 * kSPanel + j * 2048, kSPanel, 1024);
-              mma_pair_bf16_ss(tmem + kColO + nb * 128, ad, bd, idesc_pv,
-                               (first && ks == 0) ? 0u : 1u);
+              for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t bd = smem_desc_sw128(kb + ks * 32, 16, 1024);
+                if (panel < 8)
+                  mma_bf16_ts(dt, tmem + kColQ + 32 * panel + 8 * ks, bd, idesc_qk, (panel | ks) ? 1u : 0u);
+                else
+                  mma_bf16_ss(dt, smem_desc_sw128(qr0 + ks * 32, 16, 1024), bd, idesc_qk, 1u);
+              }
             }
+            mma_commit(&bar->ring_empty[slot]);
           }
-          mma_pair_commit_both(&bar->vempty[slot]);
-          ++nv;
+          if (!ok) break;
+          mma_commit(&bar->s_full[sb]);
         }
-        mma_pair_commit_both(&bar->p_empty[pb]);
-        mma_pair_commit_both(&bar->o_done[pb]);
-        return true;
-      };
-      // per-tile flags: from shared memory, or computed here for long runs
-      auto flags_of = [&](int i) -> uint32_t {
-        return n_tiles <= kFlagTiles ? bar->tflags[i]
-                                     : unit_flags<kGather>(p, w.u + i, w.u, w.s);
-      };
-      uint32_t f = n_tiles > 0 ? flags_of(0) : 0u;
-      for (; it < n_tiles && ok; ++it) {
-        const bool first = f & 1u;
-        if (first) ++n_streams;
-        if (f & 2u) {
-          if (!mbar_wait(&bar->q_full, n_q & 1)) { fail(ok); break; }
-          ++n_q;
-        }
-        const int sb = it & 1;
-        if (!mbar_wait_cluster(&bar->sp_done[sb], ((it >> 1) & 1) ^ 1)) { fail(ok); break; }
-        tc_fence_after();
-        const uint32_t qa = smem_u32(sQ);
-        // S (64 columns: page 0 rows in lanes 0-63, page 1 rows in lanes
-        // 64-127) accumulates over the two column stages of the tile
-        for (int j = 0; j < 2 && ok; ++j) {
-          if (!mbar_wait(&bar->kfull[j], (nk / kKStages) & 1)) { fail(ok); break; }
-          tc_fence_after();
-          const uint32_t kb = smem_u32(sK + (j ? kKStage0 : 0));
-          const int p0 = j ? kKSplit : 0, p1 = j ? kQPanels : kKSplit;
-          for (int pn = p0; pn < p1; ++pn) {
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              const uint64_t ad = smem_desc_sw128(qa + pn * kQPanel + ks * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(kb + (pn - p0) * kKPanel + ks * 32, 16, 1024);
-              mma_pair_bf16_ss(tmem + kColS + sb * 64, ad, bd, idesc_qk, (pn | ks) ? 1u : 0u);
-            }
-          }
-          mma_pair_commit_both(&bar->kempty[j]);
-          ++nk;
-        }
-        if (!ok) break;
-        mma_pair_commit_both(&bar->s_full[sb]);
-        const uint32_t fn = it + 1 < n_tiles ? flags_of(it + 1) : 0u;
-        if (fn & 2u) mma_pair_commit_both(&bar->q_empty);   // the next tile reloads Q
-        if (it > 0 && !issue_pv(it - 1, prev_first, prev_stream_idx)) { fail(ok); break; }
-        prev_first = first;
-        prev_stream_idx = n_streams - 1;
-        f = fn;
+        if (ok && nq > 0) mma_commit(&bar->qr_empty);
+        mma_commit(&bar->mma_drain);
+        if (!mbar_wait(&bar->mma_drain, 0)) fail(ok);
       }
-      if (ok && it > 0 && !issue_pv(it - 1, prev_first, prev_stream_idx)) fail(ok);
-      mma_pair_commit_own(&bar->mma_drain);
-      if (!mbar_wait(&bar->mma_drain, 0)) fail(ok);
-    }
-  } else {
-    // ------------------------------------------------------------ softmax
-    const int quad = warp & 3;
-    const int t = quad * 32 + lane;           // TMEM lane
-    const int half = t >> 6;                  // tile rows [64 half, +64)
-    const int hl = t & 63;                    // head row of this CTA
-    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-    int it = 0, n_epi = 0;
-    // P.c of tile t is complete.  o_done[t & 1] completes once per two tiles;
-    // the P buffer waits (p_empty) already ordered every earlier product of
-    // the same parity, so the barrier is never a phase ahead or behind.
-    auto wait_o_done = [&](int t) -> bool {
-      return wait_warp(&bar->o_done[t & 1], (t >> 1) & 1);
-    };
-    while (has_work && ok && w.u < w.u1) {
-      const int s = w.s;
-      const StreamPos sp = stream_pos(p, s);
-      const int qi = sp.b * a.s_q + sp.j;
-      const int qp = a.q_pos[qi];
-      const int hrow = sp.hb * kM + kMh * (int)rank + hl;   // head within [h0, h0 + n_h)
-      const bool row_valid = hrow < a.n_h;
-      const int T = stream_tiles(p, s);
-      float m_run = -INFINITY, l_run = 0.f;
-      bool have_o = false;
-      while (ok && w.u < w.u1 && w.s == s) {
-        const Tile tl = describe<kGather>(a, sp.b, w.k);
-        const int sb = it & 1;
-        const uint64_t vis = visible_rows<kGather>(a, tl, sp.b, half, qp, lane);
+    } else if (warp < kProducerWarp) {
+      // ------------------------------------------------------------ softmax
+      // Two warps per TMEM lane quarter: warp 2 + 4 hf owns columns
+      // [64 hf, 64 hf + 64) of the tile (page hf) for the quarter's 32 rows.
+      const int quad = warp & 3;
+      const int hf = (warp - 2) >> 2;
+      const int h = quad * 32 + lane;            // head row of the block = TMEM lane
+      const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16) + kColS + 64 * hf;
+      float* sMax = reinterpret_cast<float*>(smem + kOffMax);   // [buffer][half][row]
+      const uint32_t mbase = peer + kOffMsg, ebase = peer + kOffEnd;
+      int n_str = 0;
+      float m_run = -INFINITY, l_run = 0.f;      // l_run: this half's share of the row sum
+      // P, the rescale factors and the flags travel as asynchronous remote
+      // stores (st.async) whose bytes complete a transaction count on the value
+      // CTA's barrier: the warp never waits for them.  Each warp announces its
+      // share of the bytes with one remote arrival.
+      const uint32_t p_bytes = 32 * 8 * 16 + (hf == 0 ? 4 * 32 : 0) + 4;
+      const uint32_t e_bytes = 4 * 32 + (hf == 0 ? 4 * 32 : 0);
+      for (int it = 0; it < n_units && ok; ++it) {
+        if (!desc_wait(bar, it, true)) { fail(ok); break; }
+        const Desc d = ring_d[it % kDescRing];
+        const StreamPos sp = stream_pos(p, d.s);
+        const bool valid = sp.hb * kM + h < a.n_h;
+        if (d.flags & kFirst) {
+          m_run = -INFINITY;
+          l_run = 0.f;
+        }
+        const uint64_t vis = visibility<kGather>(a, d, sp.b, hf, lane);
+        const uint32_t v0 = (uint32_t)vis, v1 = (uint32_t)(vis >> 32);
+        const int sb = it & 1, pb = it & 1;
         if (!wait_warp(&bar->s_full[sb], (it >> 1) & 1)) { fail(ok); break; }
         tc_fence_after();
-        const uint32_t s_col = trow + kColS + sb * 64;
+        float x[64];
+        tmem_ld32(trow + 128 * sb, *reinterpret_cast<float(*)[32]>(x));
+        tmem_ld32(trow + 128 * sb + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->s_empty[sb]);
 
-        // pass 1: max of the visible scores of this lane's 64 rows
-        float mh = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < 64; c += 16) {
-          float x[16];
-          tmem_ld16(s_col + c, x);
-          tmem_wait_ld();
-          const uint32_t bits = (uint32_t)(vis >> c);
+        // max of this half's visible scores (four independent chains), then
+        // of the row, through the partner warp (log2 units)
+        // (branch-free: a select per element keeps every element's work in one
+        // basic block, so the scheduler can overlap their latencies)
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (bits & (1u << i)) mh = fmaxf(mh, x[i]);
+        for (int c = 0; c < 64; ++c) {
+          const bool vb = ((c < 32 ? v0 : v1) >> (c & 31)) & 1u;
+          mx[c & 3] = fmaxf(mx[c & 3], vb ? x[c] : -INFINITY);
         }
-        mh *= p.scale_log2;                   // scale > 0: max commutes, -inf stays
-        // the two lanes of a head row agree on the tile max
-        sMax[(it & 1) * kM + t] = mh;
-        mbar_arrive(&bar->row_sync[it & 1]);
-        if (!wait_warp(&bar->row_sync[it & 1], (it >> 1) & 1)) { fail(ok); break; }
-        const float mt = fmaxf(mh, sMax[(it & 1) * kM + (t ^ 64)]);
-
+        const float mh = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
+        sMax[(sb * 2 + hf) * kM + h] = mh;       // scale > 0: max commutes, -inf stays
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->row_sync[sb][quad]);
+        if (!wait_warp(&bar->row_sync[sb][quad], (it >> 1) & 1)) { fail(ok); break; }
+        const float mt = fmaxf(mh, sMax[(sb * 2 + (hf ^ 1)) * kM + h]);
         // lazy rescaling: keep the reference max unless it grows by > 2^8
         const bool need = mt > m_run + kRescaleThreshold;
         const float m_new = need ? mt : m_run;
         const float factor = need ? exp2f(m_run - m_new) : 1.f;   // exp2(-inf) = 0
-        if (have_o && __any_sync(0xffffffffu, need)) {
-          if (!wait_o_done(it - 1)) { fail(ok); break; }
-          tc_fence_after();
-          scale_o(trow + kColO, need ? factor : 1.f);
-        }
+        const bool any = valid && (m_new != -INFINITY);
 
-        // pass 2: P = 2^(scale*S - m_new) on visible rows, bf16, 128-byte
-        // swizzled K-major rows of the P.c operand
-        const int pb = it & 1;
-        if (!wait_warp(&bar->p_empty[pb], ((it >> 1) & 1) ^ 1)) { fail(ok); break; }
-        uint8_t* prow = sP + pb * kPBuf + half * kQPanel + hl * 128;
-        float lsum = 0.f;
-        const bool any = (m_new != -INFINITY);
-#pragma unroll 1
-        for (int c = 0; c < 64; c += 16) {
-          float x[16];
-          tmem_ld16(s_col + c, x);
-          tmem_wait_ld();
-          const uint32_t bits = any ? (uint32_t)(vis >> c) : 0u;
-          uint32_t pk[8];
+        // P = 2^(scale*S - m_new) on visible rows, bf16, into P panel hf of the
+        // value CTA's message buffer (128-byte swizzled K-major rows) once the
+        // value CTA is done with the tile that last used it
+        if (!wait_warp_cluster(&bar->pv[pb], ((it >> 1) & 1) ^ 1)) { fail(ok); break; }
+        const uint32_t msg = mbase + pb * kMsgStride;
+        const uint32_t prow = msg + hf * (kM * 128) + h * 128;
+        const uint32_t fbar = mapa(smem_u32(&bar->p_full[pb]), 1);
+        if (lane == 0) mbar_arrive_expect_tx_cluster(fbar, p_bytes);
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int i = 0; i < 16; i += 2) {
-            const float p0 = (bits & (1u << i)) ? ex2_approx(fmaf(x[i], p.scale_log2, -m_new)) : 0.f;
-            const float p1 =
-                (bits & (2u << i)) ? ex2_approx(fmaf(x[i + 1], p.scale_log2, -m_new)) : 0.f;
+        for (int c = 0; c < 64; c += 8) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int i = 0; i < 8; i += 2) {
+            const int c0 = c + i, c1 = c + i + 1;
+            const bool b0 = any && (((c0 < 32 ? v0 : v1) >> (c0 & 31)) & 1u);
+            const bool b1 = any && (((c1 < 32 ? v0 : v1) >> (c1 & 31)) & 1u);
+            // every element's exponential is taken; the mask only selects
+            const float e0 = ex2_approx(fmaf(x[c0], p.scale_log2, -m_new));
+            const float e1 = ex2_approx(fmaf(x[c1], p.scale_log2, -m_new));
+            const float p0 = b0 ? e0 : 0.f;
+            const float p1 = b1 ? e1 : 0.f;
             const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-            lsum += __low2float(h2) + __high2float(h2);
+            ls[(i >> 1) & 3] += __low2float(h2) + __high2float(h2);
             pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
           }
-          const int ch = c >> 3;
-          *reinterpret_cast<uint4*>(prow + ((ch ^ (hl & 7)) << 4)) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          *reinterpret_cast<uint4*>(prow + (((ch + 1) ^ (hl & 7)) << 4)) =
-              make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          st_async_v4(prow + ((((c >> 3)) ^ (h & 7)) << 4), make_uint4(pk[0], pk[1], pk[2], pk[3]), fbar);
         }
-        l_run = l_run * factor + lsum;
+        l_run = l_run * factor + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
         m_run = m_new;
-        tc_fence_before();
-        fence_proxy_async();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar->sm_local[pb]);
-        // one arrival per CTA reaches the leader: the pair's MMA traffic
-        // shares the path a remote arrival takes, so fewer of them land sooner
-        if (quad == 0) {
-          if (!wait_warp(&bar->sm_local[pb], (it >> 1) & 1)) { fail(ok); break; }
-          if (lane == 0) arrive_leader(&bar->sp_done[pb], rank);
+        if (hf == 0) st_async_b32(msg + kPBuf + 4 * h, __float_as_uint(valid ? factor : 1.f), fbar);
+        // O needs a rescale before this tile's P.c when a live row's reference
+        // max moved (never on a stream's first tile: that P.c overwrites O)
+        const bool wf = __any_sync(0xffffffffu, valid && need && !(d.flags & kFirst));
+        if (lane == 0) st_async_b32(msg + kPBuf + kHdrFlag + 4 * (warp - 2), wf ? 1u : 0u, fbar);
+        if (d.flags & kLast) {
+          // stream end: each half's row sums and the row max for the epilogue
+          const int es = n_str & 1;
+          if (!wait_warp_cluster(&bar->end_empty[es], ((n_str >> 1) & 1) ^ 1)) { fail(ok); break; }
+          const uint32_t e = ebase + es * kEndBytes;
+          const uint32_t ebar = mapa(smem_u32(&bar->end_full[es]), 1);
+          if (lane == 0) mbar_arrive_expect_tx_cluster(ebar, e_bytes);
+          st_async_b32(e + hf * (4 * kM) + 4 * h, __float_as_uint(l_run), ebar);
+          if (hf == 0) st_async_b32(e + 8 * kM + 4 * h, __float_as_uint(m_run), ebar);
+          ++n_str;
         }
-        have_o = true;
-        ++it;
-        walk_next(p, w);
+        desc_done(bar, it, n_units, lane == 0);
       }
-      if (!ok) break;
-
-      // epilogue: O of the stream is complete once its last P.c is done
-      if (!wait_o_done(it - 1)) { fail(ok); break; }
-      tc_fence_after();
-      sL[t] = l_run;
-      mbar_arrive(&bar->l_sync);
-      if (!wait_warp(&bar->l_sync, n_epi & 1)) { fail(ok); break; }
-      ++n_epi;
-      const float l_tot = l_run + sL[t ^ 64];
-      const int off_s = p.stream_off[s];
-      const int range_u0 = g * p.plan->C;
-      const bool whole = (off_s >= range_u0) && (off_s + T <= w.u1);
-      const bool empty = !(l_tot > 0.f);
-      const float inv = empty ? 0.f : 1.f / l_tot;
-      const float lse = empty ? -INFINITY : (m_run + log2f(l_tot)) * 0.6931471805599453f;
-      // O rows go out through the P buffers (idle here: the last P.c is done
-      // and this warp writes no new P before the next tile's pass 2).  Each
-      // warp stages its own 32 rows x 32 columns per step in an 8 KB slice
-      // (two 4 KB halves, alternating) and lane 0 stores the box by TMA, so
-      // no cross-warp barrier is involved.
-      const int slot = 2 * g + ((off_s <= range_u0) ? 0 : 1);
-      const int row0 = kMh * (int)rank + 32 * (quad & 1);   // first head row of this warp
-      const bool store = !whole || sp.hb * kM + row0 < a.n_h;
-#pragma unroll 1
-      for (int c = 0; c < 256; c += kStoreCols) {
-        const int k = c / kStoreCols;
-        uint8_t* stage = sP + quad * 8192 + (k & 1) * 4096;
-        if (k >= 2) {
-          if (lane == 0) bulk_wait_read<1>();
+    }
+  } else {
+    // ================================================================ value CTA
+    uint8_t* vbuf = smem + kOffVal;     // two page slots: 8 latent panels of 64 rows
+    uint8_t* msg = smem + kOffMsg;      // two P messages: P, then factors and the flags
+    const float* endm = reinterpret_cast<const float*>(smem + kOffEnd);
+    if (warp == 0) {
+      // ------------------------------------------------------------ loads
+      if (lane == 0) {
+        prefetch_tmap(&mp.vp);
+        if (kGather) prefetch_tmap(&mp.g4);
+      }
+      int nv = 0;
+      for (int it = 0; it < n_units && ok; ++it) {
+        if (!desc_wait(bar, it, true)) { fail(ok); break; }
+        const Desc d = ring_d[it % kDescRing];
+        const int b = stream_pos(p, d.s).b;
+        for (int hp = 0; hp < 2 && ok; ++hp, ++nv) {
+          const int slot = nv % kNV;
+          if (!wait_warp(&bar->v_empty[slot], ((nv / kNV) & 1) ^ 1)) { fail(ok); break; }
+          uint8_t* dst = vbuf + slot * kVPage;
+          uint64_t* fb = &bar->v_full[slot];
+          if (lane == 0) mbar_arrive_expect_tx(fb, kVPage);
+          __syncwarp();
+          if constexpr (kGather) {
+            // lane l: rows 4 (l & 15) .. + 3 of the page's 64 rows, latent
+            // panels (l >> 4) + 2 k, k = 0..3
+            long long gph[4];
+            int gkp[4];
+            const int r4 = 4 * (lane & 15);
+            locate_gathered<4, 1>(a, b, d.k * kT + kPg * hp + r4, d.k * kT + d.nv0, y_oob, gph, gkp);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int q = (lane >> 4) + 2 * k;
+              tma_gather4(dst + q * (kPg * 128) + r4 * 128, &mp.g4, fb, 64 * q, (int)gph[0],
+                          (int)gph[1], (int)gph[2], (int)gph[3]);
+            }
+          } else if (lane == 0) {
+            const int rows = hp ? d.nv1 : d.nv0;
+            const long long ph = hp ? d.phys1 : d.phys0;
+            if (rows == kPg) {
+              tma_load_3d(dst, &mp.vp, fb, 0, (int)ph, 0);
+            } else {
+              for (int q = 0; q < 8; ++q) {
+                load_rows(dst + q * (kPg * 128), mp, fb, 64 * q, ph, 0, rows);
+                load_rows(dst + q * (kPg * 128), mp, fb, 64 * q, y_oob, rows, kPg - rows);
+              }
+            }
+          }
           __syncwarp();
         }
-        float ov[kStoreCols];
-        tmem_ld32(trow + kColO + c, ov);
-        tmem_wait_ld();
+        desc_done(bar, it, n_units, lane == 0);
+      }
+      for (int dd = 1; dd <= kNV && dd <= nv && ok; ++dd) {
+        const int n = nv - dd;
+        if (!wait_warp(&bar->v_full[n % kNV], (n / kNV) & 1)) fail(ok);
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA
+      if (lane == 0) {
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(kM, 256, false, true);
+        const uint32_t v0 = smem_u32(vbuf), p0 = smem_u32(msg);
+        int nv = 0;
+        for (int it = 0; it < n_units && ok; ++it) {
+          if (!desc_wait(bar, it, false)) { fail(ok); break; }
+          const bool first = ring_d[it % kDescRing].flags & kFirst;
+          desc_done(bar, it, n_units, true);
+          const int pb = it & 1;
+          if (!mbar_wait_cluster(&bar->p_full[pb], (it >> 1) & 1) ||
+              !mbar_wait(&bar->o_ok[pb], (it >> 1) & 1)) { fail(ok); break; }
+          // P arrived as generic-proxy stores: order them before the tensor
+          // core's (async-proxy) reads of the buffer
+          fence_proxy_async();
+          tc_fence_after();
+          const uint32_t pa = p0 + pb * kMsgStride;
+          for (int hp = 0; hp < 2 && ok; ++hp, ++nv) {
+            const int slot = nv % kNV;
+            if (!mbar_wait(&bar->v_full[slot], (nv / kNV) & 1)) { fail(ok); break; }
+            tc_fence_after();
+            const uint32_t vb = v0 + slot * kVPage;
 #pragma unroll
-        for (int i = 0; i < kStoreCols; i += 4)
-          *reinterpret_cast<float4*>(stage + lane * 128 + (((i >> 2) ^ (lane & 7)) << 4)) =
-              make_float4(ov[i] * inv, ov[i + 1] * inv, ov[i + 2] * inv, ov[i + 3] * inv);
-        fence_proxy_async();
+            for (int ks = 0; ks < 4; ++ks) {
+              // P panel hp holds the page's 64 tokens; 16 of them per step
+              const uint64_t ad = smem_desc_sw128(pa + hp * (kM * 128) + ks * 32, 16, 1024);
+#pragma unroll
+              for (int nb = 0; nb < 2; ++nb) {
+                const uint64_t bd = smem_desc_sw128(vb + nb * 4 * (kPg * 128) + ks * 2048, kPg * 128, 1024);
+                mma_bf16_ss(tmem + 256 * nb, ad, bd, idesc_pv, (first && hp == 0 && ks == 0) ? 0u : 1u);
+              }
+            }
+            mma_commit(&bar->v_empty[slot]);
+          }
+          if (!ok) break;
+          mma_commit_mask(&bar->pv[pb], 0x3);    // this CTA's epilogue and the score CTA's P buffer
+        }
+        mma_commit(&bar->mma_drain);
+        if (!mbar_wait(&bar->mma_drain, 0)) fail(ok);
+      }
+    } else if (warp < 6) {
+      // ------------------------------------------------------------ rescale and epilogue
+      const int quad = warp & 3;
+      const int h = quad * 32 + lane;
+      const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+      float4* stage = reinterpret_cast<float4*>(smem + kOffStage + quad * kStageWarp);
+      int n_str = 0;
+      for (int it = 0; it < n_units && ok; ++it) {
+        if (!desc_wait(bar, it, true)) { fail(ok); break; }
+        const Desc d = ring_d[it % kDescRing];
+        desc_done(bar, it, n_units, lane == 0);
+        const int pb = it & 1;
+        if (!(d.flags & kFirst)) {
+          if (!wait_warp_cluster(&bar->p_full[pb], (it >> 1) & 1)) { fail(ok); break; }
+          const uint8_t* hdr = msg + pb * kMsgStride + kPBuf;
+          const volatile uint32_t* wfl = reinterpret_cast<const volatile uint32_t*>(hdr + kHdrFlag);
+          uint32_t flag = 0;
+#pragma unroll
+          for (int i = 0; i < kSoftWarps; ++i) flag |= wfl[i];
+          if (flag) {
+            // O must hold every earlier tile's P.c before it is rescaled
+            if (!wait_warp(&bar->pv[(it - 1) & 1], ((it - 1) >> 1) & 1)) { fail(ok); break; }
+            tc_fence_after();
+            const float f = reinterpret_cast<const float*>(hdr)[h];
+            scale_o(trow, f);
+            tc_fence_before();
+          }
+        }
         __syncwarp();
-        if (lane == 0 && store) {
-          const int lat = 256 * half + c;
-          if (whole) tma_store_3d(&mp.o, stage, lat, sp.hb * kM + row0, qi);
-          else tma_store_2d(&mp.part, stage, lat, slot * kM + row0);
-          bulk_commit();
+        if (lane == 0) mbar_arrive(&bar->o_ok[pb]);
+        if (d.flags & kLast) {
+          // the stream's O is complete once this tile's P.c is done
+          const int es = n_str & 1;
+          if (!wait_warp(&bar->pv[pb], (it >> 1) & 1) ||
+              !wait_warp_cluster(&bar->end_full[es], (n_str >> 1) & 1)) { fail(ok); break; }
+          tc_fence_after();
+          const float l_tot = endm[es * (kEndBytes / 4) + h] + endm[es * (kEndBytes / 4) + kM + h];
+          const float m_fin = endm[es * (kEndBytes / 4) + 2 * kM + h];
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster_addr(mapa(smem_u32(&bar->end_empty[es]), 0));
+          const StreamPos sp = stream_pos(p, d.s);
+          const int qi = sp.b * a.s_q + sp.j;
+          const bool whole = d.flags & kWhole;
+          const int slot = 2 * g + ((d.flags & kSlot1) ? 1 : 0);
+          const bool empty = !(l_tot > 0.f);
+          const float inv = empty ? 0.f : 1.f / l_tot;
+          const float lse = empty ? -INFINITY : (m_fin + log2f(l_tot)) * 0.6931471805599453f;
+          const int hrow0 = sp.hb * kM + quad * 32;        // first head row of this warp
+          float* dst0 = whole ? a.o_lat + ((size_t)qi * a.H + a.h0 + hrow0) * kDc
+                              : p.partial + ((size_t)slot * kM + quad * 32) * kDc;
+          const int live = whole ? min(32, a.n_h - hrow0) : 32;   // rows this warp may write
+          // O rows leave through a per-warp staging tile: each lane writes its
+          // row's 32 columns, then each store instruction writes 4 rows x 128 B.
+          // The next 32 columns are read from tensor memory while this chunk's
+          // stores issue.
+          float ov[32], on[32];
+          tmem_ld32(trow, ov);
+          tmem_wait_ld();
+#pragma unroll 1
+          for (int c = 0; c < kDc; c += 32) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              stage[lane * 8 + (j ^ (lane & 7))] =
+                  make_float4(ov[4 * j] * inv, ov[4 * j + 1] * inv, ov[4 * j + 2] * inv,
+                              ov[4 * j + 3] * inv);
+            if (c + 32 < kDc) tmem_ld32(trow + c + 32, on);
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int rr = 4 * k + (lane >> 3), j = lane & 7;
+              if (rr < live)
+                *reinterpret_cast<float4*>(dst0 + (size_t)rr * kDc + c + 4 * j) =
+                    stage[rr * 8 + (j ^ (rr & 7))];
+            }
+            __syncwarp();
+            if (c + 32 < kDc) {
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) ov[i] = on[i];
+            }
+          }
+          tc_fence_before();
+          if (sp.hb * kM + h < a.n_h) {
+            if (whole) a.lse[(size_t)qi * a.H + a.h0 + sp.hb * kM + h] = lse;
+            else p.partial_lse[(size_t)slot * kM + h] = lse;
+          }
+          ++n_str;
         }
       }
-      if (lane == 0) bulk_wait_read<0>();
-      __syncwarp();
-      if (row_valid && half == 0) {
-        if (whole) a.lse[(size_t)qi * a.H + a.h0 + hrow] = lse;
-        else p.partial_lse[(size_t)slot * kM + kMh * (int)rank + hl] = lse;
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) arrive_leader(&bar->o_free, rank);
     }
   }
 
-  if (warp >= 2 && warp < 6 && lane == 0) bulk_wait_all();   // epilogue stores have landed
-  asm volatile("griddepcontrol.launch_dependents;");            // the merge may be scheduled
+  asm volatile("griddepcontrol.launch_dependents;");   // the merge may be scheduled
   tc_fence_before();
   __syncthreads();
-  cluster_sync();   // no CTA leaves while its peer may still touch its memory
+  cluster_sync();   // no CTA leaves while its peer may still write its shared memory
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc_pair(tmem, kTmemCols);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 

@@ -108,42 +108,19 @@ EncodeTiledFn encode_fn() {
 
 // Tensor map over a [rows, 576] bf16 matrix (row pitch 1152 B) with 64-column
 // boxes and 128-byte swizzle.  rank 2: (col, row), box {64, h}.  rank 3:
-// (col, row, 64-column panel), box {64, h, panels}.  rank 4: (col, row, panel
-// within a 256-column group, group), box {64, h, 2, 2}.
+// (col, row, 64-column panel), box {64, h, panels}: each box row is 128 *
+// panels contiguous bytes, landing as `panels` planes of h x 128 bytes.
 bool make_map_576(CUtensorMap* m, const void* base, uint64_t rows, int rank, uint32_t h,
                   uint32_t panels = 9) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[4] = {64, (cuuint64_t)rows, 9, 1};
-  cuuint64_t strides[3] = {(cuuint64_t)tc::kRow * 2, 128, 0};
-  cuuint32_t box[4] = {64, h, panels, 1};
+  cuuint64_t dims[3] = {64, (cuuint64_t)rows, 9};
+  cuuint64_t strides[2] = {(cuuint64_t)tc::kRow * 2, 128};
+  cuuint32_t box[3] = {64, h, panels};
   if (rank == 2) dims[0] = tc::kRow;
-  if (rank == 4) {
-    dims[2] = 4;
-    dims[3] = 2;
-    strides[2] = 512;
-    box[2] = 2;
-    box[3] = 2;
-  }
-  cuuint32_t estr[4] = {1, 1, 1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims,
             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// fp32 store map for decode outputs: (column, row[, plane]) over rows of 512
-// floats, box {32, 32[, 1]}, 128-byte swizzle.  rank 3: rows are heads
-// (extent n_rows) and planes are query rows (stride plane_stride floats).
-bool make_map_out(CUtensorMap* m, float* base, uint64_t n_rows, uint64_t n_planes,
-                  uint64_t plane_stride, int rank) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)tc::kDc, (cuuint64_t)n_rows, (cuuint64_t)n_planes};
-  cuuint64_t strides[2] = {(cuuint64_t)tc::kDc * 4, (cuuint64_t)plane_stride * 4};
-  cuuint32_t box[3] = {(cuuint32_t)tc::kStoreCols, 32, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, (cuuint32_t)rank, base, dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -436,13 +413,16 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
 
   tc::Maps maps;
   const uint64_t cache_rows = (uint64_t)n_pages * kPage;
-  if (!make_map_576(&maps.q, q_abs, (uint64_t)n_ver * B * s_q * dims->H, 3, tc::kMh) ||
-      !make_map_576(&maps.k0, cache, cache_rows, 3, tc::kPg, tc::kKSplit) ||
-      !make_map_576(&maps.k1, cache, cache_rows, 3, tc::kPg, tc::kQPanels - tc::kKSplit) ||
-      !make_map_576(&maps.v, cache, cache_rows, 3, tc::kR, 4))
+  const uint64_t q_rows = (uint64_t)n_ver * B * s_q * dims->H;
+  if (!make_map_576(&maps.q3, q_abs, q_rows, 3, tc::kM, tc::kStagePanels) ||
+      !make_map_576(&maps.qr, q_abs, q_rows, 2, tc::kM) ||
+      !make_map_576(&maps.k3, cache, cache_rows, 3, tc::kT, tc::kStagePanels) ||
+      !make_map_576(&maps.kp, cache, cache_rows, 2, tc::kPg) ||
+      !make_map_576(&maps.vp, cache, cache_rows, 3, tc::kPg, 8) ||
+      !make_map_576(&maps.g4, cache, cache_rows, 2, 1))
     return MLA_ERR_CUDA;
   for (int i = 0; i < tc::kNumBoxHeights; ++i)
-    if (!make_map_576(&maps.row[i], cache, cache_rows, 2, (uint32_t)(tc::kR >> i)))
+    if (!make_map_576(&maps.row[i], cache, cache_rows, 2, (uint32_t)(32 >> i)))
       return MLA_ERR_CUDA;
 
   if (!dev->tc_attr_set) {
@@ -464,11 +444,6 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
   int* pair_stream = reinterpret_cast<int*>(ws + wl.off_pairs);
   float* partial = reinterpret_cast<float*>(ws + wl.off_partial);
   float* partial_lse = reinterpret_cast<float*>(ws + wl.off_plse);
-  if (!make_map_out(&maps.o, o_lat + (size_t)h0 * tc::kDc, (uint64_t)n_h, (uint64_t)B * s_q,
-                    (uint64_t)dims->H * tc::kDc, 3) ||
-      !make_map_out(&maps.part, partial, (uint64_t)tc::kM * 2 * G, 1, 0, 2))
-    return MLA_ERR_CUDA;
-
   if (gather)
     tc::plan_kernel<true><<<1, tc::kPlanThreads, 0, st>>>(a, n_hb, G, plan, stream_off,
                                                           stream_bad, pair_stream);
@@ -484,6 +459,7 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
   p.plan = plan;
   p.stream_off = stream_off;
   p.pair_stream = pair_stream;
+  p.partial = partial;
   p.partial_lse = partial_lse;
   p.scale_log2 = dims->scale * tc::kLog2e;
   // The attention and merge kernels are programmatic dependents of the
