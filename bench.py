@@ -1,19 +1,25 @@
-"""Benchmark of one absorbed-MLA decode step on B200 (libmla).
+"""Benchmark of the absorbed-MLA decode on B200 (libmla).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
+                    [--workload NAME] [--no-workloads] [--no-cpu-baseline]
 
 A step is one pass of the whole hot path over one batch: absorb_q (W_UK and
 the rotary query), decode over the paged latent cache (plan, split-KV
-attention, split merge) and out_proj (W_UV then W_O).  The workload is the
-B=16, H=128, 4096-row bf16 decode (d_c=512, d_r=64, d_n=d_v=128,
-d_model=7168); inputs are synthetic and seeded.  The metric is latent-cache
-GB/s: the 75.5 MB of cache rows the step reads, over the step time.
+attention, split merge) and out_proj (W_UV then W_O), each call one CUDA
+graph replayed in that order.  The workload is the B=16, H=128, 4096-row
+bf16 decode (d_c=512, d_r=64, d_n=d_v=128, d_model=7168); inputs are
+synthetic and seeded.  The metric is the decode call's latent-cache GB/s:
+the 75.5 MB of cache rows it reads over its time, the median over the K
+timed steps of CUDA events around it inside each step.  The whole step's
+time and the other calls' medians are reported beside it, and (on one GPU)
+the decode of the other configurations under ``workloads``.
 
-Between timed steps the cache rotates over copies whose total exceeds the
-126 MB L2 (and every step also streams the 235 MB W_O), so each step reads
+Between steps the cache rotates over copies whose total exceeds twice the
+126 MB L2 (and every step also streams the 235 MB W_O), so each decode reads
 its cache from HBM.  Under torchrun every rank runs its own batch of 16
-sequences (weak scaling, no collective on the data path); the time is the
-max over ranks.  ``--impl reference`` times the fp64 CPU oracle on a bounded
+sequences (weak scaling, no collective on the data path); times are the max
+over ranks.  ``--gpus N`` with N > 1 outside torchrun starts N ranks under
+torchrun.  ``--impl reference`` times the fp64 CPU oracle on a bounded
 sample of the same workload on the host cores.
 """
 from __future__ import annotations
@@ -32,8 +38,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 WORKLOAD = "bf16_b16_4k"
-METRIC = "absorbed-MLA decode: latent-cache GB/s (% of HBM peak), µs/step at B=16, 4K"
-N_COPIES = 3
+METRIC = ("absorbed-MLA decode call (plan + attention + split merge): latent-cache GB/s "
+          "(% of HBM peak) and µs at B=16, 4K")
 
 
 def _peaks():
@@ -147,7 +153,7 @@ def job_throughput(bytes_per_rank, world, ms_per_step):
 class ClockSampler:
     """Samples SM clock and throttle reasons with NVML in a thread."""
 
-    def __init__(self, index: int, period: float = 0.01):
+    def __init__(self, index: int, period: float = 0.005):
         self.index, self.period = index, period
         self.samples = []
         self._stop = threading.Event()
@@ -184,6 +190,9 @@ class ClockSampler:
         if self._t:
             self._t.join()
 
+    def count(self, t0, t1):
+        return sum(1 for s in self.samples if t0 <= s[0] <= t1)
+
     def summary(self, t0, t1):
         if not self.ok:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
@@ -201,16 +210,151 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- GPU arm
+L2_BYTES = 126 * 2 ** 20
+EXTRA_WORKLOADS = ["bf16_varlen_b64", "redknot_56_8", "bf16_long_256k"]
+
+
+def n_cache_copies(cache_bytes):
+    """Copies of the cache to rotate over so that consecutive decode calls
+    never find their rows in the 126 MB L2 (at least 3, total >= 2 x L2)."""
+    return max(3, -(-2 * L2_BYTES // max(cache_bytes, 1)) + 1)
+
+
+class Problem:
+    """One workload on the device: the uploaded problem, its rotating cache
+    copies and one CUDA graph per call (decode: one per cache copy)."""
+
+    def __init__(self, name, rank, dev, stream):
+        import torch
+
+        from head_latent_attention_02_b200 import mla, runner
+        from head_latent_attention_02_b200.workloads import WORKLOADS, make_inputs
+        self.name = name
+        wl = self.wl = WORKLOADS[name]
+        # the cache is drawn on the device (seeded); nothing here is compared
+        # with the oracle
+        inp = self.inp = make_inputs(wl, seed=rank, poison=False, draw_cache=False)
+        o_off = lse_off = None
+        if wl.n_local:
+            # the Local heads' offline (MLA-Off) partial is an input of the
+            # step: synthetic normalised rows and log-sum-exp values
+            g = np.random.default_rng([rank, 99])
+            o_off = g.standard_normal((inp.n_q, wl.H, wl.d_c)).astype(np.float32) * 0.1
+            lse_off = (g.standard_normal((inp.n_q, wl.H)) + 8.0).astype(np.float32)
+        p = self.p = runner.upload(inp, device=dev, o_off=o_off, lse_off=lse_off,
+                                   device_cache_seed=1000 + rank)
+        # cache rows the decode reads: every sequence's rows, plus the
+        # protected rows the Local heads re-read
+        self.n_read = int(sum(inp.n_rows)) + (int(np.sum(inp.n_gather))
+                                              if inp.n_gather is not None else 0)
+        self.cache_bytes = self.n_read * (wl.d_c + wl.d_r) * 2
+        self.n_copies = n_cache_copies(p.cache.numel() * p.cache.element_size())
+        self.caches = [p.cache] + [p.cache.clone() for _ in range(self.n_copies - 1)]
+        self.stream = stream
+        self.mla, self.runner = mla, runner
+
+        def dec(c):
+            p.cache = self.caches[c]
+            runner.run_decode(p)
+
+        def capture(fn):
+            gr = torch.cuda.CUDAGraph(keep_graph=True)   # keep_graph: nodes stay countable
+            with torch.cuda.graph(gr):
+                fn()
+            gr.instantiate()
+            return gr
+
+        # eager warm-up (loads the kernels, sets attributes) before capture
+        for c in range(self.n_copies):
+            p.cache = self.caches[c]
+            runner.run_step(p, stream=stream)
+        torch.cuda.synchronize(dev)
+        assert mla.get_status(stream) == 0
+        self.g_abs = capture(lambda: mla.absorb_q(p.dims, p.q_nope, p.q_rope, p.q_pos, p.deltas,
+                                                  p.w_uk, p.q_abs))
+        self.g_dec = [capture(lambda c=c: dec(c)) for c in range(self.n_copies)]
+        self.g_out = capture(lambda: mla.out_proj(p.dims, p.o_lat, p.w_uv, p.w_o, p.v, p.out))
+        self.kernels = {"absorb_q": graph_kernel_count(self.g_abs, 1),
+                        "decode": graph_kernel_count(self.g_dec[0], 3),
+                        "out_proj": graph_kernel_count(self.g_out, 2)}
+
+    def steps(self, n, events=None):
+        """n whole steps (absorb_q, decode, out_proj), each call its own graph
+        replay; with ``events`` (a list) record four CUDA events per step:
+        before absorb, before decode, after decode, after out_proj."""
+        import torch
+        for i in range(n):
+            ev = None
+            if events is not None:
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                events.append(ev)
+                ev[0].record(self.stream)
+            self.g_abs.replay()
+            if ev:
+                ev[1].record(self.stream)
+            self.g_dec[i % self.n_copies].replay()
+            if ev:
+                ev[2].record(self.stream)
+            self.g_out.replay()
+            if ev:
+                ev[3].record(self.stream)
+
+    def per_call_us(self, events):
+        """Median over steps of each call's time (µs), from steps' events."""
+        a = [e[0].elapsed_time(e[1]) * 1e3 for e in events]
+        d = [e[1].elapsed_time(e[2]) * 1e3 for e in events]
+        o = [e[2].elapsed_time(e[3]) * 1e3 for e in events]
+        return {"absorb_q": statistics.median(a), "decode": statistics.median(d),
+                "out_proj": statistics.median(o), "decode_min": min(d), "decode_max": max(d),
+                "n": len(events)}
+
+    def roofline(self, t_dec_us, peaks, src, traffic):
+        wl, inp = self.wl, self.inp
+        return decode_roofline(
+            decode_flops(wl, inp.n_rows, inp.n_gather), self.cache_bytes, t_dec_us * 1e-3,
+            peaks, src, traffic,
+            "decode calls of the step (plan + decode_tc + combine"
+            + (", twice, + merge_lse)" if wl.n_local else ")"))
+
+    def release(self):
+        import torch
+        del self.g_abs, self.g_dec, self.g_out, self.caches, self.p
+        torch.cuda.empty_cache()
+
+
+def measure_workload(name, rank, dev, stream, peaks, src, reps=20):
+    """Decode µs (median of ``reps`` steps), cache GB/s and roofline of one
+    more workload on this GPU."""
+    import torch
+    prob = Problem(name, rank, dev, stream)
+    prob.steps(3)
+    ev = []
+    prob.steps(reps, ev)
+    torch.cuda.synchronize(dev)
+    assert prob.mla.get_status(stream) == 0
+    t = prob.per_call_us(ev)
+    out = {"decode_us": round(t["decode"], 2), "decode_us_min": round(t["decode_min"], 2),
+           "repeats": reps, "cache_bytes": prob.cache_bytes,
+           "GB_s": round(prob.cache_bytes / (t["decode"] * 1e-6) / 1e9, 1),
+           "roofline": prob.roofline(t["decode"], peaks, src, None),
+           "config": {"B": prob.wl.B, "H": prob.wl.H, "s_q": prob.wl.s_q,
+                      "rows_total": int(sum(prob.inp.n_rows)),
+                      "n_local_heads": prob.wl.n_local, "cache_copies": prob.n_copies}}
+    prob.release()
+    return out
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
 
-    from head_latent_attention_02_b200 import build as hb, mla, runner
-    from head_latent_attention_02_b200.workloads import WORKLOADS, make_inputs
+    from head_latent_attention_02_b200 import build as hb, mla
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     if world > 1:
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
@@ -221,140 +365,96 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
     mla.lib()
-
-    wl = WORKLOADS[args.workload]
-    inp = make_inputs(wl, seed=rank, poison=False)
-    o_off = lse_off = None
-    if wl.n_local:
-        # the Local heads' offline (MLA-Off) partial is an input of the step:
-        # synthetic normalised rows and log-sum-exp values
-        g = np.random.default_rng([rank, 99])
-        o_off = g.standard_normal((inp.n_q, wl.H, wl.d_c)).astype(np.float32) * 0.1
-        lse_off = (g.standard_normal((inp.n_q, wl.H)) + 8.0).astype(np.float32)
-    p = runner.upload(inp, device=dev, head_order=inp.head_order, o_off=o_off, lse_off=lse_off)
-    caches = [p.cache] + [p.cache.clone() for _ in range(N_COPIES - 1)]
+    peaks, src = _peaks()
     stream = torch.cuda.current_stream(dev)
-    # cache rows the step reads: every sequence's rows, plus the protected
-    # rows the Local heads re-read
-    n_read = int(sum(inp.n_rows)) + (int(np.sum(inp.n_gather)) if inp.n_gather is not None else 0)
-    cache_bytes = n_read * (wl.d_c + wl.d_r) * 2
 
-    def step(i, s=None):
-        # s=None: the binding launches on torch's current stream (the capture
-        # stream while a graph is being recorded)
-        p.cache = caches[i % N_COPIES]
-        runner.run_step(p, stream=s)
-
-    def decode_only(i):
-        p.cache = caches[i % N_COPIES]
-        runner.run_decode(p)
-
-    for i in range(args.warmup):
-        step(i, stream)
-    torch.cuda.synchronize(dev)
-    assert mla.get_status(stream) == 0
-
-    # One CUDA graph per cache copy holds a whole step (6 kernels), so the
-    # timed loop measures the device, not Python's launch overhead.
-    def capture(fn):
-        g = torch.cuda.CUDAGraph(keep_graph=True)   # keep_graph: nodes stay countable
-        with torch.cuda.graph(g):
-            fn()
-        g.instantiate()
-        return g
-
-    g_step = [capture(lambda c=c: step(c)) for c in range(N_COPIES)]
-    g_dec = [capture(lambda c=c: decode_only(c)) for c in range(N_COPIES)]
-    kernels_per_step = graph_kernel_count(g_step[0], 6)
-    kernels_per_decode = graph_kernel_count(g_dec[0], 3)
-    g_abs = capture(lambda: mla.absorb_q(p.dims, p.q_nope, p.q_rope, p.q_pos, p.deltas,
-                                         p.w_uk, p.q_abs))
-    g_out = capture(lambda: mla.out_proj(p.dims, p.o_lat, p.w_uv, p.w_o, p.v, p.out))
-    for i in range(args.warmup):
-        g_step[i % N_COPIES].replay()
-    torch.cuda.synchronize(dev)
-    assert mla.get_status(stream) == 0
-
-    # --- device-timed region (inputs resident in HBM)
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # clocks are sampled over the whole GPU section: set-up, warm-up, the
+    # timed steps, the end-to-end steps and the other workloads
     with ClockSampler(local) as clk:
+        t_gpu0 = time.perf_counter()
+        prob = Problem(args.workload, rank, dev, stream)
+        p = prob.p
+        prob.steps(args.warmup)
+        torch.cuda.synchronize(dev)
+        assert mla.get_status(stream) == 0
+
+        # --- device-timed region: exactly K steps, inputs resident in HBM
+        events = []
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
         t0 = time.perf_counter()
-        start.record(stream)
-        for i in range(args.steps):
-            g_step[i % N_COPIES].replay()
-        stop.record(stream)
+        prob.steps(args.steps, events)
         torch.cuda.synchronize(dev)
         t1 = time.perf_counter()
         if world > 1:
             dist.barrier()
-        clocks = clk.summary(t0, t1)
-    assert mla.get_status(stream) == 0
-    ms_total = start.elapsed_time(stop)
+        assert mla.get_status(stream) == 0
+        ms_total = events[0][0].elapsed_time(events[-1][3])
+        per_call = prob.per_call_us(events)
+        if len(events) < 10:
+            # fewer than 10 timed steps: the per-call medians come from 10 more
+            more = []
+            prob.steps(10, more)
+            torch.cuda.synchronize(dev)
+            per_call = prob.per_call_us(more)
 
-    # --- per-call times: the same calls replayed on their own (decode over the
-    # rotating cache copies; the weight products re-read their weights)
-    def timed(graphs, n):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        for i in range(3):
-            graphs[i % len(graphs)].replay()
-        a.record(stream)
-        for i in range(n):
-            graphs[i % len(graphs)].replay()
-        b.record(stream)
+        # --- end-to-end through the public API with host buffers: each step
+        # copies its queries in from pinned memory and reads `out` back
+        pin_qn = p.q_nope.cpu().pin_memory()
+        pin_qr = p.q_rope.cpu().pin_memory()
+        pin_qp = p.q_pos.cpu().pin_memory()
+        pin_out = torch.empty_like(p.out, device="cpu").pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (pin_qn, pin_qr, pin_qp))
+        d2h = pin_out.numel() * pin_out.element_size()
+
+        def e2e_steps(n):
+            for i in range(n):
+                p.q_nope.copy_(pin_qn, non_blocking=True)
+                p.q_rope.copy_(pin_qr, non_blocking=True)
+                p.q_pos.copy_(pin_qp, non_blocking=True)
+                p.cache = prob.caches[i % prob.n_copies]
+                prob.runner.run_step(p, stream=stream)
+                pin_out.copy_(p.out, non_blocking=True)
+
+        e2e_steps(args.warmup)
         torch.cuda.synchronize(dev)
-        return a.elapsed_time(b) / n
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        s2.record(stream)
+        e2e_steps(args.steps)
+        e2.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = s2.elapsed_time(e2)
+        assert mla.get_status(stream) == 0
+        cache_bytes, wl, inp, kernels = prob.cache_bytes, prob.wl, prob.inp, prob.kernels
+        n_copies = prob.n_copies
+        prob.release()
 
-    n_rep = max(30, min(args.steps, 300))
-    t_dec = timed(g_dec, n_rep)
-    t_abs = timed([g_abs], n_rep)
-    t_out = timed([g_out], n_rep)
-    assert mla.get_status(stream) == 0
+        # --- the other configurations, decode only, on this GPU
+        workloads = {}
+        if world == 1 and not args.no_workloads and args.workload == WORKLOAD:
+            for name in EXTRA_WORKLOADS:
+                workloads[name] = measure_workload(name, rank, dev, stream, peaks, src)
+        t_gpu1 = time.perf_counter()
+    clocks = clk.summary(t_gpu0, t_gpu1)
+    clocks["timed_window_samples"] = clk.count(t0, t1)
 
-    # --- end-to-end through the public API with host buffers
-    pin_qn = p.q_nope.cpu().pin_memory()
-    pin_qr = p.q_rope.cpu().pin_memory()
-    pin_qp = p.q_pos.cpu().pin_memory()
-    pin_out = torch.empty_like(p.out, device="cpu").pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (pin_qn, pin_qr, pin_qp))
-    d2h = pin_out.numel() * pin_out.element_size()
-
-    def e2e_step(i):
-        p.q_nope.copy_(pin_qn, non_blocking=True)
-        p.q_rope.copy_(pin_qr, non_blocking=True)
-        p.q_pos.copy_(pin_qp, non_blocking=True)
-        step(i, stream)
-        pin_out.copy_(p.out, non_blocking=True)
-
-    for i in range(args.warmup):
-        e2e_step(i)
-    torch.cuda.synchronize(dev)
-    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    s2.record(stream)
-    for i in range(args.steps):
-        e2e_step(i)
-    e2.record(stream)
-    torch.cuda.synchronize(dev)
-    ms_e2e = s2.elapsed_time(e2)
-
-    ms_total, ms_e2e = max_over_ranks([ms_total, ms_e2e], dev, world)
+    t_dec_ms, ms_total, ms_e2e = max_over_ranks(
+        [per_call["decode"] * 1e-3, ms_total, ms_e2e], dev, world)
     if world > 1:
         dist.barrier()
 
     if rank == 0:
-        peaks, src = _peaks()
         ms_step = ms_total / args.steps
-        value = job_throughput(cache_bytes, world, ms_step)
+        value = job_throughput(cache_bytes, world, t_dec_ms)
         e2e_val = job_throughput(cache_bytes, world, ms_e2e / args.steps)
-        achieved = cache_bytes / (t_dec * 1e-3) / 1e9
+        per_step_kernels = sum(kernels.values())
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_dec_ms, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) latents/queries, N(0,1/fan_in) weights)",
             "config": {"workload": args.workload, "B": wl.B, "H": wl.H,
@@ -365,33 +465,54 @@ def run_gpu(args):
                        "d_model": wl.d_model, "page": 64, "s_q": wl.s_q,
                        "n_local_heads": wl.n_local,
                        "cache_bytes_per_step": cache_bytes,
-                       "l2": f"cache rotates over {N_COPIES} copies "
-                             f"({N_COPIES * cache_bytes / 1e6:.0f} MB) and each step streams "
+                       "l2": f"cache rotates over {n_copies} copies "
+                             f"({n_copies * cache_bytes / 1e6:.0f} MB) and each step streams "
                              f"W_O ({wl.d_model * wl.H * wl.d_v * 2 / 1e6:.0f} MB)",
                        "parallelism": f"replica x{world} (independent batches)"},
-            "timing": "CUDA graph per step (6 kernels), CUDA events around the K replays",
-            "breakdown_us": {"absorb_q": round(t_abs * 1e3, 2), "decode": round(t_dec * 1e3, 2),
-                             "out_proj": round(t_out * 1e3, 2),
-                             "how": "each call's own graph replayed back to back"},
-            "decode_only": {"us": round(t_dec * 1e3, 2), "GB_s": round(achieved, 1),
-                            "kernels": kernels_per_decode},
+            "timing": ("value and ms_per_step: the decode call (plan + attention + split "
+                       "merge), median over the K timed steps of CUDA events around its graph "
+                       "inside each step (absorb_q, decode, out_proj graphs replayed in order); "
+                       "step_ms: the whole step, first event to last over K"),
+            "step_ms": round(ms_step, 5),
+            "step_GB_s": round(job_throughput(cache_bytes, world, ms_step), 2),
+            "breakdown_us": {"absorb_q": round(per_call["absorb_q"], 2),
+                             "decode": round(per_call["decode"], 2),
+                             "out_proj": round(per_call["out_proj"], 2),
+                             "decode_min": round(per_call["decode_min"], 2),
+                             "decode_max": round(per_call["decode_max"], 2),
+                             "repeats": per_call["n"], "how": "median per call over the steps"},
             "roofline": decode_roofline(
-                decode_flops(wl, inp.n_rows, inp.n_gather), cache_bytes, t_dec, peaks, src,
+                decode_flops(wl, inp.n_rows, inp.n_gather), cache_bytes, t_dec_ms, peaks, src,
                 decode_traffic() if args.workload == WORKLOAD else None,
                 "decode calls of the step (plan + decode_tc + combine"
                 + (", twice, + merge_lse)" if wl.n_local else ")")),
             "clocks": clocks,
             "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
-            "gpu_launches": kernels_per_step * args.steps,
-            "gpu_launches_note": f"{kernels_per_step} kernel nodes per step graph (absorb, "
-                                 "decode plan, attention, split merge, W_UV, W_O)",
+                    "d2h_bytes_per_step": d2h,
+                    "how": "whole step through the public API (H2D queries, absorb, decode, "
+                           "out_proj, D2H out), cache bytes over the step time"},
+            "gpu_launches": per_step_kernels * args.steps,
+            "gpu_launches_note": f"{per_step_kernels} kernel nodes per step ({kernels})",
         }
+        if workloads:
+            line["workloads"] = workloads
         if world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD:
             line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def relaunch_under_torchrun(n):
+    """`--gpus N` (N > 1) outside torchrun: run this script again as N ranks."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__)] + sys.argv[1:]
+    os.execv(sys.executable, cmd)
 
 
 # ---------------------------------------------------------------- CPU arm
@@ -467,7 +588,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
     ap.add_argument("--workload", default=WORKLOAD,
@@ -475,8 +596,14 @@ def main():
                          "bf16_long_256k")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the decode timings of the other configurations")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.gpus < 1:
+        raise SystemExit("--gpus must be >= 1")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        relaunch_under_torchrun(args.gpus)
     if args.impl == "reference":
         run_reference(args)
     else:

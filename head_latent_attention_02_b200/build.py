@@ -7,9 +7,11 @@ import subprocess
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libmla.so")
-SOURCES = ["csrc/mla_lib.cu", "csrc/mla_static_ws.cu"]
-DEPENDS = ["csrc/mla_lib.cu", "csrc/mla_static_ws.cu", "csrc/common.cuh", "csrc/ptx.cuh",
-           "csrc/kernels_simt.cuh", "csrc/wgemm.cuh", "csrc/decode_tc.cuh", "../include/mla.h"]
+SOURCES = ["csrc/mla_lib.cu", "csrc/mla_static_ws.cu", "csrc/mla_append.cu",
+           "csrc/mla_qknorm.cu"]
+DEPENDS = ["csrc/mla_lib.cu", "csrc/mla_static_ws.cu", "csrc/mla_append.cu", "csrc/mla_qknorm.cu",
+           "csrc/common.cuh",
+           "csrc/ptx.cuh", "csrc/kernels_simt.cuh", "csrc/wgemm.cuh", "csrc/decode_tc.cuh", "../include/mla.h"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

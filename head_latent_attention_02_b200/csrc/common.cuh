@@ -36,7 +36,10 @@ constexpr float kNegInf = -__builtin_huge_valf();
 
 // Description of one mla_decode call as the kernels see it.
 struct DecodeArgs {
-  int B, s_q, n_q, H, h0, n_h, d_c, d_r, n_ver;
+  int B, s_q, n_q, H, n_h, d_c, d_r, n_ver;
+  int qH;                       // heads per query row of the q_abs the kernels read
+  const int32_t* head_ids;      // [n_h] output head of each decoded head, or null = 0..n_h-1
+  const float* key_inv;         // QK-normed decode: [n_pages * 64] inverse key RMS per cache row
   int max_pages, max_segs, max_gather;
   long long n_pages;
   float scale;
@@ -50,6 +53,19 @@ struct DecodeArgs {
   float* o_lat;
   float* lse;
 };
+
+// Output head of the k-th decoded head: head_ids[k], or k when the call gives
+// no list.  An id outside [0, H) records MLA_ERR_BAD_INDEX and yields -1 (the
+// head's results are not written).
+__device__ __forceinline__ int head_of(const DecodeArgs& a, int k) {
+  if (!a.head_ids) return k;
+  const int h = __ldg(a.head_ids + k);
+  if (h < 0 || h >= a.H) {
+    set_status(MLA_ERR_BAD_INDEX);
+    return -1;
+  }
+  return h;
+}
 
 // Cache row of attended index `i` of sequence b (page mode: i-th row of the
 // concatenated segments; gather mode: gather_rows[b][i]).  Returns false when

@@ -642,7 +642,7 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
           // the head block's absorbed queries: the rotary panel into its own
           // buffer, the 8 latent panels through the ring as three stages
           // (panels 0-2, 3-5, 6-8; the copy to tensor memory skips panel 8)
-          const int qrow = (d.ver * a.n_q + sp.b * a.s_q + sp.j) * a.H + a.h0 + sp.hb * kM;
+          const int qrow = (d.ver * a.n_q + sp.b * a.s_q + sp.j) * a.qH + sp.hb * kM;
           if (!wait_warp(&bar->qr_empty, (nq & 1) ^ 1)) { fail(ok); break; }
           if (lane == 0) {
             mbar_arrive_expect_tx(&bar->qr_full, kSlot);
@@ -794,6 +794,20 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
         const uint64_t vis = visibility<kGather>(a, d, sp.b, hf, lane);
         const uint32_t v0 = (uint32_t)vis, v1 = (uint32_t)(vis >> 32);
         const int sb = it & 1, pb = it & 1;
+        // QK-normed scores: one factor per column, the key's inverse RMS,
+        // read for this half's page before the wait so the loads overlap it
+        float kf[64];
+        if (!kGather && a.key_inv) {
+          const float4* src = reinterpret_cast<const float4*>(a.key_inv + (hf ? d.phys1 : d.phys0));
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float4 f = __ldg(src + j);
+            kf[4 * j] = f.x;
+            kf[4 * j + 1] = f.y;
+            kf[4 * j + 2] = f.z;
+            kf[4 * j + 3] = f.w;
+          }
+        }
         if (!wait_warp(&bar->s_full[sb], (it >> 1) & 1)) { fail(ok); break; }
         tc_fence_after();
         float x[64];
@@ -803,6 +817,10 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar->s_empty[sb]);
+        if (!kGather && a.key_inv) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) x[c] *= kf[c];
+        }
 
         // max of this half's visible scores (four independent chains), then
         // of the row, through the partner warp (log2 units)
@@ -1019,10 +1037,18 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
           const bool empty = !(l_tot > 0.f);
           const float inv = empty ? 0.f : 1.f / l_tot;
           const float lse = empty ? -INFINITY : (m_fin + log2f(l_tot)) * 0.6931471805599453f;
-          const int hrow0 = sp.hb * kM + quad * 32;        // first head row of this warp
-          float* dst0 = whole ? a.o_lat + ((size_t)qi * a.H + a.h0 + hrow0) * kDc
-                              : p.partial + ((size_t)slot * kM + quad * 32) * kDc;
-          const int live = whole ? min(32, a.n_h - hrow0) : 32;   // rows this warp may write
+          // Destination of this lane's head row: the split slot's row, or the
+          // output head's row of o_lat (none past n_h or for an invalid id).
+          const int my_head = sp.hb * kM + h < a.n_h ? head_of(a, sp.hb * kM + h) : -1;
+          float* my_dst = !whole ? p.partial + ((size_t)slot * kM + h) * kDc
+                        : my_head >= 0 ? a.o_lat + ((size_t)qi * a.H + my_head) * kDc
+                                       : nullptr;
+          // the rows this lane stores: 4 k + lane / 8 for k = 0..7
+          float* dst_row[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            dst_row[k] = reinterpret_cast<float*>(__shfl_sync(
+                0xffffffffu, reinterpret_cast<unsigned long long>(my_dst), 4 * k + (lane >> 3)));
           // O rows leave through a per-warp staging tile: each lane writes its
           // row's 32 columns, then each store instruction writes 4 rows x 128 B.
           // The next 32 columns are read from tensor memory while this chunk's
@@ -1042,9 +1068,8 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
               const int rr = 4 * k + (lane >> 3), j = lane & 7;
-              if (rr < live)
-                *reinterpret_cast<float4*>(dst0 + (size_t)rr * kDc + c + 4 * j) =
-                    stage[rr * 8 + (j ^ (rr & 7))];
+              if (dst_row[k])
+                *reinterpret_cast<float4*>(dst_row[k] + c + 4 * j) = stage[rr * 8 + (j ^ (rr & 7))];
             }
             __syncwarp();
             if (c + 32 < kDc) {
@@ -1054,10 +1079,8 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
             }
           }
           tc_fence_before();
-          if (sp.hb * kM + h < a.n_h) {
-            if (whole) a.lse[(size_t)qi * a.H + a.h0 + sp.hb * kM + h] = lse;
-            else p.partial_lse[(size_t)slot * kM + h] = lse;
-          }
+          if (!whole) p.partial_lse[(size_t)slot * kM + h] = lse;
+          else if (my_head >= 0) a.lse[(size_t)qi * a.H + my_head] = lse;
           ++n_str;
         }
       }
@@ -1241,7 +1264,9 @@ __global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a, int n_hb,
   const int rows = min(kM, a.n_h - hb * kM);
   if (m >= rows) return;
   const int T = stream_off[s + 1] - stream_off[s];
-  const size_t orow = (size_t)qi * a.H + a.h0 + hb * kM + m;
+  const int head = head_of(a, hb * kM + m);
+  if (head < 0) return;
+  const size_t orow = (size_t)qi * a.H + head;
   float* o = a.o_lat + orow * kDc;
   if (T == 0) {
     const float fill = stream_bad[s] ? __int_as_float(0x7fc00000) : 0.f;

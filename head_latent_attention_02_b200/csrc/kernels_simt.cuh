@@ -84,7 +84,8 @@ __global__ void __launch_bounds__(256) absorb_kernel(AbsorbArgs a) {
 template <typename T>
 __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeArgs a) {
   extern __shared__ float sm_dec[];
-  const int h = a.h0 + blockIdx.x;
+  const int h = head_of(a, blockIdx.x);
+  if (h < 0) return;
   const int qi = blockIdx.y;
   const int b = qi / a.s_q;
   const int row = a.d_c + a.d_r;
@@ -121,6 +122,7 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeArgs a) {
           float d = 0.f;
           for (int k = 0; k < row; ++k) d = fmaf(q[k], to_f(r[k]), d);
           s = d * a.scale;
+          if (a.key_inv) s *= a.key_inv[phys];
         }
       } else {
         phys = -1;
@@ -135,7 +137,7 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeArgs a) {
     __syncthreads();
     const float m_new = fmaxf(m_run, mx);
     float p = 0.f;
-    if (s != kNegInf) p = __expf(s - m_new);
+    if (s != kNegInf) p = expf(s - m_new);
     pw[tid] = p;
     prow[tid] = (p != 0.f) ? phys : -1;
     float sum = p;
@@ -143,7 +145,7 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeArgs a) {
     if ((tid & 31) == 0) red[tid >> 5] = sum;
     __syncthreads();
     sum = red[0] + red[1] + red[2] + red[3];
-    const float corr = (m_run == kNegInf) ? 0.f : __expf(m_run - m_new);
+    const float corr = (m_run == kNegInf) ? 0.f : expf(m_run - m_new);
     if (m_new != kNegInf) {
       l_run = l_run * corr + sum;
       for (int c = tid; c < a.d_c; c += 128) {
@@ -166,11 +168,37 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Gather of the listed heads' absorbed queries into a dense block:
+// q_pack[v, q, k, :] = q_abs[v, q, head_ids[k], :], so the tensor-core decode
+// loads a block of heads with one box whatever the list.  One warp per packed
+// row, 16-byte copies (row_bytes is a multiple of 16); an invalid id gives a
+// zero row, whose results the decode does not write.  256 threads per block.
+__global__ void __launch_bounds__(256) pack_heads_kernel(int rows_out, int n_h, int H,
+                                                         int row_bytes, const int32_t* head_ids,
+                                                         const uint8_t* q_abs, uint8_t* q_pack) {
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= rows_out) return;
+  const int vq = r / n_h, k = r % n_h;
+  const int h = __ldg(head_ids + k);
+  const int n16 = row_bytes / 16;
+  uint4* dst = reinterpret_cast<uint4*>(q_pack + (size_t)r * row_bytes);
+  if (h < 0 || h >= H) {
+    for (int i = lane; i < n16; i += 32) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(q_abs + ((size_t)vq * H + h) * row_bytes);
+  for (int i = lane; i < n16; i += 32) dst[i] = __ldg(src + i);
+}
+
+// ---------------------------------------------------------------------------
 // Log-sum-exp merge of two partial attentions (RedKnot-MLA abstract: offline
 // and online paths merged before the shared output projection).  One warp per
-// (query row, head); every lane reads both lse values before lane 0 writes
-// the merged one, so lse may alias lse_a or lse_b.  256 threads per block.
-__global__ void __launch_bounds__(256) merge_lse_kernel(int n_q, int H, int h0, int n_h, int d,
+// (query row, listed head); every lane reads both lse values before lane 0
+// writes the merged one, so lse may alias lse_a or lse_b.  head_ids [n_h]
+// names the heads (null: 0..n_h-1).  256 threads per block.
+__global__ void __launch_bounds__(256) merge_lse_kernel(int n_q, int H, const int32_t* head_ids,
+                                                        int n_h, int d,
                                                         const float* o_a, const float* lse_a,
                                                         const float* o_b, const float* lse_b,
                                                         float* o, float* lse) {
@@ -178,13 +206,18 @@ __global__ void __launch_bounds__(256) merge_lse_kernel(int n_q, int H, int h0, 
   const int lane = threadIdx.x & 31;
   if (wid >= (long long)n_q * n_h) return;
   const int q = (int)(wid / n_h), hh = (int)(wid % n_h);
-  const size_t r = (size_t)q * H + h0 + hh;
+  const int h = head_ids ? __ldg(head_ids + hh) : hh;
+  if (h < 0 || h >= H) {
+    if (lane == 0) set_status(MLA_ERR_BAD_INDEX);
+    return;
+  }
+  const size_t r = (size_t)q * H + h;
   const float la = lse_a[r], lb = lse_b[r];
   const float m = fmaxf(la, lb);
   float wa = 0.f, wb = 0.f, out_l = kNegInf;
   if (m != kNegInf) {
-    wa = __expf(la - m);
-    wb = __expf(lb - m);
+    wa = expf(la - m);
+    wb = expf(lb - m);
     const float tot = wa + wb;
     out_l = m + logf(tot);
     wa /= tot;

@@ -16,6 +16,9 @@
 #include "decode_tc.cuh"
 #include "wgemm.cuh"
 
+namespace mla {
+int append_take_status();   // the cache writer's module (mla_append.cu)
+}
 using namespace mla;
 
 namespace {
@@ -223,12 +226,19 @@ mla_status_t launch_wgemm(wg::Params p, const void* w, uint64_t w_rows, uint64_t
 }
 
 struct WsLayout {
-  size_t off_plan, off_streams, off_bad, off_pairs, off_partial, off_plse, total;
+  size_t off_plan, off_streams, off_bad, off_pairs, off_partial, off_plse, off_qpack, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-WsLayout ws_layout(int n_streams, int G) {
+// Bytes of the packed queries of a call with a head list (tensor-core path).
+size_t q_pack_bytes(const mla_dims_t* dims, int B, int s_q, int n_ver, int n_h) {
+  return align256((size_t)n_ver * B * s_q * n_h * (dims->d_c + dims->d_r) * elem_size(dims));
+}
+
+// q_pack_bytes: room for the listed heads' packed queries (mla_decode with a
+// head list).
+WsLayout ws_layout(int n_streams, int G, size_t q_pack_bytes) {
   WsLayout w;
   w.off_plan = 0;
   w.off_streams = align256(sizeof(tc::PlanHeader));
@@ -237,7 +247,8 @@ WsLayout ws_layout(int n_streams, int G) {
   w.off_pairs = w.off_bad + align256(sizeof(int) * (size_t)n_streams);
   w.off_partial = w.off_pairs + align256(sizeof(int) * (size_t)G);
   w.off_plse = w.off_partial + sizeof(float) * (size_t)tc::kDc * tc::kM * 2 * (size_t)G;
-  w.total = w.off_plse + sizeof(float) * (size_t)tc::kM * 2 * (size_t)G;
+  w.off_qpack = align256(w.off_plse + sizeof(float) * (size_t)tc::kM * 2 * (size_t)G);
+  w.total = w.off_qpack + q_pack_bytes;
   return w;
 }
 
@@ -271,7 +282,8 @@ mla_status_t mla_get_status(mla_stream_t stream) {
   if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
   const int zero = 0;
   if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
-  return static_cast<mla_status_t>(v);
+  const int va = mla::append_take_status();
+  return static_cast<mla_status_t>(v ? v : va);
 }
 
 mla_status_t mla_absorb_q(const mla_dims_t* dims, int32_t n_q, const void* q_nope,
@@ -329,24 +341,33 @@ mla_status_t mla_absorb_q(const mla_dims_t* dims, int32_t n_q, const void* q_nop
   return launch_ok();
 }
 
-size_t mla_decode_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t n_h) {
-  if (!dims_ok(dims) || B < 0 || s_q < 1 || n_h < 1) return 0;
+size_t mla_decode_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q, int32_t n_ver,
+                                 int32_t n_h) {
+  if (!dims_ok(dims) || B < 0 || s_q < 1 || n_ver < 1 || n_ver > kMaxVersions || n_h < 1 ||
+      n_h > dims->H)
+    return 0;
   if (!tc_eligible(dims)) return 256;   // the generic kernel needs no scratch
   DeviceInfo* d = nullptr;
   if (device_info(&d) != MLA_OK) return 0;
   const int n_hb = (n_h + tc::kM - 1) / tc::kM;
-  return ws_layout(B * s_q * n_hb, d->num_sms / 2).total;
+  return ws_layout(B * s_q * n_hb, d->num_sms / 2, q_pack_bytes(dims, B, s_q, n_ver, n_h)).total;
 }
 
-mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const void* q_abs,
-                        int32_t n_ver, int32_t h0, int32_t n_h, const void* cache,
-                        int64_t n_pages, const int32_t* block_table, int32_t max_pages,
-                        const mla_seg_t* segs, int32_t max_segs, const int32_t* gather_rows,
-                        const int32_t* n_gather, int32_t max_gather, const int32_t* q_pos,
-                        float* o_lat, float* lse, void* workspace, size_t ws_bytes,
-                        mla_stream_t stream) {
-  if (!dims_ok(dims) || B < 0 || s_q < 1 || n_ver < 1 || h0 < 0 || n_h < 1 ||
-      h0 + n_h > dims->H || n_pages < 1 || max_pages < 1 || max_segs < 1)
+}  // extern "C"
+
+namespace {
+
+// mla_decode and mla_decode_qknorm: key_inv (or null) is the per-row inverse
+// key RMS of the QK-normed scores.
+mla_status_t decode_impl(const mla_dims_t* dims, int32_t B, int32_t s_q, const void* q_abs,
+                         int32_t n_ver, const int32_t* head_ids, int32_t n_h, const void* cache,
+                         int64_t n_pages, const int32_t* block_table, int32_t max_pages,
+                         const mla_seg_t* segs, int32_t max_segs, const int32_t* gather_rows,
+                         const int32_t* n_gather, int32_t max_gather, const int32_t* q_pos,
+                         float* o_lat, float* lse, void* workspace, size_t ws_bytes,
+                         mla_stream_t stream, const float* key_inv) {
+  if (!dims_ok(dims) || B < 0 || s_q < 1 || n_ver < 1 || n_h < 1 || n_h > dims->H ||
+      n_pages < 1 || max_pages < 1 || max_segs < 1)
     return MLA_ERR_INVALID_ARG;
   if (dims->page_size != kPage || n_ver > kMaxVersions) return MLA_ERR_UNSUPPORTED;
   if (gather_rows && (!n_gather || max_gather < 1)) return MLA_ERR_INVALID_ARG;
@@ -359,15 +380,20 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
       (long long)n_ver * B * s_q * dims->H > INT32_MAX)
     return MLA_ERR_UNSUPPORTED;
   const size_t es = elem_size(dims);
-  if (!aligned(cache, 256) || !aligned(q_abs, 16) || !aligned(o_lat, 16) || !aligned(lse, 4))
+  if (!aligned(cache, 256) || !aligned(q_abs, 16) || !aligned(o_lat, 16) || !aligned(lse, 4) ||
+      !aligned(key_inv, 16))
     return MLA_ERR_INVALID_ARG;
+  // the per-row factors are read per page: gathered rows have no page run
+  if (key_inv && gather_rows) return MLA_ERR_UNSUPPORTED;
 
   DecodeArgs a;
   a.B = B;
   a.s_q = s_q;
   a.n_q = B * s_q;
   a.H = dims->H;
-  a.h0 = h0;
+  a.qH = dims->H;
+  a.head_ids = head_ids;
+  a.key_inv = key_inv;
   a.n_h = n_h;
   a.d_c = dims->d_c;
   a.d_r = dims->d_r;
@@ -407,15 +433,29 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
   const int G = dev->num_sms / 2;
   const int n_hb = (n_h + tc::kM - 1) / tc::kM;
   const int n_streams = B * s_q * n_hb;
-  const WsLayout wl = ws_layout(n_streams, G);
+  const WsLayout wl = ws_layout(n_streams, G, q_pack_bytes(dims, B, s_q, n_ver, n_h));
   if (!workspace || ws_bytes < wl.total) return MLA_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return MLA_ERR_INVALID_ARG;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+  // A head list is resolved on the device: the listed heads' queries are
+  // packed densely, and the kernels write each result to its listed head.
+  const void* q_src = q_abs;
+  if (head_ids) {
+    const int rows_out = n_ver * B * s_q * n_h;
+    pack_heads_kernel<<<(rows_out + 7) / 8, 256, 0, st>>>(
+        rows_out, n_h, dims->H, (int)(tc::kRow * es), head_ids,
+        static_cast<const uint8_t*>(q_abs), ws + wl.off_qpack);
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    q_src = ws + wl.off_qpack;
+    a.qH = n_h;
+  }
 
   tc::Maps maps;
   const uint64_t cache_rows = (uint64_t)n_pages * kPage;
-  const uint64_t q_rows = (uint64_t)n_ver * B * s_q * dims->H;
-  if (!make_map_576(&maps.q3, q_abs, q_rows, 3, tc::kM, tc::kStagePanels) ||
-      !make_map_576(&maps.qr, q_abs, q_rows, 2, tc::kM) ||
+  const uint64_t q_rows = (uint64_t)n_ver * B * s_q * a.qH;
+  if (!make_map_576(&maps.q3, q_src, q_rows, 3, tc::kM, tc::kStagePanels) ||
+      !make_map_576(&maps.qr, q_src, q_rows, 2, tc::kM) ||
       !make_map_576(&maps.k3, cache, cache_rows, 3, tc::kT, tc::kStagePanels) ||
       !make_map_576(&maps.kp, cache, cache_rows, 2, tc::kPg) ||
       !make_map_576(&maps.vp, cache, cache_rows, 3, tc::kPg, 8) ||
@@ -437,7 +477,6 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
   }
   // page mode and gathered-row mode are separate instantiations
   const bool gather = gather_rows != nullptr;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
   tc::PlanHeader* plan = reinterpret_cast<tc::PlanHeader*>(ws + wl.off_plan);
   int* stream_off = reinterpret_cast<int*>(ws + wl.off_streams);
   int* stream_bad = reinterpret_cast<int*>(ws + wl.off_bad);
@@ -490,10 +529,39 @@ mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const vo
   return launch_ok();
 }
 
-mla_status_t mla_merge_lse(int32_t n_q, int32_t H, int32_t h0, int32_t n_h, int32_t d,
-                           const float* o_a, const float* lse_a, const float* o_b,
+}  // namespace
+
+extern "C" {
+
+mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const void* q_abs,
+                        int32_t n_ver, const int32_t* head_ids, int32_t n_h, const void* cache,
+                        int64_t n_pages, const int32_t* block_table, int32_t max_pages,
+                        const mla_seg_t* segs, int32_t max_segs, const int32_t* gather_rows,
+                        const int32_t* n_gather, int32_t max_gather, const int32_t* q_pos,
+                        float* o_lat, float* lse, void* workspace, size_t ws_bytes,
+                        mla_stream_t stream) {
+  return decode_impl(dims, B, s_q, q_abs, n_ver, head_ids, n_h, cache, n_pages, block_table,
+                     max_pages, segs, max_segs, gather_rows, n_gather, max_gather, q_pos, o_lat,
+                     lse, workspace, ws_bytes, stream, nullptr);
+}
+
+mla_status_t mla_decode_qknorm(const mla_dims_t* dims, int32_t B, int32_t s_q, const void* q_abs,
+                               int32_t n_ver, const int32_t* head_ids, int32_t n_h,
+                               const void* cache, const float* key_inv_rms, int64_t n_pages,
+                               const int32_t* block_table, int32_t max_pages,
+                               const mla_seg_t* segs, int32_t max_segs, const int32_t* q_pos,
+                               float* o_lat, float* lse, void* workspace, size_t ws_bytes,
+                               mla_stream_t stream) {
+  if (!key_inv_rms) return MLA_ERR_INVALID_ARG;
+  return decode_impl(dims, B, s_q, q_abs, n_ver, head_ids, n_h, cache, n_pages, block_table,
+                     max_pages, segs, max_segs, nullptr, nullptr, 0, q_pos, o_lat, lse,
+                     workspace, ws_bytes, stream, key_inv_rms);
+}
+
+mla_status_t mla_merge_lse(int32_t n_q, int32_t H, const int32_t* head_ids, int32_t n_h,
+                           int32_t d, const float* o_a, const float* lse_a, const float* o_b,
                            const float* lse_b, float* o, float* lse, mla_stream_t stream) {
-  if (n_q < 0 || H < 1 || h0 < 0 || n_h < 1 || h0 + n_h > H || d < 1) return MLA_ERR_INVALID_ARG;
+  if (n_q < 0 || H < 1 || n_h < 1 || n_h > H || d < 1) return MLA_ERR_INVALID_ARG;
   if (n_q == 0) return MLA_OK;
   if (!o_a || !lse_a || !o_b || !lse_b || !o || !lse) return MLA_ERR_INVALID_ARG;
   DeviceInfo* dev = nullptr;
@@ -502,7 +570,7 @@ mla_status_t mla_merge_lse(int32_t n_q, int32_t H, int32_t h0, int32_t n_h, int3
   const long long blocks = (rows + 7) / 8;
   if (blocks > INT32_MAX) return MLA_ERR_INVALID_ARG;
   merge_lse_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      n_q, H, h0, n_h, d, o_a, lse_a, o_b, lse_b, o, lse);
+      n_q, H, head_ids, n_h, d, o_a, lse_a, o_b, lse_b, o, lse);
   return launch_ok();
 }
 

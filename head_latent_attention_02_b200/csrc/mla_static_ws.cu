@@ -12,13 +12,9 @@
 // that call this entry point, not by every user of the library.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "mla.h"
 
 namespace {
-
-constexpr int kMaxDevices = 64;
 
 // Scratch shared by every call on a device.  It keeps the previous call's
 // contents; nothing in it has to start at zero, because the planning kernel
@@ -28,39 +24,50 @@ constexpr int kMaxDevices = 64;
 // or other host threads) use the same bytes and race.
 static __device__ __align__(256) unsigned char g_decode_scratch[MLA_DECODE_STATIC_WS_BYTES];
 
-void* g_scratch_ptr[kMaxDevices] = {};
-std::mutex g_scratch_mu;
-
-// Set-up, once per device with that device current: the device address of
-// the array in this context.  Runs inside the first call on each device.
+// The device address of the array in the current context.  The lookup runs
+// on every call: it is a table read once the module is loaded, and it stays
+// right across a device reset or a change of context, which a cached pointer
+// would not.
 mla_status_t scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
-  std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return MLA_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) {
+    cudaGetLastError();   // clear the error the failed lookup recorded
+    return MLA_ERR_CUDA;
   }
-  *out = g_scratch_ptr[dev];
+  *out = p;
   return MLA_OK;
 }
 
 }  // namespace
 
+extern "C" mla_status_t mla_decode_static_ws_init(void) {
+  void* p = nullptr;
+  return scratch_address(&p);
+}
+
 extern "C" mla_status_t mla_decode_static_ws(
-    const mla_dims_t* dims, int32_t B, int32_t s_q, const void* q_abs, int32_t n_ver, int32_t h0,
-    int32_t n_h, const void* cache, int64_t n_pages, const int32_t* block_table,
-    int32_t max_pages, const mla_seg_t* segs, int32_t max_segs, const int32_t* gather_rows,
-    const int32_t* n_gather, int32_t max_gather, const int32_t* q_pos, float* o_lat, float* lse,
-    mla_stream_t stream) {
-  const size_t need = mla_decode_workspace_size(dims, B, s_q, n_h);
+    const mla_dims_t* dims, int32_t B, int32_t s_q, const void* q_abs, int32_t n_ver,
+    const int32_t* head_ids, int32_t n_h, const void* cache, int64_t n_pages,
+    const int32_t* block_table, int32_t max_pages, const mla_seg_t* segs, int32_t max_segs,
+    const int32_t* gather_rows, const int32_t* n_gather, int32_t max_gather, const int32_t* q_pos,
+    float* o_lat, float* lse, mla_stream_t stream) {
+  // the size query answers 0 both for invalid sizes and for a device that
+  // cannot be queried: tell the two apart before trusting it
+  if (!dims || B < 0 || s_q < 1 || n_ver < 1 || n_h < 1 || n_h > dims->H)
+    return MLA_ERR_INVALID_ARG;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MLA_ERR_CUDA;
+  }
+  const size_t need = mla_decode_workspace_size(dims, B, s_q, n_ver, n_h);
   if (need == 0) return MLA_ERR_INVALID_ARG;
   if (need > MLA_DECODE_STATIC_WS_BYTES) return MLA_ERR_WORKSPACE;
   void* ws = nullptr;
   const mla_status_t st = scratch_address(&ws);
   if (st != MLA_OK) return st;
-  return mla_decode(dims, B, s_q, q_abs, n_ver, h0, n_h, cache, n_pages, block_table, max_pages,
-                    segs, max_segs, gather_rows, n_gather, max_gather, q_pos, o_lat, lse, ws,
-                    MLA_DECODE_STATIC_WS_BYTES, stream);
+  return mla_decode(dims, B, s_q, q_abs, n_ver, head_ids, n_h, cache, n_pages, block_table,
+                    max_pages, segs, max_segs, gather_rows, n_gather, max_gather, q_pos, o_lat,
+                    lse, ws, MLA_DECODE_STATIC_WS_BYTES, stream);
 }

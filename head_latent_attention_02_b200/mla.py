@@ -43,13 +43,21 @@ _SIGS = {
     "mla_get_status": ([_vp], _i32),
     "mla_absorb_q": ([ctypes.POINTER(Dims), _i32, _vp, _vp, _vp, ctypes.POINTER(_i32), _i32, _vp,
                       _vp, _vp], _i32),
-    "mla_decode": ([ctypes.POINTER(Dims), _i32, _i32, _vp, _i32, _i32, _i32, _vp, _i64, _vp, _i32,
+    "mla_decode": ([ctypes.POINTER(Dims), _i32, _i32, _vp, _i32, _vp, _i32, _vp, _i64, _vp, _i32,
                     _vp, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
-    "mla_decode_workspace_size": ([ctypes.POINTER(Dims), _i32, _i32, _i32], _sz),
-    "mla_decode_static_ws": ([ctypes.POINTER(Dims), _i32, _i32, _vp, _i32, _i32, _i32, _vp, _i64,
+    "mla_decode_workspace_size": ([ctypes.POINTER(Dims), _i32, _i32, _i32, _i32], _sz),
+    "mla_decode_static_ws": ([ctypes.POINTER(Dims), _i32, _i32, _vp, _i32, _vp, _i32, _vp, _i64,
                               _vp, _i32, _vp, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _vp], _i32),
-    "mla_merge_lse": ([_i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
+    "mla_decode_static_ws_init": ([], _i32),
+    "mla_merge_lse": ([_i32, _i32, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
     "mla_out_proj": ([ctypes.POINTER(Dims), _i32, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
+    "mla_append_rows": ([ctypes.POINTER(Dims), _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i64,
+                         _vp, _i32, _vp, ctypes.c_float, _vp, _vp], _i32),
+    "mla_qknorm_query": ([ctypes.POINTER(Dims), _i32, _vp, _vp, _vp, ctypes.c_float, _vp, _vp],
+                         _i32),
+    "mla_qknorm_key_gram": ([ctypes.POINTER(Dims), _vp, _vp, _vp], _i32),
+    "mla_decode_qknorm": ([ctypes.POINTER(Dims), _i32, _i32, _vp, _i32, _vp, _i32, _vp, _vp, _i64,
+                           _vp, _i32, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
 }
 
 
@@ -117,42 +125,79 @@ def absorb_q(dims: Dims, q_nope, q_rope, q_pos, deltas: Sequence[int], w_uk, q_a
                                               _s(stream)))
 
 
-def workspace_size(dims: Dims, B: int, s_q: int, n_h: int) -> int:
-    return int(lib().mla_decode_workspace_size(ctypes.byref(dims), B, s_q, n_h))
+def workspace_size(dims: Dims, B: int, s_q: int, n_h: int, n_ver: int = 1) -> int:
+    return int(lib().mla_decode_workspace_size(ctypes.byref(dims), B, s_q, n_ver, n_h))
 
 
-def decode(dims: Dims, B: int, s_q: int, q_abs, n_ver: int, h0: int, n_h: int, cache,
+def decode(dims: Dims, B: int, s_q: int, q_abs, n_ver: int, head_ids, n_h: int, cache,
            block_table, segs, q_pos, o_lat, lse, workspace, gather_rows=None, n_gather=None,
            stream=None):
+    """mla_decode; ``head_ids`` is an int32 device tensor of n_h head ids, or
+    None for heads 0 .. n_h-1."""
     n_pages = cache.shape[0]
     max_pages = block_table.shape[1]
     max_segs = segs.shape[1]
     max_gather = gather_rows.shape[1] if gather_rows is not None else 0
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check("mla_decode", lib().mla_decode(
-        ctypes.byref(dims), B, s_q, _p(q_abs), n_ver, h0, n_h, _p(cache), n_pages,
+        ctypes.byref(dims), B, s_q, _p(q_abs), n_ver, _p(head_ids), n_h, _p(cache), n_pages,
         _p(block_table), max_pages, _p(segs), max_segs, _p(gather_rows), _p(n_gather),
         max_gather, _p(q_pos), _p(o_lat), _p(lse), _p(workspace), ws_bytes, _s(stream)))
 
 
-def decode_static_ws(dims: Dims, B: int, s_q: int, q_abs, n_ver: int, h0: int, n_h: int, cache,
+def decode_static_ws(dims: Dims, B: int, s_q: int, q_abs, n_ver: int, head_ids, n_h: int, cache,
                      block_table, segs, q_pos, o_lat, lse, gather_rows=None, n_gather=None,
                      stream=None):
     """mla_decode with the library's fixed scratch array instead of a workspace."""
     max_gather = gather_rows.shape[1] if gather_rows is not None else 0
     _check("mla_decode_static_ws", lib().mla_decode_static_ws(
-        ctypes.byref(dims), B, s_q, _p(q_abs), n_ver, h0, n_h, _p(cache), cache.shape[0],
+        ctypes.byref(dims), B, s_q, _p(q_abs), n_ver, _p(head_ids), n_h, _p(cache), cache.shape[0],
         _p(block_table), block_table.shape[1], _p(segs), segs.shape[1], _p(gather_rows),
         _p(n_gather), max_gather, _p(q_pos), _p(o_lat), _p(lse), _s(stream)))
 
 
-def merge_lse(n_q: int, H: int, h0: int, n_h: int, d: int, o_a, lse_a, o_b, lse_b, o, lse,
+def decode_static_ws_init():
+    """Loads the static scratch array on the current device."""
+    _check("mla_decode_static_ws_init", lib().mla_decode_static_ws_init())
+
+
+def merge_lse(n_q: int, H: int, head_ids, n_h: int, d: int, o_a, lse_a, o_b, lse_b, o, lse,
               stream=None):
-    _check("mla_merge_lse", lib().mla_merge_lse(n_q, H, h0, n_h, d, _p(o_a), _p(lse_a), _p(o_b),
-                                                _p(lse_b), _p(o), _p(lse), _s(stream)))
+    _check("mla_merge_lse", lib().mla_merge_lse(n_q, H, _p(head_ids), n_h, d, _p(o_a), _p(lse_a),
+                                                _p(o_b), _p(lse_b), _p(o), _p(lse), _s(stream)))
 
 
 def out_proj(dims: Dims, o_lat, w_uv, w_o, v, out, stream=None):
     n_q = o_lat.shape[0]
     _check("mla_out_proj", lib().mla_out_proj(ctypes.byref(dims), n_q, _p(o_lat), _p(w_uv),
                                               _p(w_o), _p(v), _p(out), _s(stream)))
+
+
+def append_rows(dims, c_new, k_rope_raw, cache_pos, seq, row, cache, block_table,
+                key_gram=None, qk_eps=0.0, key_inv_rms=None, stream=None):
+    """mla_append_rows: entries i -> cache row (seq[i], row[i]) = [c | R(cache_pos) k_raw]
+    (QK-normed caches: with key_gram, also key_inv_rms and a rescaled k_rope)."""
+    _check("mla_append_rows", lib().mla_append_rows(
+        ctypes.byref(dims), c_new.shape[0], _p(c_new), _p(k_rope_raw), _p(cache_pos), _p(seq),
+        _p(row), block_table.shape[0], _p(cache), cache.shape[0], _p(block_table),
+        block_table.shape[1], _p(key_gram), qk_eps, _p(key_inv_rms), _s(stream)))
+
+
+def qknorm_query(dims, q_nope, g_q, g_k, eps, q_out, stream=None):
+    _check("mla_qknorm_query", lib().mla_qknorm_query(
+        ctypes.byref(dims), q_nope.shape[0], _p(q_nope), _p(g_q), _p(g_k), eps, _p(q_out),
+        _s(stream)))
+
+
+def qknorm_key_gram(dims, w_uk, gram, stream=None):
+    _check("mla_qknorm_key_gram", lib().mla_qknorm_key_gram(ctypes.byref(dims), _p(w_uk),
+                                                            _p(gram), _s(stream)))
+
+
+def decode_qknorm(dims, B, s_q, q_abs, n_ver, head_ids, n_h, cache, key_inv_rms, block_table,
+                  segs, q_pos, o_lat, lse, workspace, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("mla_decode_qknorm", lib().mla_decode_qknorm(
+        ctypes.byref(dims), B, s_q, _p(q_abs), n_ver, _p(head_ids), n_h, _p(cache),
+        _p(key_inv_rms), cache.shape[0], _p(block_table), block_table.shape[1], _p(segs),
+        segs.shape[1], _p(q_pos), _p(o_lat), _p(lse), _p(workspace), ws_bytes, _s(stream)))

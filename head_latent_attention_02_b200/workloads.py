@@ -142,7 +142,7 @@ class DecodeInputs:
     n_rows: np.ndarray        # [B] logical rows per sequence (end of its last segment)
     gather_rows: Optional[np.ndarray] = None  # [B, max_gather] int32
     n_gather: Optional[np.ndarray] = None     # [B] int32
-    head_order: Optional[np.ndarray] = None   # physical->logical head map (RedKnot)
+    head_order: Optional[np.ndarray] = None   # head ids, Local heads first (RedKnot)
     nan_page: int = -1
 
     @property
@@ -171,11 +171,15 @@ def make_weights(wl: Workload, seed: int = 0):
 
 
 def make_inputs(wl: Workload, seed: int = 0, lengths: Optional[list] = None,
-                poison: bool = True, with_weights: bool = True) -> DecodeInputs:
+                poison: bool = True, with_weights: bool = True,
+                draw_cache: bool = True) -> DecodeInputs:
     """Draw every input of one decode step for ``wl``.
 
     ``lengths`` overrides the per-sequence lengths (used by parity tests to
     build ragged variants of a workload at sizes the oracle finishes fast).
+    ``draw_cache=False`` leaves the pool's values undrawn (an uninitialised
+    array of the right shape) for callers that fill the cache on the device
+    and compare nothing against the oracle (throughput runs).
     """
     L = list(lengths) if lengths is not None else _lengths(wl, seed)
     assert len(L) == wl.B
@@ -203,17 +207,20 @@ def make_inputs(wl: Workload, seed: int = 0, lengths: Optional[list] = None,
         off += pages_per_seq[b]
 
     # one contiguous draw for all used rows, in (sequence, row) order
-    n_used = sum(rows)
-    rng = _rng(seed, _K_CACHE)
-    lat = _normal(rng, (n_used, wl.row), 1.0, wl.dtype)
-    pool = np.full((n_pages, PAGE, wl.row), np.nan if poison else 0.0, np.float32)
-    off = 0
-    for b in range(wl.B):
-        for p in range(pages_per_seq[b]):
-            take = min(PAGE, rows[b] - p * PAGE)
-            pool[block_table[b, p], :take] = lat[off:off + take]
-            off += take
-    del lat
+    if draw_cache:
+        n_used = sum(rows)
+        rng = _rng(seed, _K_CACHE)
+        lat = _normal(rng, (n_used, wl.row), 1.0, wl.dtype)
+        pool = np.full((n_pages, PAGE, wl.row), np.nan if poison else 0.0, np.float32)
+        off = 0
+        for b in range(wl.B):
+            for p in range(pages_per_seq[b]):
+                take = min(PAGE, rows[b] - p * PAGE)
+                pool[block_table[b, p], :take] = lat[off:off + take]
+                off += take
+        del lat
+    else:
+        pool = np.empty((n_pages, PAGE, wl.row), np.float32)
 
     # segments: one per sequence, or prefix + document for the RedKnot layout
     if wl.doc:

@@ -123,7 +123,7 @@ mla_status_t mla_absorb_q(const mla_dims_t* dims, int32_t n_q, const void* q_nop
 
 /* ---------------------------------------------------------------------------
  * mla_decode -- absorbed attention of every query token over its sequence's
- * packed latent cache, for the head range [h0, h0 + n_h).
+ * packed latent cache, for a list of heads.
  * [T27] "Move the Key Projection Into the Query" and "Position Rotations
  * Complicate the Absorption": score(t) = scale * (q_abs_content . c_t +
  * q_abs_rope . k_rope_t), masked where key_pos(t) > q_pos, softmaxed.
@@ -135,7 +135,12 @@ mla_status_t mla_absorb_q(const mla_dims_t* dims, int32_t n_q, const void* q_nop
  *   B, s_q        sequences and query tokens per sequence; query row i =
  *                 b * s_q + j
  *   q_abs         [n_ver, B*s_q, H, d_c + d_r] from mla_absorb_q (dtype)
- *   h0, n_h       head range; 0 <= h0, n_h >= 1, h0 + n_h <= H
+ *   head_ids      [n_h] distinct head ids in [0, H) (int32, device), or NULL
+ *                 for heads 0 .. n_h-1.  [RK]: the Local and Global heads
+ *                 are sets of head ids, decoded by separate calls over the
+ *                 same q_abs and cache.  An id outside [0, H) records
+ *                 BAD_INDEX and that head's results are not written.
+ *   n_h           heads decoded, 1 <= n_h <= H
  *   cache         [n_pages, page_size, d_c + d_r]: row = [c_KV | k_rope],
  *                 k_rope already rotated at its cache position (dtype);
  *                 256-byte aligned
@@ -152,12 +157,13 @@ mla_status_t mla_absorb_q(const mla_dims_t* dims, int32_t n_q, const void* q_nop
  *                 that breaks either rule records BAD_INDEX and gets NaN
  *                 o_lat and lse.
  *   q_pos         [B*s_q] request positions (int32)
- *   o_lat         [B*s_q, H, d_c] out (float): heads outside [h0, h0+n_h)
- *                 are not written
+ *   o_lat         [B*s_q, H, d_c] out (float), indexed by head id: heads
+ *                 not listed are not written
  *   lse           [B*s_q, H] out (float): natural-log sum of exp of the
  *                 scaled visible scores; a query that sees no row gets
  *                 o_lat = 0 and lse = -inf
- *   workspace     scratch of ws_bytes >= mla_decode_workspace_size(...),
+ *   workspace     scratch of ws_bytes >= mla_decode_workspace_size(dims, B,
+ *                 s_q, n_ver, n_h),
  *                 256-byte aligned; contents need not be initialised
  * Rows past the end of a segment in its last page, and pages no table
  * references, may hold anything (NaN included) without affecting results.
@@ -166,17 +172,19 @@ mla_status_t mla_absorb_q(const mla_dims_t* dims, int32_t n_q, const void* q_nop
  * n_ver * B * s_q * H beyond 2^31 - 1: device indices are 32-bit),
  * WORKSPACE (ws_bytes too small). */
 mla_status_t mla_decode(const mla_dims_t* dims, int32_t B, int32_t s_q, const void* q_abs,
-                        int32_t n_ver, int32_t h0, int32_t n_h, const void* cache,
+                        int32_t n_ver, const int32_t* head_ids, int32_t n_h,
+                        const void* cache,
                         int64_t n_pages, const int32_t* block_table, int32_t max_pages,
                         const mla_seg_t* segs, int32_t max_segs, const int32_t* gather_rows,
                         const int32_t* n_gather, int32_t max_gather, const int32_t* q_pos,
                         float* o_lat, float* lse, void* workspace, size_t ws_bytes,
                         mla_stream_t stream);
 
-/* Bytes of workspace mla_decode needs for these sizes on the current device
- * (0 if the arguments are invalid or the device cannot be queried). */
+/* Bytes of workspace mla_decode needs for these sizes on the current device,
+ * with or without a head list (0 if the arguments are invalid or the device
+ * cannot be queried). */
 size_t mla_decode_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q,
-                                 int32_t n_h);
+                                 int32_t n_ver, int32_t n_h);
 
 /* ---------------------------------------------------------------------------
  * mla_decode_static_ws -- mla_decode without a caller workspace.  The papers
@@ -186,24 +194,35 @@ size_t mla_decode_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q,
  *
  * Arguments, layouts, results and errors are those of mla_decode minus
  * workspace/ws_bytes.  The scratch is a static device array of
- * MLA_DECODE_STATIC_WS_BYTES (40 MiB) inside the library, reserved when its
+ * MLA_DECODE_STATIC_WS_BYTES (48 MiB) inside the library, reserved when its
  * module loads; nothing is allocated per call.
  *   - Sizes whose mla_decode_workspace_size exceeds the array are rejected
  *     with MLA_ERR_WORKSPACE before anything is launched (on a 148-SM device
- *     the split partials take 38.9 MB, leaving room for about 380,000
- *     streams of B * s_q * ceil(n_h / 128)).  Invalid dims or sizes give
- *     MLA_ERR_INVALID_ARG.
- *   - The first call on each device looks up the array's address with that
- *     device current (a runtime query that may load the module); make that
- *     first call before any stream capture.
+ *     the split partials take 38.9 MB; the rest holds the plan of up to
+ *     B * s_q * ceil(n_h / 128) streams and the packed queries of a head
+ *     list, n_ver * B * s_q * n_h * 1152 bytes).  Invalid dims or sizes give
+ *     MLA_ERR_INVALID_ARG; a device that cannot be queried gives
+ *     MLA_ERR_CUDA.
+ *   - The array is reserved when the library's module for it loads, which
+ *     the runtime does lazily, at the first call of mla_decode_static_ws_init
+ *     or mla_decode_static_ws on a device.  A host that reserves the rest of
+ *     device memory (a KV page pool) must make one of those calls first, and
+ *     before any stream capture.  Every call looks the address up again, so
+ *     a device reset or a new context needs only that first call again.
  *   - Every call on a device shares the one array, which keeps the previous
  *     call's contents (nothing in it needs clearing).  Calls that overlap on
  *     the GPU -- other streams, other host threads -- race on it: serialise
  *     them on one stream. */
-#define MLA_DECODE_STATIC_WS_BYTES ((size_t)40 << 20)
+#define MLA_DECODE_STATIC_WS_BYTES ((size_t)48 << 20)
+
+/* Loads the static scratch array on the current device (reserving its 48 MiB)
+ * and checks that its address resolves; launches nothing.  MLA_OK, or
+ * MLA_ERR_CUDA when the module cannot be loaded (e.g. no room left). */
+mla_status_t mla_decode_static_ws_init(void);
 
 mla_status_t mla_decode_static_ws(const mla_dims_t* dims, int32_t B, int32_t s_q,
-                                  const void* q_abs, int32_t n_ver, int32_t h0, int32_t n_h,
+                                  const void* q_abs, int32_t n_ver, const int32_t* head_ids,
+                                  int32_t n_h,
                                   const void* cache, int64_t n_pages,
                                   const int32_t* block_table, int32_t max_pages,
                                   const mla_seg_t* segs, int32_t max_segs,
@@ -215,7 +234,9 @@ mla_status_t mla_decode_static_ws(const mla_dims_t* dims, int32_t B, int32_t s_q
  * mla_merge_lse -- merge two partial attentions over disjoint key sets.
  * [RK]: certified Local-head contributions kept offline (MLA-Off) and the
  * rows recomputed online (MLA-Online) are merged before the single shared
- * output projection.  For each query row q and head h in [h0, h0 + n_h):
+ * output projection.  For each query row q and listed head h = head_ids[k]
+ * (k < n_h; NULL lists heads 0 .. n_h-1; an id outside [0, H) records
+ * BAD_INDEX and is skipped):
  *   lse = log(exp(lse_a) + exp(lse_b))
  *   o   = exp(lse_a - lse) * o_a + exp(lse_b - lse) * o_b
  * with lse = -inf and o = 0 when both sides are empty.
@@ -223,8 +244,8 @@ mla_status_t mla_decode_static_ws(const mla_dims_t* dims, int32_t B, int32_t s_q
  *   lse_a, lse_b, lse [n_q, H]    (float)
  * o may equal o_a or o_b and lse may equal lse_a or lse_b (in place); no
  * other aliasing.  Errors: INVALID_ARG. */
-mla_status_t mla_merge_lse(int32_t n_q, int32_t H, int32_t h0, int32_t n_h, int32_t d,
-                           const float* o_a, const float* lse_a, const float* o_b,
+mla_status_t mla_merge_lse(int32_t n_q, int32_t H, const int32_t* head_ids, int32_t n_h,
+                           int32_t d, const float* o_a, const float* lse_a, const float* o_b,
                            const float* lse_b, float* o, float* lse, mla_stream_t stream);
 
 /* ---------------------------------------------------------------------------
@@ -243,6 +264,86 @@ mla_status_t mla_merge_lse(int32_t n_q, int32_t H, int32_t h0, int32_t n_h, int3
 mla_status_t mla_out_proj(const mla_dims_t* dims, int32_t n_q, const float* o_lat,
                           const void* w_uv, const void* w_o, float* v, float* out,
                           mla_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * mla_append_rows -- write new tokens into the paged latent cache (the cache
+ * writer upstream of mla_decode).
+ * [T27] "Position Rotations Complicate the Absorption": the decoupled rotary
+ * key is cached beside the latent, already rotated.  [RK]: a document is
+ * cached at canonical positions 0, 1, ... and relocated on the query side.
+ * Entry i becomes the cache row of logical row row[i] of sequence seq[i]
+ * (page block_table[seq[i]][row[i] / page_size], slot row[i] % page_size):
+ *     [ c_new[i] | R(cache_pos[i]) k_rope_raw[i] ]
+ * with the rotation of mla_absorb_q (adjacent pairs, angle cache_pos *
+ * rope_base^(-2j/d_r) in double, result rounded to dtype).  cache_pos is the
+ * row's request position minus the relocation offset it will be served with
+ * (a prefix row: its request position; a document cached on its own: 0, 1, ...).
+ *
+ *   n_new         entries (0 is a no-op)
+ *   c_new         [n_new, d_c] latents (dtype)
+ *   k_rope_raw    [n_new, d_r] rotary keys before rotation (dtype)
+ *   cache_pos     [n_new] int32 rotation positions
+ *   seq, row      [n_new] int32 sequence index (< B) and logical row
+ *   cache         [n_pages, page_size, d_c + d_r] (dtype), written in place
+ *   block_table   [B, max_pages] int32 page ids
+ *   key_gram      NULL for plain rows; for a QK-normed cache ("QK-Normed
+ *                 MLA" abstract) the Gram matrix [d_c, d_c] (float) from
+ *                 mla_qknorm_key_gram.  Then each written row also gets
+ *                 key_inv_rms[page * page_size + slot] = 1 / sqrt(c^T G c +
+ *                 qk_eps), the inverse RMS of its H * d_n content keys, and
+ *                 its rotary key is stored multiplied by sqrt(c^T G c +
+ *                 qk_eps), the form mla_decode_qknorm reads.
+ *   qk_eps        RMSNorm epsilon (>= 0; read with key_gram only)
+ *   key_inv_rms   [n_pages * page_size] float, written in place; NULL
+ *                 exactly when key_gram is NULL
+ * Only the addressed rows change.  Two entries naming one row race.
+ * Errors: INVALID_ARG (null pointers, sizes, misaligned element pointers),
+ * UNSUPPORTED (page_size != 64).  An entry whose sequence, row or page id is
+ * out of range is skipped and records BAD_INDEX in the status word. */
+mla_status_t mla_append_rows(const mla_dims_t* dims, int32_t n_new, const void* c_new,
+                             const void* k_rope_raw, const int32_t* cache_pos,
+                             const int32_t* seq, const int32_t* row, int32_t B, void* cache,
+                             int64_t n_pages, const int32_t* block_table, int32_t max_pages,
+                             const float* key_gram, float qk_eps, float* key_inv_rms,
+                             mla_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * QK-normed MLA ("QK-Normed MLA" abstract): RMSNorm of the content query and
+ * of each token's content keys after the key up-projection, with all heads
+ * one group (statistics over H * d_n values).  In the absorbed form the
+ * query carries both norm weights and is absorbed as usual; the key side is
+ * one inverse RMS per cached token, applied per score column:
+ *   score(t) = scale * (q_abs_content . c_t * inv_t + q_abs_rope . k_rope_t)
+ * with the cached rotary key of a QK-normed cache stored times 1 / inv_t
+ * (mla_append_rows with key_gram), so the score is scale * inv_t times the
+ * plain 576-wide product.
+ *
+ * mla_qknorm_query -- q_out[r] = q_nope[r] / sqrt(mean(q_nope[r]^2) + eps)
+ *   * g_q * g_k over the H * d_n values of query row r (rounded to dtype);
+ *   pass q_out to mla_absorb_q as q_nope.
+ *   q_nope, q_out [n_rows, H, d_n] (dtype); g_q, g_k [H * d_n] (float).
+ * mla_qknorm_key_gram -- gram = W_UK^T W_UK / (H * d_n), [d_c, d_c] float,
+ *   with W_UK [H, d_n, d_c] (dtype) seen as [H * d_n, d_c]: then
+ *   mean_j (W_UK c)_j^2 = c^T gram c.  Depends on the weights only.
+ * mla_decode_qknorm -- mla_decode with the per-column factor inv_t read from
+ *   key_inv_rms [n_pages * page_size] (float, 16-byte aligned; a row's
+ *   entry at page * page_size + slot, as the writer stores it).  Page mode
+ *   only: no gathered rows.  Other arguments, layouts and errors are those
+ *   of mla_decode; INVALID_ARG when key_inv_rms is NULL. */
+mla_status_t mla_qknorm_query(const mla_dims_t* dims, int32_t n_rows, const void* q_nope,
+                              const float* g_q, const float* g_k, float eps, void* q_out,
+                              mla_stream_t stream);
+
+mla_status_t mla_qknorm_key_gram(const mla_dims_t* dims, const void* w_uk, float* gram,
+                                 mla_stream_t stream);
+
+mla_status_t mla_decode_qknorm(const mla_dims_t* dims, int32_t B, int32_t s_q,
+                               const void* q_abs, int32_t n_ver, const int32_t* head_ids,
+                               int32_t n_h, const void* cache, const float* key_inv_rms,
+                               int64_t n_pages, const int32_t* block_table, int32_t max_pages,
+                               const mla_seg_t* segs, int32_t max_segs, const int32_t* q_pos,
+                               float* o_lat, float* lse, void* workspace, size_t ws_bytes,
+                               mla_stream_t stream);
 
 #ifdef __cplusplus
 }  /* extern "C" */

@@ -41,17 +41,17 @@ NULL = None
 FAKE = 0x1000   # never dereferenced: every case below fails validation first
 
 
-def _decode(d, B=1, s_q=1, n_ver=1, h0=0, n_h=None, n_pages=4, max_pages=4, max_segs=1,
-            gather=NULL, n_gather=NULL, max_gather=0, ws_bytes=0):
+def _decode(d, B=1, s_q=1, n_ver=1, head_ids=NULL, n_h=None, n_pages=4, max_pages=4,
+            max_segs=1, gather=NULL, n_gather=NULL, max_gather=0, ws_bytes=0):
     n_h = (d.H if d is not None else 8) if n_h is None else n_h
     return mla.lib().mla_decode(ctypes.byref(d) if d is not None else None, B, s_q, FAKE, n_ver,
-                                h0, n_h, FAKE, n_pages, FAKE, max_pages, FAKE, max_segs, gather,
+                                head_ids, n_h, FAKE, n_pages, FAKE, max_pages, FAKE, max_segs, gather,
                                 n_gather, max_gather, FAKE, FAKE, FAKE, FAKE, ws_bytes, None)
 
 
 @pytest.mark.parametrize("case", [
-    dict(d=None), dict(B=-1), dict(s_q=0), dict(n_ver=0), dict(h0=-1), dict(n_h=0),
-    dict(h0=100, n_h=29), dict(n_pages=0), dict(max_pages=0), dict(max_segs=0),
+    dict(d=None), dict(B=-1), dict(s_q=0), dict(n_ver=0), dict(n_h=0), dict(n_h=129),
+    dict(head_ids=FAKE, n_h=129), dict(n_pages=0), dict(max_pages=0), dict(max_segs=0),
     dict(gather=FAKE, n_gather=NULL, max_gather=4), dict(gather=FAKE, n_gather=FAKE, max_gather=0),
 ])
 def test_decode_rejects_bad_arguments(L, case):
@@ -77,7 +77,7 @@ def test_decode_rejects_sizes_past_32_bit_indices(L):
 
 def test_decode_rejects_misaligned_cache(L):
     d = _dims()
-    rc = mla.lib().mla_decode(ctypes.byref(d), 1, 1, FAKE, 1, 0, 128, FAKE + 16, 4, FAKE, 4,
+    rc = mla.lib().mla_decode(ctypes.byref(d), 1, 1, FAKE, 1, None, 128, FAKE + 16, 4, FAKE, 4,
                               FAKE, 1, None, None, 0, FAKE, FAKE, FAKE, FAKE, 0, None)
     assert rc == 1
 
@@ -92,10 +92,11 @@ def test_absorb_merge_outproj_reject_bad_arguments(L):
     assert f.mla_absorb_q(ctypes.byref(d), -1, FAKE, FAKE, FAKE, arr, 1, FAKE, FAKE, None) == 1
     assert f.mla_absorb_q(ctypes.byref(d), 4, None, FAKE, FAKE, arr, 1, FAKE, FAKE, None) == 1
     assert f.mla_absorb_q(ctypes.byref(d), 0, None, None, None, arr, 1, None, None, None) == 0
-    assert f.mla_merge_lse(2, 64, 60, 8, 512, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
-    assert f.mla_merge_lse(2, 64, 0, 8, 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
-    assert f.mla_merge_lse(2, 64, 0, 8, 512, None, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
-    assert f.mla_merge_lse(0, 64, 0, 8, 512, None, None, None, None, None, None, None) == 0
+    assert f.mla_merge_lse(2, 64, None, 65, 512, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert f.mla_merge_lse(2, 64, FAKE, 0, 512, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert f.mla_merge_lse(2, 64, None, 8, 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert f.mla_merge_lse(2, 64, None, 8, 512, None, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert f.mla_merge_lse(0, 64, None, 8, 512, None, None, None, None, None, None, None) == 0
     assert f.mla_out_proj(ctypes.byref(d), 2, None, FAKE, FAKE, FAKE, FAKE, None) == 1
     assert f.mla_out_proj(ctypes.byref(d), 2, FAKE, FAKE, FAKE, FAKE, None, None) == 1
     assert f.mla_out_proj(ctypes.byref(d), -1, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
@@ -103,7 +104,50 @@ def test_absorb_merge_outproj_reject_bad_arguments(L):
 
 def test_workspace_size_rejects_bad_arguments(L):
     d = _dims()
-    assert mla.lib().mla_decode_workspace_size(None, 1, 1, 128) == 0
-    assert mla.lib().mla_decode_workspace_size(ctypes.byref(d), 1, 0, 128) == 0
+    assert mla.lib().mla_decode_workspace_size(None, 1, 1, 1, 128) == 0
+    assert mla.lib().mla_decode_workspace_size(ctypes.byref(d), 1, 0, 1, 128) == 0
+    assert mla.lib().mla_decode_workspace_size(ctypes.byref(d), 1, 1, 0, 128) == 0
+    assert mla.lib().mla_decode_workspace_size(ctypes.byref(d), 1, 1, 9, 128) == 0
+    assert mla.lib().mla_decode_workspace_size(ctypes.byref(d), 1, 1, 1, 129) == 0
     # the generic (non-576-wide) kernel needs only a token workspace
-    assert mla.lib().mla_decode_workspace_size(ctypes.byref(_dims(dtype=mla.MLA_F32)), 1, 1, 8) == 256
+    assert mla.lib().mla_decode_workspace_size(ctypes.byref(_dims(dtype=mla.MLA_F32)), 1, 1, 1,
+                                               8) == 256
+
+
+def test_append_rows_rejects_bad_arguments(L):
+    f = mla.lib()
+    d = _dims()
+    args = lambda **kw: [kw.get(k, v) for k, v in dict(
+        dims=ctypes.byref(d), n=4, c=FAKE, k=FAKE, pos=FAKE, seq=FAKE, row=FAKE, B=2, cache=FAKE,
+        n_pages=4, bt=FAKE, max_pages=2, gram=None, eps=0.0, inv=None, stream=None).items()]
+    assert f.mla_append_rows(*args(dims=None)) == 1
+    assert f.mla_append_rows(*args(n=-1)) == 1
+    assert f.mla_append_rows(*args(B=0)) == 1
+    assert f.mla_append_rows(*args(n_pages=0)) == 1
+    assert f.mla_append_rows(*args(max_pages=0)) == 1
+    assert f.mla_append_rows(*args(c=None)) == 1
+    assert f.mla_append_rows(*args(cache=FAKE + 1)) == 1            # misaligned bf16 pointer
+    assert f.mla_append_rows(*args(dims=ctypes.byref(_dims(d_r=63)))) == 1
+    assert f.mla_append_rows(*args(dims=ctypes.byref(_dims(page_size=32)))) == 2
+    assert f.mla_append_rows(*args(gram=FAKE)) == 1                # key_inv_rms missing
+    assert f.mla_append_rows(*args(inv=FAKE)) == 1                 # key_gram missing
+    assert f.mla_append_rows(*args(gram=FAKE, inv=FAKE, eps=-1.0)) == 1
+    assert f.mla_append_rows(*args(n=0, c=None, k=None, pos=None, seq=None, row=None,
+                                   cache=None, bt=None)) == 0
+
+
+def test_qknorm_calls_reject_bad_arguments(L):
+    f = mla.lib()
+    d = _dims()
+    assert f.mla_qknorm_query(None, 2, FAKE, FAKE, FAKE, 1e-6, FAKE, None) == 1
+    assert f.mla_qknorm_query(ctypes.byref(d), -1, FAKE, FAKE, FAKE, 1e-6, FAKE, None) == 1
+    assert f.mla_qknorm_query(ctypes.byref(d), 2, FAKE, None, FAKE, 1e-6, FAKE, None) == 1
+    assert f.mla_qknorm_query(ctypes.byref(d), 2, FAKE, FAKE, FAKE, -1.0, FAKE, None) == 1
+    assert f.mla_qknorm_query(ctypes.byref(d), 0, None, None, None, 1e-6, None, None) == 0
+    assert f.mla_qknorm_key_gram(ctypes.byref(d), None, FAKE, None) == 1
+    assert f.mla_qknorm_key_gram(None, FAKE, FAKE, None) == 1
+    qk = lambda **kw: f.mla_decode_qknorm(
+        ctypes.byref(d), 1, 1, FAKE, 1, None, 128, FAKE, kw.get("inv", FAKE), 4, FAKE, 4, FAKE,
+        1, FAKE, FAKE, FAKE, FAKE, 0, None)
+    assert qk(inv=None) == 1
+    assert qk(inv=FAKE + 4) == 1                                   # not 16-byte aligned

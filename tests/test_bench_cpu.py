@@ -56,3 +56,19 @@ def test_decode_flops_and_roofline_bound():
         else:
             assert r["unit"] == "TFLOP/s" and r["achieved"] == round(flops / 0.05e-3 / 1e12, 1)
         assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-4
+
+
+def test_cache_copies_keep_each_decode_out_of_l2():
+    sys.path.insert(0, ROOT)
+    import bench
+    for cache_bytes in (28_311_552, 75_497_472, 604_045_312, 1_340_657_664):
+        n = bench.n_cache_copies(cache_bytes)
+        assert n >= 3 and (n - 1) * cache_bytes >= 2 * bench.L2_BYTES
+
+
+def test_gpu_count_must_match_the_launched_ranks():
+    # a rank count that disagrees with --gpus is refused before any GPU work
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                          "--steps", "1"], env=env, capture_output=True, text=True, timeout=300)
+    assert res.returncode != 0 and "WORLD_SIZE=1" in res.stderr

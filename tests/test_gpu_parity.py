@@ -175,9 +175,10 @@ def test_redknot_offline_online_merge(mode, perm):
     o_off, l_off = O.decode_absorbed_fast(inp_off, heads=local, rows_override={0: k_off})
     o_off_dev = np.zeros((inp.n_q, wl.H, wl.d_c), np.float32)
     l_off_dev = np.full((inp.n_q, wl.H), -np.inf, np.float32)
-    o_off_dev[:, :wl.n_local] = o_off
-    l_off_dev[:, :wl.n_local] = l_off
-    p = _gpu(inp, head_order=order, o_off=o_off_dev, lse_off=l_off_dev)
+    o_off_dev[:, local] = o_off
+    l_off_dev[:, local] = l_off
+    # the weights stay in the workload's head order: the calls take id lists
+    p = _gpu(inp, o_off=o_off_dev, lse_off=l_off_dev)
     # reference: Local heads attend the whole document (offline + protected),
     # Global heads attend prefix + document; then one shared projection
     inp_all = make_inputs(wl, seed=5)
@@ -191,9 +192,99 @@ def test_redknot_offline_online_merge(mode, perm):
     o_ref[:, glob], l_ref[:, glob] = og, lg
     _, out_ref = O.out_proj(o_ref, inp.w_uv, inp.w_o)
     tol = TOL["bf16"]
-    _cmp(p.o_lat.cpu().numpy(), o_ref[:, order], tol, "o_lat")
-    _cmp(p.lse.cpu().numpy(), l_ref[:, order], tol, "lse", lse=True)
+    _cmp(p.o_lat.cpu().numpy(), o_ref, tol, "o_lat")
+    _cmp(p.lse.cpu().numpy(), l_ref, tol, "lse", lse=True)
     _cmp(p.out.cpu().numpy(), out_ref, tol, "out")
+
+
+def _decode_heads(inp, heads):
+    """mla_decode over a list of head ids into NaN-filled outputs."""
+    p = runner.upload(inp, with_out_proj=False)
+    mla.absorb_q(p.dims, p.q_nope, p.q_rope, p.q_pos, p.deltas, p.w_uk, p.q_abs)
+    p.o_lat.fill_(float("nan"))
+    p.lse.fill_(float("nan"))
+    ids = torch.tensor(np.asarray(heads, np.int32), device="cuda")
+    mla.decode(p.dims, p.B, p.s_q, p.q_abs, p.n_ver, ids, len(heads), p.cache, p.block_table,
+               p.segs, p.q_pos, p.o_lat, p.lse, p.workspace)
+    torch.cuda.synchronize()
+    return p
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_head_list_writes_listed_heads_only(dtype):
+    # 40 scattered heads of 128 (bf16, tensor-core path; packed queries) or 5
+    # of 8 (fp32 generic path): each result lands in its head's row and every
+    # other row is left as it was
+    if dtype == "bf16":
+        inp = make_inputs(_bf16(B=3, lengths=[300, 1000, 77]), seed=12)
+        heads = np.random.default_rng(12).permutation(128)[:40]
+    else:
+        inp = make_inputs(WORKLOADS["tiny_f32"], seed=12)
+        heads = np.array([6, 0, 3, 7, 2])
+    p = _decode_heads(inp, heads)
+    assert mla.get_status() == 0
+    o, l = p.o_lat.cpu().numpy(), p.lse.cpu().numpy()
+    o_ref, l_ref = O.decode_absorbed_fast(inp, heads=heads)
+    _cmp(o[:, heads], o_ref, TOL[dtype], "o_lat")
+    _cmp(l[:, heads], l_ref, TOL[dtype], "lse", lse=True)
+    rest = np.setdiff1d(np.arange(inp.wl.H), heads)
+    assert np.isnan(o[:, rest]).all() and np.isnan(l[:, rest]).all()
+
+
+def test_head_list_with_an_id_out_of_range_is_reported():
+    inp = make_inputs(_bf16(B=2, lengths=[200, 500]), seed=13)
+    p = _decode_heads(inp, [5, 700, 9, -1])
+    assert mla.get_status() == 6                       # MLA_ERR_BAD_INDEX
+    o, l = p.o_lat.cpu().numpy(), p.lse.cpu().numpy()
+    o_ref, l_ref = O.decode_absorbed_fast(inp, heads=[5, 9])
+    _cmp(o[:, [5, 9]], o_ref, TOL["bf16"], "o_lat")
+    _cmp(l[:, [5, 9]], l_ref, TOL["bf16"], "lse", lse=True)
+    rest = np.setdiff1d(np.arange(128), [5, 9])
+    assert np.isnan(o[:, rest]).all()
+    assert mla.get_status() == 0
+
+
+def test_redknot_offline_partial_made_on_the_gpu():
+    # the MLA-Off partial of the Local heads (document rows not protected) is
+    # computed by the decode call itself, then merged with the online part
+    wl = Workload("rk", "bf16", B=1, H=64, d_model=512, prefix=128, doc=512, n_local=56,
+                  protected=100, head_perm=True)
+    inp = make_inputs(wl, seed=15)
+    local = inp.head_order[:wl.n_local]
+    doc = np.arange(wl.prefix, wl.prefix + wl.doc)
+    k_off = np.setdiff1d(doc, inp.gather_rows[0])
+    p = runner.upload(inp, o_off=np.zeros((inp.n_q, wl.H, wl.d_c), np.float32),
+                      lse_off=np.full((inp.n_q, wl.H), -np.inf, np.float32))
+    mla.absorb_q(p.dims, p.q_nope, p.q_rope, p.q_pos, p.deltas, p.w_uk, p.q_abs)
+    runner.offline_partial(p, k_off[None, :])
+    runner.run_decode(p)
+    mla.out_proj(p.dims, p.o_lat, p.w_uv, p.w_o, p.v, p.out)
+    torch.cuda.synchronize()
+    assert mla.get_status() == 0
+    inp_all = make_inputs(wl, seed=15)
+    inp_all.gather_rows = None
+    o_off, l_off = O.decode_absorbed_fast(inp_all, heads=local, rows_override={0: k_off})
+    _cmp(p.o_off.cpu().numpy()[:, local], o_off, TOL["bf16"], "o_off")
+    _cmp(p.lse_off.cpu().numpy()[:, local], l_off, TOL["bf16"], "lse_off", lse=True)
+    o_ref = np.zeros((inp.n_q, wl.H, wl.d_c))
+    l_ref = np.zeros((inp.n_q, wl.H))
+    o_ref[:, local], l_ref[:, local] = O.decode_absorbed_fast(inp_all, heads=local,
+                                                              rows_override={0: doc})
+    glob = inp.head_order[wl.n_local:]
+    o_ref[:, glob], l_ref[:, glob] = O.decode_absorbed_fast(inp_all, heads=glob)
+    _, out_ref = O.out_proj(o_ref, inp.w_uv, inp.w_o)
+    _cmp(p.o_lat.cpu().numpy(), o_ref, TOL["bf16"], "o_lat")
+    _cmp(p.lse.cpu().numpy(), l_ref, TOL["bf16"], "lse", lse=True)
+    _cmp(p.out.cpu().numpy(), out_ref, TOL["bf16"], "out")
+
+
+@pytest.mark.parametrize("s_q", [48, 130])
+def test_prefill_chunk_causal(s_q):
+    # a prefill chunk: the last s_q cached rows are the query tokens, each
+    # sees the rows up to its own position (one stream per query token)
+    inp = make_inputs(_bf16(B=2, s_q=s_q, lengths=[300, 1000], H=64), seed=16)
+    p = _gpu(inp)
+    _check_all(inp, p, TOL["bf16"])
 
 
 # ----------------------------------------------------------------- edge cases
