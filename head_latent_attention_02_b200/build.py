@@ -11,7 +11,7 @@ SOURCES = ["csrc/mla_lib.cu", "csrc/mla_static_ws.cu", "csrc/mla_append.cu",
            "csrc/mla_qknorm.cu"]
 DEPENDS = ["csrc/mla_lib.cu", "csrc/mla_static_ws.cu", "csrc/mla_append.cu", "csrc/mla_qknorm.cu",
            "csrc/common.cuh",
-           "csrc/ptx.cuh", "csrc/kernels_simt.cuh", "csrc/wgemm.cuh", "csrc/decode_tc.cuh", "../include/mla.h"]
+           "csrc/ptx.cuh", "csrc/kernels_simt.cuh", "csrc/kernels_lowbit.cuh", "csrc/wgemm.cuh", "csrc/decode_tc.cuh", "../include/mla.h"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -24,7 +24,7 @@
 //     a release arrival on its barrier.
 //   - the value CTA (rank 1) holds O = P . c for the 128 heads in all 512
 //     tensor-memory columns.  It streams the same tile's latent columns again
-//     (an L2 hit: the score CTA fetched them moments before) one page at a
+//     (an L2 hit: the score CTA fetched them moments before) half a page at a
 //     time and issues M=128 x N=256 MMAs with P as the A operand.  Its four
 //     epilogue warps apply the occasional rescale of O and write the result.
 // Work is split over clusters as contiguous runs of (sequence, query token,
@@ -37,7 +37,8 @@
 // stage is three such panels.  When the two pages sit next to each other in
 // the pool the stage is one 3-D box; otherwise each page-panel is its own box,
 // which the TMA unit serves at about half the rate (a fixed cost per box).
-// A value slot is one page's 8 latent panels (one 3-D box).  Rows without
+// A value slot is half a page's 8 latent panels (one 3-D box); the four
+// slots hold a tile, refilled 32 KB at a time as each slot's MMAs finish.  Rows without
 // data (past a sequence's end, behind a bad page id) come from boxes placed
 // past the end of the cache, which the hardware fills with zeros, so NaN in
 // unused rows never reaches a product.  Gathered rows (attended through a
@@ -62,13 +63,17 @@ constexpr int kSlot = kT * 128;          // score panel: 128 rows x 128 B = 16 K
 constexpr int kStagePanels = 3;          // score ring stage: three panels (one 3-D box when
 constexpr int kStage = kStagePanels * kSlot;   //   both pages of the tile are adjacent)
 constexpr int kNStages = 4;              // score-side ring stages (192 KB)
-constexpr int kVPage = 8 * kPg * 128;    // value slot: one page's 8 latent panels = 64 KB
-constexpr int kNV = 2;                   // value-side ring slots
+constexpr int kVRows = 32;               // value slot: 32 rows of a page, 8 latent panels
+constexpr int kVSlot = 8 * kVRows * 128; //   = 32 KB
+constexpr int kNV = 4;                   // value-side ring slots (128 KB)
+constexpr int kVPerTile = kT / kVRows;   // value slots per tile
 constexpr int kPBuf = 2 * kM * 128;      // P: 128 rows x 128 tokens bf16, two 64-token panels
 constexpr int kHdrFlag = 512;            // header after P: rescale factor per row (512 B),
 constexpr int kMsgStride = 33 * 1024;    //   then one flag word per softmax warp
 constexpr int kEndBytes = 1536;          // per stream end: row sums of both halves, row max
-constexpr int kStageWarp = 32 * 128;     // epilogue staging: 32 rows x 32 floats per warp
+constexpr int kEpiWarps = 8;             // value CTA: rescale / epilogue warps (2 per lane quarter)
+constexpr int kStageRow = 80;            // epilogue staging row: 16 floats + 16 B pad
+constexpr int kStageWarp = 32 * kStageRow;   // staging: 32 rows x 16 floats per warp
 // score CTA
 constexpr int kOffRing = 0;
 constexpr int kOffQr = kOffRing + kNStages * kStage;           // rotary query panel
@@ -76,10 +81,10 @@ constexpr int kOffMax = kOffQr + kSlot;                        // row-max exchan
 constexpr int kEndScore = kOffMax + 2 * 2 * kM * 4;
 // value CTA
 constexpr int kOffVal = 0;
-constexpr int kOffMsg = kOffVal + kNV * kVPage;                // two incoming P messages
+constexpr int kOffMsg = kOffVal + kNV * kVSlot;                // two incoming P messages
 constexpr int kOffEnd = kOffMsg + 2 * kMsgStride;
 constexpr int kOffStage = kOffEnd + 2 * kEndBytes;
-constexpr int kEndValue = kOffStage + 4 * kStageWarp;
+constexpr int kEndValue = kOffStage + kEpiWarps * kStageWarp;
 // unit descriptors, then barriers, at the same offsets in both CTAs (commits
 // multicast to both)
 constexpr int kOffDesc = kEndScore > kEndValue ? kEndScore : kEndValue;
@@ -88,8 +93,8 @@ constexpr int kBarBytes = 1024;
 constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;   // + alignment slack
 // warp 0 loads, warp 1 issues MMAs; score CTA: warps 2-9 run the softmax (two
 // per TMEM lane quarter, one 64-column half of the tile each); value CTA:
-// warps 2-5 rescale O and write it out, warps 6-9 have no role; warp 10 of
-// both computes the unit descriptors
+// warps 2-9 rescale O and write it out (two per lane quarter, one 256-column
+// half of O each); warp 10 of both computes the unit descriptors
 constexpr int kThreads = 352;
 constexpr int kProducerWarp = 10;
 constexpr int kSoftWarps = 8;
@@ -102,7 +107,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: lazy rescale margin
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kOffMsg % 1024 == 0 && kMsgStride % 1024 == 0 && kSlot % 1024 == 0 &&
-              kVPage % 1024 == 0 && kPBuf + kHdrFlag + 4 * kSoftWarps <= kMsgStride,
+              kVSlot % 1024 == 0 && kPBuf + kHdrFlag + 4 * kSoftWarps <= kMsgStride &&
+              kVRows % 16 == 0 && kPg % kVRows == 0,
               "swizzle alignment and message size");
 
 struct PlanHeader {
@@ -117,7 +123,7 @@ struct PlanHeader {
 //   kp   2-D (col, cache row), box {64, 64}: one panel of a page
 //   row  2-D (col, cache row), boxes of 32 >> i rows (i = 0..5) for partial
 //        pages and zero rows past the end of the cache
-//   vp   3-D (col, cache row, panel), box {64, 64, 8}: a page's latent panels
+//   vp   3-D (col, cache row, panel), box {64, 32, 8}: half a page's latent panels
 //   g4   2-D (col, cache row), box {64, 1}: four-row gathers
 struct Maps {
   CUtensorMap q3, qr, k3, kp;
@@ -384,6 +390,25 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= kBarBytes, "barrier block too large");
 
+// A phase that never completes: one thread per warp waits on a barrier that
+// nothing arrives on, with the given limit, through the decode's own bounded
+// wait, then records the timeout the way the decode's roles do.  Nothing is
+// in flight, so the block returns cleanly.  1 block of 32 threads.
+__global__ void __launch_bounds__(32) wait_probe_kernel(uint64_t limit_ns, int* waited) {
+  __shared__ uint64_t never;
+  if (threadIdx.x == 0) {
+    mbar_init(&never, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) {
+    const uint64_t t0 = globaltimer();
+    const bool ok = mbar_wait(&never, 0, limit_ns);
+    *waited = (int)((globaltimer() - t0) / 1000);   // microseconds
+    if (!ok) set_status(MLA_ERR_TIMEOUT);
+  }
+}
+
 __device__ __forceinline__ void fail(bool& ok) {
   if (ok) set_status(MLA_ERR_TIMEOUT);
   ok = false;
@@ -455,7 +480,7 @@ __device__ __forceinline__ uint64_t visibility(const DecodeArgs& a, const Desc& 
 // Rescale this warp's 32 lanes of O (all 512 columns) by f.
 __device__ __noinline__ void scale_o(uint32_t taddr, float f) {
 #pragma unroll 1
-  for (int c = 0; c < 512; c += 32) {
+  for (int c = 0; c < kDc / 2; c += 32) {
     float ov[32];
     tmem_ld32(taddr + c, ov);
     tmem_wait_ld();
@@ -563,16 +588,16 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar->s_full[i], 1);
       mbar_init(&bar->s_empty[i], kSoftWarps);
-      mbar_init(&bar->end_empty[i], 4);
+      mbar_init(&bar->end_empty[i], kEpiWarps);
       for (int q = 0; q < 4; ++q) mbar_init(&bar->row_sync[i][q], 2);
       mbar_init(&bar->pv[i], 1);
       mbar_init(&bar->p_full[i], kSoftWarps);
-      mbar_init(&bar->o_ok[i], 4);
+      mbar_init(&bar->o_ok[i], kEpiWarps);
       mbar_init(&bar->end_full[i], kSoftWarps);
       mbar_init(&bar->d_full[i], 1);
       // consumers of each descriptor batch: loader, MMA issuer, and the eight
       // softmax warps (score CTA) or four epilogue warps (value CTA)
-      mbar_init(&bar->d_empty[i], rank == 0 ? 2 + kSoftWarps : 2 + 4);
+      mbar_init(&bar->d_empty[i], rank == 0 ? 2 + kSoftWarps : 2 + kEpiWarps);
     }
     mbar_init(&bar->mma_drain, 1);
     fence_mbar_init();
@@ -594,7 +619,7 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
   const long long y_oob = a.n_pages * kPg;   // first row past the cache: reads as zeros
   const uint32_t peer = mapa(smem_u32(smem), rank ^ 1u);   // the other CTA's shared memory
   // roles with a per-unit loop (the other warps of the value CTA have none)
-  const bool consumer = warp < (rank == 0 ? 2 + kSoftWarps : 6);
+  const bool consumer = warp < (rank == 0 ? 2 + kSoftWarps : 2 + kEpiWarps);
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ descriptors
@@ -895,7 +920,7 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
     }
   } else {
     // ================================================================ value CTA
-    uint8_t* vbuf = smem + kOffVal;     // two page slots: 8 latent panels of 64 rows
+    uint8_t* vbuf = smem + kOffVal;     // kNV slots: 8 latent panels of kVRows rows
     uint8_t* msg = smem + kOffMsg;      // two P messages: P, then factors and the flags
     const float* endm = reinterpret_cast<const float*>(smem + kOffEnd);
     if (warp == 0) {
@@ -909,35 +934,38 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
         if (!desc_wait(bar, it, true)) { fail(ok); break; }
         const Desc d = ring_d[it % kDescRing];
         const int b = stream_pos(p, d.s).b;
-        for (int hp = 0; hp < 2 && ok; ++hp, ++nv) {
+        for (int hq = 0; hq < kVPerTile && ok; ++hq, ++nv) {
           const int slot = nv % kNV;
           if (!wait_warp(&bar->v_empty[slot], ((nv / kNV) & 1) ^ 1)) { fail(ok); break; }
-          uint8_t* dst = vbuf + slot * kVPage;
+          uint8_t* dst = vbuf + slot * kVSlot;
           uint64_t* fb = &bar->v_full[slot];
-          if (lane == 0) mbar_arrive_expect_tx(fb, kVPage);
+          if (lane == 0) mbar_arrive_expect_tx(fb, kVSlot);
           __syncwarp();
           if constexpr (kGather) {
-            // lane l: rows 4 (l & 15) .. + 3 of the page's 64 rows, latent
-            // panels (l >> 4) + 2 k, k = 0..3
+            // kVRows / 4 four-row groups x 8 latent panels, spread over the lanes
+            constexpr int kQuads = kVRows / 4, kPer = kQuads * 8 / 32;
             long long gph[4];
             int gkp[4];
-            const int r4 = 4 * (lane & 15);
-            locate_gathered<4, 1>(a, b, d.k * kT + kPg * hp + r4, d.k * kT + d.nv0, y_oob, gph, gkp);
+            const int r4 = 4 * (lane % kQuads);
+            locate_gathered<4, 1>(a, b, d.k * kT + kVRows * hq + r4, d.k * kT + d.nv0, y_oob, gph,
+                                  gkp);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int q = (lane >> 4) + 2 * k;
-              tma_gather4(dst + q * (kPg * 128) + r4 * 128, &mp.g4, fb, 64 * q, (int)gph[0],
+            for (int k = 0; k < kPer; ++k) {
+              const int q = lane / kQuads + (32 / kQuads) * k;
+              tma_gather4(dst + q * (kVRows * 128) + r4 * 128, &mp.g4, fb, 64 * q, (int)gph[0],
                           (int)gph[1], (int)gph[2], (int)gph[3]);
             }
           } else if (lane == 0) {
-            const int rows = hp ? d.nv1 : d.nv0;
-            const long long ph = hp ? d.phys1 : d.phys0;
-            if (rows == kPg) {
+            // rows [ro, ro + kVRows) of page hp of the tile
+            const int hp = hq * kVRows / kPg, ro = hq * kVRows % kPg;
+            const int rows = max(0, min(kVRows, (hp ? d.nv1 : d.nv0) - ro));
+            const long long ph = (hp ? d.phys1 : d.phys0) + ro;
+            if (rows == kVRows) {
               tma_load_3d(dst, &mp.vp, fb, 0, (int)ph, 0);
             } else {
               for (int q = 0; q < 8; ++q) {
-                load_rows(dst + q * (kPg * 128), mp, fb, 64 * q, ph, 0, rows);
-                load_rows(dst + q * (kPg * 128), mp, fb, 64 * q, y_oob, rows, kPg - rows);
+                load_rows(dst + q * (kVRows * 128), mp, fb, 64 * q, ph, 0, rows);
+                load_rows(dst + q * (kVRows * 128), mp, fb, 64 * q, y_oob, rows, kVRows - rows);
               }
             }
           }
@@ -967,19 +995,23 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
           fence_proxy_async();
           tc_fence_after();
           const uint32_t pa = p0 + pb * kMsgStride;
-          for (int hp = 0; hp < 2 && ok; ++hp, ++nv) {
+          for (int hq = 0; hq < kVPerTile && ok; ++hq, ++nv) {
             const int slot = nv % kNV;
             if (!mbar_wait(&bar->v_full[slot], (nv / kNV) & 1)) { fail(ok); break; }
             tc_fence_after();
-            const uint32_t vb = v0 + slot * kVPage;
+            const uint32_t vb = v0 + slot * kVSlot;
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              // P panel hp holds the page's 64 tokens; 16 of them per step
-              const uint64_t ad = smem_desc_sw128(pa + hp * (kM * 128) + ks * 32, 16, 1024);
+            for (int ks = 0; ks < kVRows / 16; ++ks) {
+              // tokens [t, t + 16) of the tile: P panel t / 64, 16-token step
+              // (t % 64) / 16 within it
+              const int t = hq * kVRows + 16 * ks;
+              const uint64_t ad =
+                  smem_desc_sw128(pa + (t / kPg) * (kM * 128) + ((t % kPg) / 16) * 32, 16, 1024);
 #pragma unroll
               for (int nb = 0; nb < 2; ++nb) {
-                const uint64_t bd = smem_desc_sw128(vb + nb * 4 * (kPg * 128) + ks * 2048, kPg * 128, 1024);
-                mma_bf16_ss(tmem + 256 * nb, ad, bd, idesc_pv, (first && hp == 0 && ks == 0) ? 0u : 1u);
+                const uint64_t bd =
+                    smem_desc_sw128(vb + nb * 4 * (kVRows * 128) + ks * 2048, kVRows * 128, 1024);
+                mma_bf16_ss(tmem + 256 * nb, ad, bd, idesc_pv, (first && t == 0) ? 0u : 1u);
               }
             }
             mma_commit(&bar->v_empty[slot]);
@@ -990,12 +1022,16 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
         mma_commit(&bar->mma_drain);
         if (!mbar_wait(&bar->mma_drain, 0)) fail(ok);
       }
-    } else if (warp < 6) {
+    } else if (warp < 2 + kEpiWarps) {
       // ------------------------------------------------------------ rescale and epilogue
+      // warps 2-5 take columns [0, 256) and warps 6-9 columns [256, 512) of
+      // O; a warp's lane quarter (its rows) is warp & 3
       const int quad = warp & 3;
+      const int ch = (warp - 2) >> 2;
       const int h = quad * 32 + lane;
-      const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-      float4* stage = reinterpret_cast<float4*>(smem + kOffStage + quad * kStageWarp);
+      const int col0 = ch * (kDc / 2);
+      const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16) + col0;
+      float4* stage = reinterpret_cast<float4*>(smem + kOffStage + (warp - 2) * kStageWarp);
       int n_str = 0;
       for (int it = 0; it < n_units && ok; ++it) {
         if (!desc_wait(bar, it, true)) { fail(ok); break; }
@@ -1043,44 +1079,50 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
           float* my_dst = !whole ? p.partial + ((size_t)slot * kM + h) * kDc
                         : my_head >= 0 ? a.o_lat + ((size_t)qi * a.H + my_head) * kDc
                                        : nullptr;
-          // the rows this lane stores: 4 k + lane / 8 for k = 0..7
-          float* dst_row[8];
+          // the rows this lane stores: 8 k + lane / 4 for k = 0..3
+          float* dst_row[4];
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
+          for (int k = 0; k < 4; ++k)
             dst_row[k] = reinterpret_cast<float*>(__shfl_sync(
-                0xffffffffu, reinterpret_cast<unsigned long long>(my_dst), 4 * k + (lane >> 3)));
-          // O rows leave through a per-warp staging tile: each lane writes its
-          // row's 32 columns, then each store instruction writes 4 rows x 128 B.
-          // The next 32 columns are read from tensor memory while this chunk's
-          // stores issue.
+                0xffffffffu, reinterpret_cast<unsigned long long>(my_dst), 8 * k + (lane >> 2)));
+          // O rows leave through a per-warp staging tile (rows padded to 80 B):
+          // each lane writes 16 columns of its row, then each store
+          // instruction writes 8 rows x 64 B.  The next 32 columns are read
+          // from tensor memory while this chunk's stores issue.
           float ov[32], on[32];
           tmem_ld32(trow, ov);
           tmem_wait_ld();
 #pragma unroll 1
-          for (int c = 0; c < kDc; c += 32) {
+          for (int c = 0; c < kDc / 2; c += 32) {
+            if (c + 32 < kDc / 2) tmem_ld32(trow + c + 32, on);
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              stage[lane * 8 + (j ^ (lane & 7))] =
-                  make_float4(ov[4 * j] * inv, ov[4 * j + 1] * inv, ov[4 * j + 2] * inv,
-                              ov[4 * j + 3] * inv);
-            if (c + 32 < kDc) tmem_ld32(trow + c + 32, on);
-            __syncwarp();
+            for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const int rr = 4 * k + (lane >> 3), j = lane & 7;
-              if (dst_row[k])
-                *reinterpret_cast<float4*>(dst_row[k] + c + 4 * j) = stage[rr * 8 + (j ^ (rr & 7))];
+              for (int j = 0; j < 4; ++j)
+                stage[lane * (kStageRow / 16) + j] =
+                    make_float4(ov[16 * hh + 4 * j] * inv, ov[16 * hh + 4 * j + 1] * inv,
+                                ov[16 * hh + 4 * j + 2] * inv, ov[16 * hh + 4 * j + 3] * inv);
+              __syncwarp();
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int rr = 8 * k + (lane >> 2), j = lane & 3;
+                if (dst_row[k])
+                  *reinterpret_cast<float4*>(dst_row[k] + col0 + c + 16 * hh + 4 * j) =
+                      stage[rr * (kStageRow / 16) + j];
+              }
+              __syncwarp();
             }
-            __syncwarp();
-            if (c + 32 < kDc) {
+            if (c + 32 < kDc / 2) {
               tmem_wait_ld();
 #pragma unroll
               for (int i = 0; i < 32; ++i) ov[i] = on[i];
             }
           }
           tc_fence_before();
-          if (!whole) p.partial_lse[(size_t)slot * kM + h] = lse;
-          else if (my_head >= 0) a.lse[(size_t)qi * a.H + my_head] = lse;
+          if (ch == 0) {
+            if (!whole) p.partial_lse[(size_t)slot * kM + h] = lse;
+            else if (my_head >= 0) a.lse[(size_t)qi * a.H + my_head] = lse;
+          }
           ++n_str;
         }
       }

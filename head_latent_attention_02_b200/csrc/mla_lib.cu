@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "ptx.cuh"
 #include "kernels_simt.cuh"
+#include "kernels_lowbit.cuh"
 #include "decode_tc.cuh"
 #include "wgemm.cuh"
 
@@ -458,7 +459,7 @@ mla_status_t decode_impl(const mla_dims_t* dims, int32_t B, int32_t s_q, const v
       !make_map_576(&maps.qr, q_src, q_rows, 2, tc::kM) ||
       !make_map_576(&maps.k3, cache, cache_rows, 3, tc::kT, tc::kStagePanels) ||
       !make_map_576(&maps.kp, cache, cache_rows, 2, tc::kPg) ||
-      !make_map_576(&maps.vp, cache, cache_rows, 3, tc::kPg, 8) ||
+      !make_map_576(&maps.vp, cache, cache_rows, 3, tc::kVRows, 8) ||
       !make_map_576(&maps.g4, cache, cache_rows, 2, 1))
     return MLA_ERR_CUDA;
   for (int i = 0; i < tc::kNumBoxHeights; ++i)
@@ -556,6 +557,127 @@ mla_status_t mla_decode_qknorm(const mla_dims_t* dims, int32_t B, int32_t s_q, c
   return decode_impl(dims, B, s_q, q_abs, n_ver, head_ids, n_h, cache, n_pages, block_table,
                      max_pages, segs, max_segs, nullptr, nullptr, 0, q_pos, o_lat, lse,
                      workspace, ws_bytes, stream, key_inv_rms);
+}
+
+}  // extern "C"
+
+namespace {
+
+bool lowbit_ok(const mla_dims_t* dims, int bits_c, int bits_r) {
+  return ((bits_c == 4 && bits_r == 4) || (bits_c == 2 && bits_r == 4)) &&
+         (dims->d_c * bits_c) % 32 == 0 && (dims->d_r * bits_r) % 32 == 0;
+}
+
+template <typename T>
+void launch_pack(int bits_c, int n, const mla_dims_t* d, const void* rows, const float* sc,
+                 const float* sr, void* out, cudaStream_t st) {
+  const unsigned blocks = (unsigned)((n + 7) / 8);
+  if (bits_c == 4)
+    pack_rows_kernel<T, 4, 4><<<blocks, 256, 0, st>>>(n, d->d_c, d->d_r,
+                                                      static_cast<const T*>(rows), sc, sr,
+                                                      static_cast<uint8_t*>(out));
+  else
+    pack_rows_kernel<T, 2, 4><<<blocks, 256, 0, st>>>(n, d->d_c, d->d_r,
+                                                      static_cast<const T*>(rows), sc, sr,
+                                                      static_cast<uint8_t*>(out));
+}
+
+template <typename T>
+void launch_lowbit(int bits_c, dim3 grid, size_t smem, const DecodeArgs& a, const float* sc,
+                   const float* sr, cudaStream_t st) {
+  if (bits_c == 4)
+    decode_lowbit_kernel<T, 4, 4><<<grid, 128, smem, st>>>(a, sc, sr);
+  else
+    decode_lowbit_kernel<T, 2, 4><<<grid, 128, smem, st>>>(a, sc, sr);
+}
+
+}  // namespace
+
+extern "C" {
+
+mla_status_t mla_pack_rows(const mla_dims_t* dims, int32_t bits_c, int32_t bits_r, int64_t n_rows,
+                           const void* rows, const float* scale_c, const float* scale_r,
+                           void* packed, mla_stream_t stream) {
+  if (!dims_ok(dims) || n_rows < 0) return MLA_ERR_INVALID_ARG;
+  if (!lowbit_ok(dims, bits_c, bits_r)) return MLA_ERR_UNSUPPORTED;
+  if (n_rows == 0) return MLA_OK;
+  if (!rows || !scale_c || !scale_r || !packed || !aligned(packed, 4)) return MLA_ERR_INVALID_ARG;
+  if (n_rows > (int64_t)INT32_MAX - 8) return MLA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dims->dtype == MLA_BF16)
+    launch_pack<__nv_bfloat16>(bits_c, (int)n_rows, dims, rows, scale_c, scale_r, packed, st);
+  else
+    launch_pack<float>(bits_c, (int)n_rows, dims, rows, scale_c, scale_r, packed, st);
+  return launch_ok();
+}
+
+mla_status_t mla_decode_lowbit(const mla_dims_t* dims, int32_t bits_c, int32_t bits_r, int32_t B,
+                               int32_t s_q, const void* q_abs, int32_t n_ver,
+                               const int32_t* head_ids, int32_t n_h, const void* cache,
+                               const float* scale_c, const float* scale_r, int64_t n_pages,
+                               const int32_t* block_table, int32_t max_pages,
+                               const mla_seg_t* segs, int32_t max_segs,
+                               const int32_t* gather_rows, const int32_t* n_gather,
+                               int32_t max_gather, const int32_t* q_pos, float* o_lat, float* lse,
+                               mla_stream_t stream) {
+  if (!dims_ok(dims) || B < 0 || s_q < 1 || n_ver < 1 || n_h < 1 || n_h > dims->H ||
+      n_pages < 1 || max_pages < 1 || max_segs < 1)
+    return MLA_ERR_INVALID_ARG;
+  if (!lowbit_ok(dims, bits_c, bits_r)) return MLA_ERR_UNSUPPORTED;
+  if (dims->page_size != kPage || n_ver > kMaxVersions) return MLA_ERR_UNSUPPORTED;
+  if (gather_rows && (!n_gather || max_gather < 1)) return MLA_ERR_INVALID_ARG;
+  if (B == 0) return MLA_OK;
+  if (!q_abs || !cache || !scale_c || !scale_r || !block_table || !segs || !q_pos || !o_lat ||
+      !lse || !aligned(cache, 4))
+    return MLA_ERR_INVALID_ARG;
+  if (n_pages * kPage + 2 * kPage > INT32_MAX || (long long)max_pages * kPage > INT32_MAX ||
+      (long long)n_ver * B * s_q * dims->H > INT32_MAX)
+    return MLA_ERR_UNSUPPORTED;
+  DecodeArgs a;
+  a.B = B;
+  a.s_q = s_q;
+  a.n_q = B * s_q;
+  a.H = dims->H;
+  a.qH = dims->H;
+  a.head_ids = head_ids;
+  a.key_inv = nullptr;
+  a.n_h = n_h;
+  a.d_c = dims->d_c;
+  a.d_r = dims->d_r;
+  a.n_ver = n_ver;
+  a.max_pages = max_pages;
+  a.max_segs = max_segs;
+  a.max_gather = gather_rows ? max_gather : 0;
+  a.n_pages = n_pages;
+  a.scale = dims->scale;
+  a.q_abs = q_abs;
+  a.cache = cache;
+  a.block_table = block_table;
+  a.segs = segs;
+  a.gather_rows = gather_rows;
+  a.n_gather = gather_rows ? n_gather : nullptr;
+  a.q_pos = q_pos;
+  a.o_lat = o_lat;
+  a.lse = lse;
+  const int row = dims->d_c + dims->d_r;
+  const size_t smem = sizeof(float) * ((size_t)n_ver * row + dims->d_c + 128 + 4) +
+                      sizeof(long long) * 128 + 64;
+  if (smem > 48 * 1024) return MLA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 grid(n_h, B * s_q);
+  if (dims->dtype == MLA_BF16)
+    launch_lowbit<__nv_bfloat16>(bits_c, grid, smem, a, scale_c, scale_r, st);
+  else
+    launch_lowbit<float>(bits_c, grid, smem, a, scale_c, scale_r, st);
+  return launch_ok();
+}
+
+mla_status_t mla_debug_wait_probe(int64_t limit_ns, int32_t* waited_us, mla_stream_t stream) {
+  if (limit_ns < 1000 || limit_ns > 100000000 || !waited_us || !aligned(waited_us, 4))
+    return MLA_ERR_INVALID_ARG;
+  tc::wait_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      (uint64_t)limit_ns, waited_us);
+  return launch_ok();
 }
 
 mla_status_t mla_merge_lse(int32_t n_q, int32_t H, const int32_t* head_ids, int32_t n_h,

@@ -56,6 +56,11 @@ _SIGS = {
     "mla_qknorm_query": ([ctypes.POINTER(Dims), _i32, _vp, _vp, _vp, ctypes.c_float, _vp, _vp],
                          _i32),
     "mla_qknorm_key_gram": ([ctypes.POINTER(Dims), _vp, _vp, _vp], _i32),
+    "mla_debug_wait_probe": ([_i64, _vp, _vp], _i32),
+    "mla_pack_rows": ([ctypes.POINTER(Dims), _i32, _i32, _i64, _vp, _vp, _vp, _vp, _vp], _i32),
+    "mla_decode_lowbit": ([ctypes.POINTER(Dims), _i32, _i32, _i32, _i32, _vp, _i32, _vp, _i32,
+                           _vp, _vp, _vp, _i64, _vp, _i32, _vp, _i32, _vp, _vp, _i32, _vp, _vp,
+                           _vp, _vp], _i32),
     "mla_decode_qknorm": ([ctypes.POINTER(Dims), _i32, _i32, _vp, _i32, _vp, _i32, _vp, _vp, _i64,
                            _vp, _i32, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
 }
@@ -201,3 +206,22 @@ def decode_qknorm(dims, B, s_q, q_abs, n_ver, head_ids, n_h, cache, key_inv_rms,
         ctypes.byref(dims), B, s_q, _p(q_abs), n_ver, _p(head_ids), n_h, _p(cache),
         _p(key_inv_rms), cache.shape[0], _p(block_table), block_table.shape[1], _p(segs),
         segs.shape[1], _p(q_pos), _p(o_lat), _p(lse), _p(workspace), ws_bytes, _s(stream)))
+
+
+def pack_rows(dims, bits_c, bits_r, rows, scale_c, scale_r, packed, stream=None):
+    """mla_pack_rows: rows [n, d_c + d_r] -> packed codes [n, row bytes]."""
+    _check("mla_pack_rows", lib().mla_pack_rows(ctypes.byref(dims), bits_c, bits_r,
+                                                rows.shape[0], _p(rows), _p(scale_c),
+                                                _p(scale_r), _p(packed), _s(stream)))
+
+
+def decode_lowbit(dims, bits_c, bits_r, B, s_q, q_abs, n_ver, head_ids, n_h, cache, scale_c,
+                  scale_r, block_table, segs, q_pos, o_lat, lse, gather_rows=None, n_gather=None,
+                  stream=None):
+    """mla_decode_lowbit over a packed pool cache [n_pages, 64, row bytes] (uint8)."""
+    max_gather = gather_rows.shape[1] if gather_rows is not None else 0
+    _check("mla_decode_lowbit", lib().mla_decode_lowbit(
+        ctypes.byref(dims), bits_c, bits_r, B, s_q, _p(q_abs), n_ver, _p(head_ids), n_h,
+        _p(cache), _p(scale_c), _p(scale_r), cache.shape[0], _p(block_table),
+        block_table.shape[1], _p(segs), segs.shape[1], _p(gather_rows), _p(n_gather),
+        max_gather, _p(q_pos), _p(o_lat), _p(lse), _s(stream)))

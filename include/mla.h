@@ -307,6 +307,53 @@ mla_status_t mla_append_rows(const mla_dims_t* dims, int32_t n_new, const void* 
                              const float* key_gram, float qk_eps, float* key_inv_rms,
                              mla_stream_t stream);
 
+/* mla_debug_wait_probe -- checks the bounded-wait path without a fault: one
+ * thread waits, through the decode kernels' own bounded wait, on a barrier
+ * phase that never completes, gives up after limit_ns (1 us .. 100 ms), and
+ * records MLA_ERR_TIMEOUT in the status word as a decode role does; nothing
+ * is in flight, so the kernel returns and the context stays usable.
+ * waited_us (device, int32) receives the time it waited, in microseconds.
+ * Errors: INVALID_ARG for a limit out of range or a null / misaligned
+ * waited_us. */
+mla_status_t mla_debug_wait_probe(int64_t limit_ns, int32_t* waited_us, mla_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Low-bit latent cache (QuantMLA abstract: the content and rotary caches
+ * kept as INT4 / INT4 or INT2 / INT4 codes, unpacked and dequantised inside
+ * the attention).  A packed row is d_c content codes of bits_c bits, then
+ * d_r rotary codes of bits_r bits, little-end first: code k of a segment
+ * occupies bits [bits*k mod 8, ...) of byte bits*k/8 of the segment, as a
+ * two's complement field.  Row bytes: (d_c*bits_c + d_r*bits_r) / 8 (288 at
+ * INT4/INT4, 160 at INT2/INT4 for 512 + 64 channels).  One static scale per
+ * channel: a code stands for code * scale_c[k] (content channel k) or
+ * code * scale_r[k] (rotary channel k).  (bits_c, bits_r) is (4, 4) or
+ * (2, 4), and d_c * bits_c and d_r * bits_r must be multiples of 32.
+ *
+ * mla_pack_rows -- packed[i] = codes of rows[i] [n_rows, d_c + d_r] (dtype):
+ *   code = round-half-even(x / scale) in fp32, clamped to the signed range.
+ *   packed [n_rows, row bytes], 4-byte aligned.
+ * mla_decode_lowbit -- mla_decode over a pool of packed rows
+ *   cache [n_pages, page_size, row bytes] (4-byte aligned): the result is
+ *   attention over the dequantised rows.  The scales are folded into the
+ *   query and the output (scores of the scaled query against the codes; the
+ *   weighted sum of codes times scale_c), so no row is ever dequantised in
+ *   memory.  Head lists, segments, gathered rows, masking and outputs are
+ *   those of mla_decode; no workspace.  UNSUPPORTED for other bit pairs.
+ *   This kernel is a SIMT kernel: one CTA per (head, query row). */
+mla_status_t mla_pack_rows(const mla_dims_t* dims, int32_t bits_c, int32_t bits_r,
+                           int64_t n_rows, const void* rows, const float* scale_c,
+                           const float* scale_r, void* packed, mla_stream_t stream);
+
+mla_status_t mla_decode_lowbit(const mla_dims_t* dims, int32_t bits_c, int32_t bits_r,
+                               int32_t B, int32_t s_q, const void* q_abs, int32_t n_ver,
+                               const int32_t* head_ids, int32_t n_h, const void* cache,
+                               const float* scale_c, const float* scale_r, int64_t n_pages,
+                               const int32_t* block_table, int32_t max_pages,
+                               const mla_seg_t* segs, int32_t max_segs,
+                               const int32_t* gather_rows, const int32_t* n_gather,
+                               int32_t max_gather, const int32_t* q_pos, float* o_lat,
+                               float* lse, mla_stream_t stream);
+
 /* ---------------------------------------------------------------------------
  * QK-normed MLA ("QK-Normed MLA" abstract): RMSNorm of the content query and
  * of each token's content keys after the key up-projection, with all heads

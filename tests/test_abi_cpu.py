@@ -151,3 +151,27 @@ def test_qknorm_calls_reject_bad_arguments(L):
         1, FAKE, FAKE, FAKE, FAKE, 0, None)
     assert qk(inv=None) == 1
     assert qk(inv=FAKE + 4) == 1                                   # not 16-byte aligned
+
+
+def test_lowbit_calls_reject_bad_arguments(L):
+    f = mla.lib()
+    d = _dims()
+    assert f.mla_pack_rows(ctypes.byref(d), 3, 4, 4, FAKE, FAKE, FAKE, FAKE, None) == 2
+    assert f.mla_pack_rows(ctypes.byref(d), 4, 2, 4, FAKE, FAKE, FAKE, FAKE, None) == 2
+    assert f.mla_pack_rows(ctypes.byref(d), 4, 4, -1, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert f.mla_pack_rows(ctypes.byref(d), 4, 4, 4, FAKE, None, FAKE, FAKE, None) == 1
+    assert f.mla_pack_rows(ctypes.byref(d), 4, 4, 4, FAKE, FAKE, FAKE, FAKE + 2, None) == 1
+    assert f.mla_pack_rows(ctypes.byref(d), 2, 4, 0, None, None, None, None, None) == 0
+    lb = lambda bc=4, br=4, cache=FAKE, sc=FAKE, n_h=128: f.mla_decode_lowbit(
+        ctypes.byref(d), bc, br, 1, 1, FAKE, 1, None, n_h, cache, sc, FAKE, 4, FAKE, 4, FAKE, 1,
+        None, None, 0, FAKE, FAKE, FAKE, None)
+    assert lb(bc=8) == 2 and lb(bc=2, br=2) == 2
+    assert lb(cache=FAKE + 1) == 1 and lb(sc=None) == 1 and lb(n_h=129) == 1
+
+
+def test_wait_probe_rejects_bad_arguments(L):
+    f = mla.lib()
+    assert f.mla_debug_wait_probe(10, FAKE, None) == 1             # below 1 us
+    assert f.mla_debug_wait_probe(10 ** 9, FAKE, None) == 1        # above 100 ms
+    assert f.mla_debug_wait_probe(10 ** 6, None, None) == 1
+    assert f.mla_debug_wait_probe(10 ** 6, FAKE + 2, None) == 1

@@ -411,3 +411,20 @@ def test_full_redknot_56_8():
 
 def test_full_bf16_long_256k_sampled():
     _full("bf16_long_256k", seqs=[1])
+
+
+# ----------------------------------------------------------------- bounded waits
+
+def test_bounded_wait_gives_up_with_timeout_status():
+    # a barrier phase that never completes: the wait gives up after its limit,
+    # the status word says MLA_ERR_TIMEOUT, and the context keeps working
+    waited = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rc = mla.lib().mla_debug_wait_probe(2_000_000, waited.data_ptr(), None)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert mla.STATUS[mla.get_status()] == "MLA_ERR_TIMEOUT"
+    assert 2000 <= int(waited.item()) < 1_000_000
+    assert mla.get_status() == 0
+    inp = make_inputs(_bf16(B=1, lengths=[300]), seed=17)
+    p = _gpu(inp)
+    _check_all(inp, p, TOL["bf16"])
