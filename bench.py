@@ -316,15 +316,98 @@ class Problem:
             "decode calls of the step (plan + decode_tc + combine"
             + (", twice, + merge_lse)" if wl.n_local else ")"))
 
+    def _median_us(self, graphs, reps):
+        """Median µs of single replays (CUDA events around each), rotating
+        over ``graphs``."""
+        import torch
+        for i in range(3):
+            graphs[i % len(graphs)].replay()
+        ts = []
+        for i in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(self.stream)
+            graphs[i % len(graphs)].replay()
+            b.record(self.stream)
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        assert self.mla.get_status(self.stream) == 0
+        return statistics.median(x.elapsed_time(y) * 1e3 for x, y in ts)
+
+    def _capture(self, fn):
+        import torch
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        return g
+
+    def qknorm_overhead(self, reps=20):
+        """mla_decode_qknorm (one inverse-RMS factor per score column, read
+        per page) against mla_decode on the same rows, both as decode-only
+        graphs over the rotating cache copies."""
+        import torch
+        p, mla = self.p, self.mla
+        n_rows = p.cache.shape[0] * p.cache.shape[1]
+        g = torch.Generator(device=p.cache.device)
+        g.manual_seed(7)
+        key_inv = torch.rand(n_rows, generator=g, device=p.cache.device) + 0.5
+        qk = [self._capture(lambda c=c: mla.decode_qknorm(
+            p.dims, p.B, p.s_q, p.q_abs, p.n_ver, None, p.H, self.caches[c], key_inv,
+            p.block_table, p.segs, p.q_pos, p.o_lat, p.lse, p.workspace))
+            for c in range(self.n_copies)]
+        t_plain = self._median_us(self.g_dec, reps)
+        t_qk = self._median_us(qk, reps)
+        del qk
+        return {"decode_us": round(t_plain, 2), "qknorm_decode_us": round(t_qk, 2),
+                "overhead_pct": round(100.0 * (t_qk / t_plain - 1.0), 2), "repeats": reps,
+                "how": "decode-only graph replays, median of single replays"}
+
+    def lowbit(self, reps=10):
+        """mla_decode_lowbit over the rows packed as INT4/INT4 (288 B) and
+        INT2/INT4 (160 B): µs and GB/s of packed rows read."""
+        import torch
+        p, mla, wl = self.p, self.mla, self.wl
+        out = {}
+        g = torch.Generator(device=p.cache.device)
+        g.manual_seed(11)
+        for bits_c, bits_r in ((4, 4), (2, 4)):
+            row_bytes = (wl.d_c * bits_c + wl.d_r * bits_r) // 8
+            lo = 0.3 if bits_c == 4 else 0.8
+            sc = torch.rand(wl.d_c, generator=g, device=p.cache.device) * 0.3 + lo
+            sr = torch.rand(wl.d_r, generator=g, device=p.cache.device) * 0.3 + 0.3
+            n_rows = p.cache.shape[0] * p.cache.shape[1]
+            n_copies = n_cache_copies(n_rows * row_bytes)
+            packed = []
+            for c in range(n_copies):
+                src = self.caches[c % self.n_copies].view(n_rows, wl.d_c + wl.d_r)
+                dst = torch.empty((p.cache.shape[0], p.cache.shape[1], row_bytes),
+                                  dtype=torch.uint8, device=p.cache.device)
+                mla.pack_rows(p.dims, bits_c, bits_r, src, sc, sr, dst.view(n_rows, row_bytes))
+                packed.append(dst)
+            gr = [self._capture(lambda c=c: mla.decode_lowbit(
+                p.dims, bits_c, bits_r, p.B, p.s_q, p.q_abs, p.n_ver, None, p.H, packed[c], sc,
+                sr, p.block_table, p.segs, p.q_pos, p.o_lat, p.lse)) for c in range(n_copies)]
+            t = self._median_us(gr, reps)
+            nbytes = self.n_read * row_bytes
+            out[f"int{bits_c}_int{bits_r}"] = {
+                "row_bytes": row_bytes, "decode_us": round(t, 2), "packed_bytes": nbytes,
+                "GB_s": round(nbytes / (t * 1e-6) / 1e9, 1),
+                "frac_of_hbm": round(nbytes / (t * 1e-6) / 1e9 / _peaks()[0]["hbm_gbs"], 4),
+                "kernel": "decode_lowbit_kernel (SIMT, one CTA per head and query row)",
+                "repeats": reps}
+            del gr, packed
+        torch.cuda.empty_cache()
+        return out
+
     def release(self):
         import torch
         del self.g_abs, self.g_dec, self.g_out, self.caches, self.p
         torch.cuda.empty_cache()
 
 
-def measure_workload(name, rank, dev, stream, peaks, src, reps=20):
+def measure_workload(name, rank, dev, stream, peaks, src, reps=20, qknorm=False):
     """Decode µs (median of ``reps`` steps), cache GB/s and roofline of one
-    more workload on this GPU."""
+    more workload on this GPU (with ``qknorm``, also the QK-normed decode's
+    overhead on it)."""
     import torch
     prob = Problem(name, rank, dev, stream)
     prob.steps(3)
@@ -340,6 +423,8 @@ def measure_workload(name, rank, dev, stream, peaks, src, reps=20):
            "config": {"B": prob.wl.B, "H": prob.wl.H, "s_q": prob.wl.s_q,
                       "rows_total": int(sum(prob.inp.n_rows)),
                       "n_local_heads": prob.wl.n_local, "cache_copies": prob.n_copies}}
+    if qknorm:
+        out["qknorm"] = prob.qknorm_overhead()
     prob.release()
     return out
 
@@ -431,13 +516,18 @@ def run_gpu(args):
         assert mla.get_status(stream) == 0
         cache_bytes, wl, inp, kernels = prob.cache_bytes, prob.wl, prob.inp, prob.kernels
         n_copies = prob.n_copies
+        variants = {}
+        if world == 1 and not args.no_workloads and args.workload == WORKLOAD:
+            variants["qknorm"] = prob.qknorm_overhead()
+            variants["lowbit"] = prob.lowbit()
         prob.release()
 
         # --- the other configurations, decode only, on this GPU
         workloads = {}
         if world == 1 and not args.no_workloads and args.workload == WORKLOAD:
             for name in EXTRA_WORKLOADS:
-                workloads[name] = measure_workload(name, rank, dev, stream, peaks, src)
+                workloads[name] = measure_workload(name, rank, dev, stream, peaks, src,
+                                                   qknorm=(name == "bf16_long_256k"))
         t_gpu1 = time.perf_counter()
     clocks = clk.summary(t_gpu0, t_gpu1)
     clocks["timed_window_samples"] = clk.count(t0, t1)
@@ -496,6 +586,8 @@ def run_gpu(args):
         }
         if workloads:
             line["workloads"] = workloads
+        if variants:
+            line["variants"] = variants
         if world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD:
             line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
         print(json.dumps(line), flush=True)

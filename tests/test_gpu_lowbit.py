@@ -115,6 +115,7 @@ def test_pack_rows_matches_oracle_packing(bits_c, bits_r):
     exp = np.concatenate([O.pack_codes(codes(x[:, :wl.d_c], sc, bits_c), bits_c),
                           O.pack_codes(codes(x[:, wl.d_c:], sr, bits_r), bits_r)], axis=-1)
     assert np.array_equal(out.cpu().numpy(), exp)
-    # ties went to the even code, and the far value saturated
-    hi = (1 << (bits_c - 1)) - 1
-    assert O.unpack_codes(exp[0], bits_c)[:4].tolist() == [0, 2, -2, hi]
+    # ties went to the even code (then clamped to the range), and the far
+    # value saturated
+    lo, hi = -(1 << (bits_c - 1)), (1 << (bits_c - 1)) - 1
+    assert O.unpack_codes(exp[0], bits_c)[:4].tolist() == [0, min(2, hi), max(-2, lo), hi]
