@@ -24,8 +24,8 @@
 //     a release arrival on its barrier.
 //   - the value CTA (rank 1) holds O = P . c for the 128 heads in all 512
 //     tensor-memory columns.  It streams the same tile's latent columns again
-//     (an L2 hit: the score CTA fetched them moments before) half a page at a
-//     time and issues M=128 x N=256 MMAs with P as the A operand.  Its four
+//     (an L2 hit: the score CTA fetched them moments before) 16 rows at a
+//     time and issues M=128 x N=256 MMAs with P as the A operand.  Its
 //     epilogue warps apply the occasional rescale of O and write the result.
 // Work is split over clusters as contiguous runs of (sequence, query token,
 // head block, tile) units; a cluster writes the final result of a stream it
@@ -37,8 +37,8 @@
 // stage is three such panels.  When the two pages sit next to each other in
 // the pool the stage is one 3-D box; otherwise each page-panel is its own box,
 // which the TMA unit serves at about half the rate (a fixed cost per box).
-// A value slot is half a page's 8 latent panels (one 3-D box); the four
-// slots hold a tile, refilled 32 KB at a time as each slot's MMAs finish.  Rows without
+// A value slot is 16 rows' 8 latent panels (one 3-D box of 16 KB); the
+// eight slots hold a tile, each refilled as soon as its two MMAs finish.  Rows without
 // data (past a sequence's end, behind a bad page id) come from boxes placed
 // past the end of the cache, which the hardware fills with zeros, so NaN in
 // unused rows never reaches a product.  Gathered rows (attended through a
@@ -63,15 +63,16 @@ constexpr int kSlot = kT * 128;          // score panel: 128 rows x 128 B = 16 K
 constexpr int kStagePanels = 3;          // score ring stage: three panels (one 3-D box when
 constexpr int kStage = kStagePanels * kSlot;   //   both pages of the tile are adjacent)
 constexpr int kNStages = 4;              // score-side ring stages (192 KB)
-constexpr int kVRows = 32;               // value slot: 32 rows of a page, 8 latent panels
-constexpr int kVSlot = 8 * kVRows * 128; //   = 32 KB
-constexpr int kNV = 4;                   // value-side ring slots (128 KB)
+constexpr int kVRows = 16;               // value slot: 16 rows of a page, 8 latent panels
+constexpr int kVSlot = 8 * kVRows * 128; //   = 16 KB
+constexpr int kNV = 8;                   // value-side ring slots (128 KB)
 constexpr int kVPerTile = kT / kVRows;   // value slots per tile
 constexpr int kPBuf = 2 * kM * 128;      // P: 128 rows x 128 tokens bf16, two 64-token panels
 constexpr int kHdrFlag = 512;            // header after P: rescale factor per row (512 B),
 constexpr int kMsgStride = 33 * 1024;    //   then one flag word per softmax warp
 constexpr int kEndBytes = 1536;          // per stream end: row sums of both halves, row max
-constexpr int kEpiWarps = 8;             // value CTA: rescale / epilogue warps (2 per lane quarter)
+constexpr int kEpiWarps = 4;             // value CTA: rescale / epilogue warps (4 or 8)
+constexpr int kEpiCols = kDc * 4 / kEpiWarps;   // O columns per epilogue warp
 constexpr int kStageRow = 80;            // epilogue staging row: 16 floats + 16 B pad
 constexpr int kStageWarp = 32 * kStageRow;   // staging: 32 rows x 16 floats per warp
 // score CTA
@@ -93,8 +94,8 @@ constexpr int kBarBytes = 1024;
 constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;   // + alignment slack
 // warp 0 loads, warp 1 issues MMAs; score CTA: warps 2-9 run the softmax (two
 // per TMEM lane quarter, one 64-column half of the tile each); value CTA:
-// warps 2-9 rescale O and write it out (two per lane quarter, one 256-column
-// half of O each); warp 10 of both computes the unit descriptors
+// warps 2 .. 1 + kEpiWarps rescale O and write it out (kEpiCols columns
+// each); warp 10 of both computes the unit descriptors
 constexpr int kThreads = 352;
 constexpr int kProducerWarp = 10;
 constexpr int kSoftWarps = 8;
@@ -123,7 +124,7 @@ struct PlanHeader {
 //   kp   2-D (col, cache row), box {64, 64}: one panel of a page
 //   row  2-D (col, cache row), boxes of 32 >> i rows (i = 0..5) for partial
 //        pages and zero rows past the end of the cache
-//   vp   3-D (col, cache row, panel), box {64, 32, 8}: half a page's latent panels
+//   vp   3-D (col, cache row, panel), box {64, 16, 8}: 16 rows' latent panels
 //   g4   2-D (col, cache row), box {64, 1}: four-row gathers
 struct Maps {
   CUtensorMap q3, qr, k3, kp;
@@ -480,7 +481,7 @@ __device__ __forceinline__ uint64_t visibility(const DecodeArgs& a, const Desc& 
 // Rescale this warp's 32 lanes of O (all 512 columns) by f.
 __device__ __noinline__ void scale_o(uint32_t taddr, float f) {
 #pragma unroll 1
-  for (int c = 0; c < kDc / 2; c += 32) {
+  for (int c = 0; c < kEpiCols; c += 32) {
     float ov[32];
     tmem_ld32(taddr + c, ov);
     tmem_wait_ld();
@@ -1024,12 +1025,12 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
       }
     } else if (warp < 2 + kEpiWarps) {
       // ------------------------------------------------------------ rescale and epilogue
-      // warps 2-5 take columns [0, 256) and warps 6-9 columns [256, 512) of
-      // O; a warp's lane quarter (its rows) is warp & 3
+      // warps 2-5 take columns [0, kEpiCols) of O (with eight warps, warps
+      // 6-9 the rest); a warp's lane quarter (its rows) is warp & 3
       const int quad = warp & 3;
       const int ch = (warp - 2) >> 2;
       const int h = quad * 32 + lane;
-      const int col0 = ch * (kDc / 2);
+      const int col0 = ch * kEpiCols;
       const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16) + col0;
       float4* stage = reinterpret_cast<float4*>(smem + kOffStage + (warp - 2) * kStageWarp);
       int n_str = 0;
@@ -1093,8 +1094,8 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
           tmem_ld32(trow, ov);
           tmem_wait_ld();
 #pragma unroll 1
-          for (int c = 0; c < kDc / 2; c += 32) {
-            if (c + 32 < kDc / 2) tmem_ld32(trow + c + 32, on);
+          for (int c = 0; c < kEpiCols; c += 32) {
+            if (c + 32 < kEpiCols) tmem_ld32(trow + c + 32, on);
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll
@@ -1112,7 +1113,7 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
               }
               __syncwarp();
             }
-            if (c + 32 < kDc / 2) {
+            if (c + 32 < kEpiCols) {
               tmem_wait_ld();
 #pragma unroll
               for (int i = 0; i < 32; ++i) ov[i] = on[i];
