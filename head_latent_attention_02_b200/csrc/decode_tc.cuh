@@ -73,8 +73,8 @@ constexpr int kMsgStride = 33 * 1024;    //   then one flag word per softmax war
 constexpr int kEndBytes = 1536;          // per stream end: row sums of both halves, row max
 constexpr int kEpiWarps = 4;             // value CTA: rescale / epilogue warps (4 or 8)
 constexpr int kEpiCols = kDc * 4 / kEpiWarps;   // O columns per epilogue warp
-constexpr int kStageRow = 80;            // epilogue staging row: 16 floats + 16 B pad
-constexpr int kStageWarp = 32 * kStageRow;   // staging: 32 rows x 16 floats per warp
+constexpr int kStoreCols = 32;           // epilogue: O columns per TMA store box
+constexpr int kStageWarp = 32 * kStoreCols * 4;   // staging: 32 rows x 32 floats per warp
 // score CTA
 constexpr int kOffRing = 0;
 constexpr int kOffQr = kOffRing + kNStages * kStage;           // rotary query panel
@@ -126,10 +126,15 @@ struct PlanHeader {
 //        pages and zero rows past the end of the cache
 //   vp   3-D (col, cache row, panel), box {64, 16, 8}: 16 rows' latent panels
 //   g4   2-D (col, cache row), box {64, 1}: four-row gathers
+//   o    3-D fp32 (col, head, query row) over the whole-stream outputs (o_lat,
+//        or the packed output of a head list), box {32, 32, 1}: heads past
+//        n_h fall outside the map and are not written
+//   part 2-D fp32 (col, partial row), box {32, 32}: split partials
 struct Maps {
   CUtensorMap q3, qr, k3, kp;
   CUtensorMap row[kNumBoxHeights];
   CUtensorMap vp, g4;
+  CUtensorMap o, part;
 };
 
 struct Params {
@@ -141,6 +146,7 @@ struct Params {
   const int* pair_stream;  // stream holding the first unit of each cluster's run
   float* partial;          // [2G x 128, 512] normalised split partials
   float* partial_lse;      // [2G x 128]
+  float* lse_pack;         // head list: [n_q, n_h] lse of whole streams (else null)
   float scale_log2;
 };
 
@@ -1074,55 +1080,50 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
           const bool empty = !(l_tot > 0.f);
           const float inv = empty ? 0.f : 1.f / l_tot;
           const float lse = empty ? -INFINITY : (m_fin + log2f(l_tot)) * 0.6931471805599453f;
-          // Destination of this lane's head row: the split slot's row, or the
-          // output head's row of o_lat (none past n_h or for an invalid id).
-          const int my_head = sp.hb * kM + h < a.n_h ? head_of(a, sp.hb * kM + h) : -1;
-          float* my_dst = !whole ? p.partial + ((size_t)slot * kM + h) * kDc
-                        : my_head >= 0 ? a.o_lat + ((size_t)qi * a.H + my_head) * kDc
-                                       : nullptr;
-          // the rows this lane stores: 8 k + lane / 4 for k = 0..3
-          float* dst_row[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            dst_row[k] = reinterpret_cast<float*>(__shfl_sync(
-                0xffffffffu, reinterpret_cast<unsigned long long>(my_dst), 8 * k + (lane >> 2)));
-          // O rows leave through a per-warp staging tile (rows padded to 80 B):
-          // each lane writes 16 columns of its row, then each store
-          // instruction writes 8 rows x 64 B.  The next 32 columns are read
-          // from tensor memory while this chunk's stores issue.
+          // O leaves through a per-warp staging tile (32 rows x 32 floats,
+          // 128-byte swizzled as the store map expects) by TMA tensor stores:
+          // a whole stream's rows to its heads (the map clips heads past n_h),
+          // a split's rows to the pair's partial slot.  The next 32 columns
+          // are read from tensor memory while a store drains.
+          const int hrow0 = sp.hb * kM + quad * 32;
           float ov[32], on[32];
           tmem_ld32(trow, ov);
           tmem_wait_ld();
 #pragma unroll 1
-          for (int c = 0; c < kEpiCols; c += 32) {
-            if (c + 32 < kEpiCols) tmem_ld32(trow + c + 32, on);
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                stage[lane * (kStageRow / 16) + j] =
-                    make_float4(ov[16 * hh + 4 * j] * inv, ov[16 * hh + 4 * j + 1] * inv,
-                                ov[16 * hh + 4 * j + 2] * inv, ov[16 * hh + 4 * j + 3] * inv);
-              __syncwarp();
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const int rr = 8 * k + (lane >> 2), j = lane & 3;
-                if (dst_row[k])
-                  *reinterpret_cast<float4*>(dst_row[k] + col0 + c + 16 * hh + 4 * j) =
-                      stage[rr * (kStageRow / 16) + j];
-              }
+          for (int c = 0; c < kEpiCols; c += kStoreCols) {
+            if (c + kStoreCols < kEpiCols) tmem_ld32(trow + c + kStoreCols, on);
+            if (c > 0) {
+              if (lane == 0) bulk_wait_read<0>();   // the staging tile is free again
               __syncwarp();
             }
-            if (c + 32 < kEpiCols) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              stage[lane * 8 + (j ^ (lane & 7))] =
+                  make_float4(ov[4 * j] * inv, ov[4 * j + 1] * inv, ov[4 * j + 2] * inv,
+                              ov[4 * j + 3] * inv);
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+              if (whole) tma_store_3d(&mp.o, stage, col0 + c, hrow0, qi);
+              else tma_store_2d(&mp.part, stage, col0 + c, slot * kM + quad * 32);
+              bulk_commit();
+            }
+            if (c + kStoreCols < kEpiCols) {
               tmem_wait_ld();
 #pragma unroll
               for (int i = 0; i < 32; ++i) ov[i] = on[i];
             }
           }
+          if (lane == 0) bulk_wait_all();   // the stores are complete before the merge reads them
+          __syncwarp();
           tc_fence_before();
           if (ch == 0) {
+            const int hr = sp.hb * kM + h;
             if (!whole) p.partial_lse[(size_t)slot * kM + h] = lse;
-            else if (my_head >= 0) a.lse[(size_t)qi * a.H + my_head] = lse;
+            else if (hr < a.n_h) {
+              if (p.lse_pack) p.lse_pack[(size_t)qi * a.n_h + hr] = lse;
+              else a.lse[(size_t)qi * a.H + hr] = lse;
+            }
           }
           ++n_str;
         }
@@ -1295,7 +1296,9 @@ __global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a, int n_hb,
                                                       const int* stream_off,
                                                       const int* stream_bad,
                                                       const float* partial,
-                                                      const float* partial_lse) {
+                                                      const float* partial_lse,
+                                                      const float* o_pack,
+                                                      const float* lse_pack) {
   // a programmatic dependent of the decode kernel: its outputs are complete
   // and visible only after this wait
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -1320,7 +1323,19 @@ __global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a, int n_hb,
   const int C = plan->C;
   const int off = stream_off[s];
   const int g0 = off / C, g1 = (off + T - 1) / C;
-  if (g0 == g1) return;   // one pair covered the stream and wrote it
+  if (g0 == g1) {
+    // one pair covered the stream and wrote it: to o_lat directly, or (head
+    // list) packed by list position, moved here to the listed head's row
+    if (lse_pack) {
+      const size_t prow = (size_t)qi * a.n_h + hb * kM + m;
+      const float4* src = reinterpret_cast<const float4*>(o_pack + prow * kDc);
+      float4* dst = reinterpret_cast<float4*>(o);
+#pragma unroll
+      for (int i = 0; i < kDc / 128; ++i) dst[lane + 32 * i] = src[lane + 32 * i];
+      if (lane == 0) a.lse[orow] = lse_pack[prow];
+    }
+    return;
+  }
   auto slot_of = [&](int gg) { return 2 * gg + ((off <= gg * C) ? 0 : 1); };
   float lmax = -INFINITY;
   for (int gg = g0 + lane; gg <= g1; gg += 32)

@@ -128,6 +128,22 @@ bool make_map_576(CUtensorMap* m, const void* base, uint64_t rows, int rank, uin
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 store map for decode outputs: (column, row[, plane]) over rows of 512
+// floats, box {32, 32[, 1]}, 128-byte swizzle.  rank 3: rows are heads
+// (extent n_rows) and planes are query rows (stride plane_stride floats).
+bool make_map_out(CUtensorMap* m, float* base, uint64_t n_rows, uint64_t n_planes,
+                  uint64_t plane_stride, int rank) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)tc::kDc, (cuuint64_t)n_rows, (cuuint64_t)n_planes};
+  cuuint64_t strides[2] = {(cuuint64_t)tc::kDc * 4, (cuuint64_t)plane_stride * 4};
+  cuuint32_t box[3] = {(cuuint32_t)tc::kStoreCols, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, (cuuint32_t)rank, base, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 3-D bf16 map over a row-major [rows, cols] matrix seen as (64-column
 // offset, row, 64-column panel), box {64, box_rows, box_panels}, 128-byte
 // swizzle: a box is box_panels panels of box_rows x 128 bytes, and each row of
@@ -227,7 +243,8 @@ mla_status_t launch_wgemm(wg::Params p, const void* w, uint64_t w_rows, uint64_t
 }
 
 struct WsLayout {
-  size_t off_plan, off_streams, off_bad, off_pairs, off_partial, off_plse, off_qpack, total;
+  size_t off_plan, off_streams, off_bad, off_pairs, off_partial, off_plse, off_qpack, off_opack,
+      off_lpack, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -238,8 +255,9 @@ size_t q_pack_bytes(const mla_dims_t* dims, int B, int s_q, int n_ver, int n_h) 
 }
 
 // q_pack_bytes: room for the listed heads' packed queries (mla_decode with a
-// head list).
-WsLayout ws_layout(int n_streams, int G, size_t q_pack_bytes) {
+// head list); o_rows: rows (query x head) of the packed whole-stream outputs
+// of a head list.
+WsLayout ws_layout(int n_streams, int G, size_t q_pack_bytes, size_t o_rows) {
   WsLayout w;
   w.off_plan = 0;
   w.off_streams = align256(sizeof(tc::PlanHeader));
@@ -249,7 +267,9 @@ WsLayout ws_layout(int n_streams, int G, size_t q_pack_bytes) {
   w.off_partial = w.off_pairs + align256(sizeof(int) * (size_t)G);
   w.off_plse = w.off_partial + sizeof(float) * (size_t)tc::kDc * tc::kM * 2 * (size_t)G;
   w.off_qpack = align256(w.off_plse + sizeof(float) * (size_t)tc::kM * 2 * (size_t)G);
-  w.total = w.off_qpack + q_pack_bytes;
+  w.off_opack = align256(w.off_qpack + q_pack_bytes);
+  w.off_lpack = w.off_opack + sizeof(float) * (size_t)tc::kDc * o_rows;
+  w.total = align256(w.off_lpack + sizeof(float) * o_rows);
   return w;
 }
 
@@ -351,7 +371,8 @@ size_t mla_decode_workspace_size(const mla_dims_t* dims, int32_t B, int32_t s_q,
   DeviceInfo* d = nullptr;
   if (device_info(&d) != MLA_OK) return 0;
   const int n_hb = (n_h + tc::kM - 1) / tc::kM;
-  return ws_layout(B * s_q * n_hb, d->num_sms / 2, q_pack_bytes(dims, B, s_q, n_ver, n_h)).total;
+  return ws_layout(B * s_q * n_hb, d->num_sms / 2, q_pack_bytes(dims, B, s_q, n_ver, n_h),
+                   (size_t)B * s_q * n_h).total;
 }
 
 }  // extern "C"
@@ -434,7 +455,8 @@ mla_status_t decode_impl(const mla_dims_t* dims, int32_t B, int32_t s_q, const v
   const int G = dev->num_sms / 2;
   const int n_hb = (n_h + tc::kM - 1) / tc::kM;
   const int n_streams = B * s_q * n_hb;
-  const WsLayout wl = ws_layout(n_streams, G, q_pack_bytes(dims, B, s_q, n_ver, n_h));
+  const WsLayout wl = ws_layout(n_streams, G, q_pack_bytes(dims, B, s_q, n_ver, n_h),
+                                (size_t)B * s_q * n_h);
   if (!workspace || ws_bytes < wl.total) return MLA_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return MLA_ERR_INVALID_ARG;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -484,6 +506,13 @@ mla_status_t decode_impl(const mla_dims_t* dims, int32_t B, int32_t s_q, const v
   int* pair_stream = reinterpret_cast<int*>(ws + wl.off_pairs);
   float* partial = reinterpret_cast<float*>(ws + wl.off_partial);
   float* partial_lse = reinterpret_cast<float*>(ws + wl.off_plse);
+  // whole-stream outputs: straight to o_lat, or packed by list position
+  float* o_pack = head_ids ? reinterpret_cast<float*>(ws + wl.off_opack) : nullptr;
+  float* lse_pack = head_ids ? reinterpret_cast<float*>(ws + wl.off_lpack) : nullptr;
+  if (!make_map_out(&maps.o, head_ids ? o_pack : o_lat, (uint64_t)n_h, (uint64_t)B * s_q,
+                    (uint64_t)(head_ids ? n_h : dims->H) * tc::kDc, 3) ||
+      !make_map_out(&maps.part, partial, (uint64_t)tc::kM * 2 * G, 1, 0, 2))
+    return MLA_ERR_CUDA;
   if (gather)
     tc::plan_kernel<true><<<1, tc::kPlanThreads, 0, st>>>(a, n_hb, G, plan, stream_off,
                                                           stream_bad, pair_stream);
@@ -501,6 +530,7 @@ mla_status_t decode_impl(const mla_dims_t* dims, int32_t B, int32_t s_q, const v
   p.pair_stream = pair_stream;
   p.partial = partial;
   p.partial_lse = partial_lse;
+  p.lse_pack = lse_pack;
   p.scale_log2 = dims->scale * tc::kLog2e;
   // The attention and merge kernels are programmatic dependents of the
   // kernel before them: each may start its set-up early and waits on device
@@ -525,7 +555,9 @@ mla_status_t decode_impl(const mla_dims_t* dims, int32_t B, int32_t s_q, const v
   if (cudaLaunchKernelEx(&cfg, tc::combine_kernel, a, n_hb, static_cast<const tc::PlanHeader*>(plan),
                          static_cast<const int*>(stream_off), static_cast<const int*>(stream_bad),
                          static_cast<const float*>(partial),
-                         static_cast<const float*>(partial_lse)) != cudaSuccess)
+                         static_cast<const float*>(partial_lse),
+                         static_cast<const float*>(o_pack),
+                         static_cast<const float*>(lse_pack)) != cudaSuccess)
     return MLA_ERR_CUDA;
   return launch_ok();
 }
