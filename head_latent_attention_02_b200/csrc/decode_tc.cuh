@@ -48,6 +48,8 @@
 #pragma once
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -489,8 +491,7 @@ __device__ __noinline__ void scale_o(uint32_t taddr, float f) {
 #pragma unroll 1
   for (int c = 0; c < kEpiCols; c += 32) {
     float ov[32];
-    tmem_ld32(taddr + c, ov);
-    tmem_wait_ld();
+    tmem_ld32_sync(taddr + c, ov);
 #pragma unroll
     for (int i = 0; i < 32; ++i) ov[i] *= f;
     tmem_st32(taddr + c, ov);
@@ -843,9 +844,7 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
         if (!wait_warp(&bar->s_full[sb], (it >> 1) & 1)) { fail(ok); break; }
         tc_fence_after();
         float x[64];
-        tmem_ld32(trow + 128 * sb, *reinterpret_cast<float(*)[32]>(x));
-        tmem_ld32(trow + 128 * sb + 32, *reinterpret_cast<float(*)[32]>(x + 32));
-        tmem_wait_ld();
+        tmem_ld64_sync(trow + 128 * sb, *reinterpret_cast<float(*)[2][32]>(x));
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar->s_empty[sb]);
@@ -858,11 +857,20 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
         // of the row, through the partner warp (log2 units)
         // (branch-free: a select per element keeps every element's work in one
         // basic block, so the scheduler can overlap their latencies)
+        // (a half whose 64 rows are all visible takes the loops without the
+        // mask selects: the common case, and fewer instructions beside the
+        // single-thread load and MMA issuers that share these schedulers)
+        const bool all_vis = (v0 & v1) == 0xffffffffu;
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (all_vis) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const bool vb = ((c < 32 ? v0 : v1) >> (c & 31)) & 1u;
-          mx[c & 3] = fmaxf(mx[c & 3], vb ? x[c] : -INFINITY);
+          for (int c = 0; c < 64; ++c) mx[c & 3] = fmaxf(mx[c & 3], x[c]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const bool vb = ((c < 32 ? v0 : v1) >> (c & 31)) & 1u;
+            mx[c & 3] = fmaxf(mx[c & 3], vb ? x[c] : -INFINITY);
+          }
         }
         const float mh = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
         sMax[(sb * 2 + hf) * kM + h] = mh;       // scale > 0: max commutes, -inf stays
@@ -885,25 +893,32 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
         const uint32_t fbar = mapa(smem_u32(&bar->p_full[pb]), 1);
         if (lane == 0) mbar_arrive_expect_tx_cluster(fbar, p_bytes);
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        auto p_pass = [&](auto masked) {
 #pragma unroll
-        for (int c = 0; c < 64; c += 8) {
-          uint32_t pk[4];
+          for (int c = 0; c < 64; c += 8) {
+            uint32_t pk[4];
 #pragma unroll
-          for (int i = 0; i < 8; i += 2) {
-            const int c0 = c + i, c1 = c + i + 1;
-            const bool b0 = any && (((c0 < 32 ? v0 : v1) >> (c0 & 31)) & 1u);
-            const bool b1 = any && (((c1 < 32 ? v0 : v1) >> (c1 & 31)) & 1u);
-            // every element's exponential is taken; the mask only selects
-            const float e0 = ex2_approx(fmaf(x[c0], p.scale_log2, -m_new));
-            const float e1 = ex2_approx(fmaf(x[c1], p.scale_log2, -m_new));
-            const float p0 = b0 ? e0 : 0.f;
-            const float p1 = b1 ? e1 : 0.f;
-            const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-            ls[(i >> 1) & 3] += __low2float(h2) + __high2float(h2);
-            pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
+            for (int i = 0; i < 8; i += 2) {
+              const int c0 = c + i, c1 = c + i + 1;
+              // every element's exponential is taken; the mask only selects
+              float p0 = ex2_approx(fmaf(x[c0], p.scale_log2, -m_new));
+              float p1 = ex2_approx(fmaf(x[c1], p.scale_log2, -m_new));
+              if constexpr (decltype(masked)::value) {
+                const bool b0 = any && (((c0 < 32 ? v0 : v1) >> (c0 & 31)) & 1u);
+                const bool b1 = any && (((c1 < 32 ? v0 : v1) >> (c1 & 31)) & 1u);
+                p0 = b0 ? p0 : 0.f;
+                p1 = b1 ? p1 : 0.f;
+              }
+              const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+              ls[(i >> 1) & 3] += __low2float(h2) + __high2float(h2);
+              pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+            st_async_v4(prow + ((((c >> 3)) ^ (h & 7)) << 4), make_uint4(pk[0], pk[1], pk[2], pk[3]),
+                        fbar);
           }
-          st_async_v4(prow + ((((c >> 3)) ^ (h & 7)) << 4), make_uint4(pk[0], pk[1], pk[2], pk[3]), fbar);
-        }
+        };
+        if (all_vis && any) p_pass(std::false_type{});
+        else p_pass(std::true_type{});
         l_run = l_run * factor + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
         m_run = m_new;
         if (hf == 0) st_async_b32(msg + kPBuf + 4 * h, __float_as_uint(valid ? factor : 1.f), fbar);
@@ -1083,15 +1098,12 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
           // O leaves through a per-warp staging tile (32 rows x 32 floats,
           // 128-byte swizzled as the store map expects) by TMA tensor stores:
           // a whole stream's rows to its heads (the map clips heads past n_h),
-          // a split's rows to the pair's partial slot.  The next 32 columns
-          // are read from tensor memory while a store drains.
+          // a split's rows to the pair's partial slot.
           const int hrow0 = sp.hb * kM + quad * 32;
-          float ov[32], on[32];
-          tmem_ld32(trow, ov);
-          tmem_wait_ld();
+          float ov[32];
 #pragma unroll 1
           for (int c = 0; c < kEpiCols; c += kStoreCols) {
-            if (c + kStoreCols < kEpiCols) tmem_ld32(trow + c + kStoreCols, on);
+            tmem_ld32_sync(trow + c, ov);
             if (c > 0) {
               if (lane == 0) bulk_wait_read<0>();   // the staging tile is free again
               __syncwarp();
@@ -1107,11 +1119,6 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
               if (whole) tma_store_3d(&mp.o, stage, col0 + c, hrow0, qi);
               else tma_store_2d(&mp.part, stage, col0 + c, slot * kM + quad * 32);
               bulk_commit();
-            }
-            if (c + kStoreCols < kEpiCols) {
-              tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 32; ++i) ov[i] = on[i];
             }
           }
           if (lane == 0) bulk_wait_all();   // the stores are complete before the merge reads them

@@ -223,8 +223,7 @@ wgemm_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorM
 #pragma unroll 1
       for (int c0 = 0; c0 < p.n_pad; c0 += 16) {
         float d[16];
-        tmem_ld16(trow + ab * ncols + c0, d);
-        tmem_wait_ld();
+        tmem_ld16_sync(trow + ab * ncols + c0, d);
         const int nq = min(16, p.n - c0);
         if (p.mode == kOutput) {
           float* o = static_cast<float*>(p.out) + (size_t)(p.q0 + c0) * p.d_model + m;
