@@ -1100,25 +1100,35 @@ decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps 
           // a whole stream's rows to its heads (the map clips heads past n_h),
           // a split's rows to the pair's partial slot.
           const int hrow0 = sp.hb * kM + quad * 32;
-          float ov[32];
+          // a lane quarter whose 32 head rows all lie past n_h has nothing
+          // live to write (heads of a partly filled block, e.g. 8 Global
+          // heads): neither its rows of o_lat nor its partial rows are read
+          const int n_store = hrow0 < a.n_h ? kEpiCols : 0;
+          // 64 columns per tensor-memory round trip (two loads, one wait):
+          // the epilogue pays a load's latency, not its size
 #pragma unroll 1
-          for (int c = 0; c < kEpiCols; c += kStoreCols) {
-            tmem_ld32_sync(trow + c, ov);
-            if (c > 0) {
-              if (lane == 0) bulk_wait_read<0>();   // the staging tile is free again
-              __syncwarp();
-            }
+          for (int c0 = 0; c0 < n_store; c0 += 2 * kStoreCols) {
+            float ov[2][32];
+            tmem_ld64_sync(trow + c0, ov);
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              stage[lane * 8 + (j ^ (lane & 7))] =
-                  make_float4(ov[4 * j] * inv, ov[4 * j + 1] * inv, ov[4 * j + 2] * inv,
-                              ov[4 * j + 3] * inv);
-            fence_proxy_async();
-            __syncwarp();
-            if (lane == 0) {
-              if (whole) tma_store_3d(&mp.o, stage, col0 + c, hrow0, qi);
-              else tma_store_2d(&mp.part, stage, col0 + c, slot * kM + quad * 32);
-              bulk_commit();
+            for (int k = 0; k < 2; ++k) {
+              const int c = c0 + k * kStoreCols;
+              if (c > 0) {
+                if (lane == 0) bulk_wait_read<0>();   // the staging tile is free again
+                __syncwarp();
+              }
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                stage[lane * 8 + (j ^ (lane & 7))] =
+                    make_float4(ov[k][4 * j] * inv, ov[k][4 * j + 1] * inv,
+                                ov[k][4 * j + 2] * inv, ov[k][4 * j + 3] * inv);
+              fence_proxy_async();
+              __syncwarp();
+              if (lane == 0) {
+                if (whole) tma_store_3d(&mp.o, stage, col0 + c, hrow0, qi);
+                else tma_store_2d(&mp.part, stage, col0 + c, slot * kM + quad * 32);
+                bulk_commit();
+              }
             }
           }
           if (lane == 0) bulk_wait_all();   // the stores are complete before the merge reads them

@@ -292,27 +292,6 @@ __device__ __forceinline__ void tmem_ld128_sync(uint32_t taddr, float (&v)[4][32
     for (int i = 0; i < 32; ++i) v[k][i] = __uint_as_float(r[32 * k + i]);
 }
 
-// Packed fp32 pairs (sm_100 f32x2 arithmetic): one instruction for two lanes
-// of work, rounded as the scalar operations would be.
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void f2_unpack(uint64_t r, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-
 // 2^x on the special-function unit (flushes denormal results to zero).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
