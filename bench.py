@@ -299,6 +299,30 @@ class Problem:
             if ev:
                 ev[3].record(self.stream)
 
+    def step_graphs(self, n):
+        """n one-step CUDA graphs (absorb_q, decode over cache copy i % copies,
+        out_proj), each with its own four timing events recorded inside the
+        graph around the calls: a call's time is then its kernels' span on the
+        device, with no graph-launch gap in it."""
+        import torch
+        p, mla, runner = self.p, self.mla, self.runner
+        graphs, events = [], []
+        for i in range(n):
+            ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                ev[0].record()
+                mla.absorb_q(p.dims, p.q_nope, p.q_rope, p.q_pos, p.deltas, p.w_uk, p.q_abs)
+                ev[1].record()
+                p.cache = self.caches[i % self.n_copies]
+                runner.run_decode(p)
+                ev[2].record()
+                mla.out_proj(p.dims, p.o_lat, p.w_uv, p.w_o, p.v, p.out)
+                ev[3].record()
+            graphs.append(g)
+            events.append(ev)
+        return graphs, events
+
     def per_call_us(self, events):
         """Median over steps of each call's time (µs), from steps' events."""
         a = [e[0].elapsed_time(e[1]) * 1e3 for e in events]
@@ -410,12 +434,15 @@ def measure_workload(name, rank, dev, stream, peaks, src, reps=20, qknorm=False)
     overhead on it)."""
     import torch
     prob = Problem(name, rank, dev, stream)
-    prob.steps(3)
-    ev = []
-    prob.steps(reps, ev)
+    graphs, ev = prob.step_graphs(reps)
+    for g in graphs[:3]:
+        g.replay()
+    for g in graphs:
+        g.replay()
     torch.cuda.synchronize(dev)
     assert prob.mla.get_status(stream) == 0
     t = prob.per_call_us(ev)
+    del graphs
     out = {"decode_us": round(t["decode"], 2), "decode_us_min": round(t["decode_min"], 2),
            "repeats": reps, "cache_bytes": prob.cache_bytes,
            "GB_s": round(prob.cache_bytes / (t["decode"] * 1e-6) / 1e9, 1),
@@ -463,26 +490,37 @@ def run_gpu(args):
         torch.cuda.synchronize(dev)
         assert mla.get_status(stream) == 0
 
-        # --- device-timed region: exactly K steps, inputs resident in HBM
-        events = []
+        # --- device-timed region: exactly K steps, inputs resident in HBM.
+        # One graph per step (up to 64, replayed in turn), each with timing
+        # events inside it around its three calls.
+        n_g = min(max(args.steps, 10), 64)
+        graphs, g_events = prob.step_graphs(n_g)
+        for g in graphs[:3]:
+            g.replay()
+        torch.cuda.synchronize(dev)
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
         t0 = time.perf_counter()
-        prob.steps(args.steps, events)
+        start.record(stream)
+        for i in range(args.steps):
+            graphs[i % n_g].replay()
+        stop.record(stream)
         torch.cuda.synchronize(dev)
         t1 = time.perf_counter()
         if world > 1:
             dist.barrier()
         assert mla.get_status(stream) == 0
-        ms_total = events[0][0].elapsed_time(events[-1][3])
-        per_call = prob.per_call_us(events)
-        if len(events) < 10:
-            # fewer than 10 timed steps: the per-call medians come from 10 more
-            more = []
-            prob.steps(10, more)
+        ms_total = start.elapsed_time(stop)
+        if args.steps < n_g:
+            # fewer than 10 timed steps: every graph runs once more, so each
+            # holds a step's times for the per-call medians
+            for g in graphs[args.steps:]:
+                g.replay()
             torch.cuda.synchronize(dev)
-            per_call = prob.per_call_us(more)
+        per_call = prob.per_call_us(g_events)
+        del graphs
 
         # --- end-to-end through the public API with host buffers: each step
         # copies its queries in from pinned memory and reads `out` back
@@ -560,9 +598,9 @@ def run_gpu(args):
                              f"W_O ({wl.d_model * wl.H * wl.d_v * 2 / 1e6:.0f} MB)",
                        "parallelism": f"replica x{world} (independent batches)"},
             "timing": ("value and ms_per_step: the decode call (plan + attention + split "
-                       "merge), median over the K timed steps of CUDA events around its graph "
-                       "inside each step (absorb_q, decode, out_proj graphs replayed in order); "
-                       "step_ms: the whole step, first event to last over K"),
+                       "merge), median over the timed steps of CUDA events recorded inside each "
+                       "step's graph around the call (one graph per step: absorb_q, decode, "
+                       "out_proj); step_ms: K graph replays between two events, divided by K"),
             "step_ms": round(ms_step, 5),
             "step_GB_s": round(job_throughput(cache_bytes, world, ms_step), 2),
             "breakdown_us": {"absorb_q": round(per_call["absorb_q"], 2),
