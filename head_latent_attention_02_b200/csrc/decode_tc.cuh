@@ -103,7 +103,7 @@ constexpr int kProducerWarp = 10;
 constexpr int kSoftWarps = 8;
 constexpr int kTmemCols = 512;
 constexpr int kColQ = 0, kColS = 256;    // score CTA: Q latent (256 columns), S double buffer
-constexpr int kMinChunk = 2;
+constexpr int kMinChunk = 1;
 constexpr int kPlanThreads = 1024;       // planner block (one CTA)
 constexpr int kNumBoxHeights = 6;        // 32, 16, 8, 4, 2, 1 rows
 constexpr float kLog2e = 1.4426950408889634f;

@@ -5,7 +5,7 @@ of the rules' own properties).
 Per (sequence, query token, 128-head block) stream: its tile count --
 ceil(pages / 2) per segment in page mode, ceil(n_gather / 128) for gathered
 rows -- or 0 for an invalid sequence; the exclusive prefix sum of the counts;
-the chunk C of consecutive tiles per CTA pair (ceil(U / G), at least 2, or
+the chunk C of consecutive tiles per CTA pair (ceil(U / G), at least 1, or
 for equal counts T0 > 0 a divisor of T0 with at most G / n_streams parts, or
 a multiple of T0 when there are more streams than pairs, taken when it costs
 at most a quarter more than the even split); the stream of each pair's first
@@ -13,7 +13,7 @@ tile.
 """
 import numpy as np
 
-PAGE, TILE, MIN_CHUNK = 64, 128, 2
+PAGE, TILE, MIN_CHUNK = 64, 128, 1
 
 
 def seq_plan(inp, b):
