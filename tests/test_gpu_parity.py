@@ -428,3 +428,39 @@ def test_bounded_wait_gives_up_with_timeout_status():
     inp = make_inputs(_bf16(B=1, lengths=[300]), seed=17)
     p = _gpu(inp)
     _check_all(inp, p, TOL["bf16"])
+
+
+# ----------------------------------------------------------------- the timed step
+
+def test_graph_captured_step_matches_oracle():
+    # the bench times one CUDA graph per step (absorb_q, decode, out_proj);
+    # replaying such a graph must give the oracle's results, as eager calls do
+    inp = make_inputs(_bf16(B=2, lengths=[700, 130]), seed=18)
+    p = runner.upload(inp)
+    runner.run_step(p)                      # loads the kernels before capture
+    torch.cuda.synchronize()
+    p.o_lat.fill_(float("nan"))
+    p.out.fill_(float("nan"))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        runner.run_step(p)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    assert mla.get_status() == 0
+    _check_all(inp, p, TOL["bf16"])
+
+
+def test_f32_generic_path_wide_score_range():
+    # scores far from |s| ~ 1: the fp32 generic kernel's exponentials must keep
+    # the 1e-5 bar when the softmax is sharp (queries scaled by 8)
+    inp = make_inputs(WORKLOADS["tiny_f32"], seed=19)
+    inp.q_nope = (inp.q_nope * 8).astype(np.float32)
+    inp.q_rope = (inp.q_rope * 8).astype(np.float32)
+    p = _gpu(inp)
+    o_ref, l_ref, v_ref = O.decode(inp)
+    _, out_ref = O.out_proj(o_ref, inp.w_uv, inp.w_o)
+    tol = TOL["f32"]
+    _cmp(p.o_lat.cpu().numpy(), o_ref, tol, "o_lat")
+    _cmp(p.lse.cpu().numpy(), l_ref, tol, "lse", lse=True)
+    _cmp(p.out.cpu().numpy(), out_ref, tol, "out")
