@@ -415,14 +415,30 @@ class Problem:
                 p.dims, bits_c, bits_r, p.B, p.s_q, p.q_abs, p.n_ver, None, p.H, packed[c], sc,
                 sr, p.block_table, p.segs, p.q_pos, p.o_lat, p.lse)) for c in range(n_copies)]
             t = self._median_us(gr, reps)
+            del gr
+            # the tensor-core route: dequantise the whole packed pool into one
+            # bf16 scratch pool, then the tensor-core decode over it
+            dq = torch.empty(mla.lowbit_dequant_bytes(p.dims, p.cache.shape[0]),
+                             dtype=torch.uint8, device=p.cache.device)
+            gt = [self._capture(lambda c=c: mla.decode_lowbit_tc(
+                p.dims, bits_c, bits_r, p.B, p.s_q, p.q_abs, p.n_ver, None, p.H, packed[c], sc,
+                sr, p.block_table, p.segs, p.q_pos, p.o_lat, p.lse, dq, p.workspace))
+                for c in range(n_copies)]
+            t_tc = self._median_us(gt, reps)
+            del gt, dq
             nbytes = self.n_read * row_bytes
+            pool_bytes = n_rows * row_bytes
             out[f"int{bits_c}_int{bits_r}"] = {
                 "row_bytes": row_bytes, "decode_us": round(t, 2), "packed_bytes": nbytes,
                 "GB_s": round(nbytes / (t * 1e-6) / 1e9, 1),
                 "frac_of_hbm": round(nbytes / (t * 1e-6) / 1e9 / _peaks()[0]["hbm_gbs"], 4),
                 "kernel": "decode_lowbit_kernel (SIMT, one CTA per head and query row)",
+                "tc_route_us": round(t_tc, 2),
+                "tc_route": "dequant_rows_kernel over the whole packed pool ({:.1f} MB) into a "
+                            "bf16 scratch pool, then the tensor-core decode".format(
+                                pool_bytes / 1e6),
                 "repeats": reps}
-            del gr, packed
+            del packed
         torch.cuda.empty_cache()
         return out
 

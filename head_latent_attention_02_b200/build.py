@@ -8,9 +8,9 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libmla.so")
 SOURCES = ["csrc/mla_lib.cu", "csrc/mla_static_ws.cu", "csrc/mla_append.cu",
-           "csrc/mla_qknorm.cu"]
+           "csrc/mla_qknorm.cu", "csrc/mla_lowbit_tc.cu"]
 DEPENDS = ["csrc/mla_lib.cu", "csrc/mla_static_ws.cu", "csrc/mla_append.cu", "csrc/mla_qknorm.cu",
-           "csrc/common.cuh",
+           "csrc/mla_lowbit_tc.cu", "csrc/common.cuh",
            "csrc/ptx.cuh", "csrc/kernels_simt.cuh", "csrc/kernels_lowbit.cuh", "csrc/wgemm.cuh", "csrc/decode_tc.cuh", "../include/mla.h"]
 
 NVCC_FLAGS = [

@@ -61,6 +61,11 @@ _SIGS = {
     "mla_decode_lowbit": ([ctypes.POINTER(Dims), _i32, _i32, _i32, _i32, _vp, _i32, _vp, _i32,
                            _vp, _vp, _vp, _i64, _vp, _i32, _vp, _i32, _vp, _vp, _i32, _vp, _vp,
                            _vp, _vp], _i32),
+    "mla_lowbit_dequant_bytes": ([ctypes.POINTER(Dims), _i64], _sz),
+    "mla_dequant_rows": ([ctypes.POINTER(Dims), _i32, _i32, _i64, _vp, _vp, _vp, _vp, _vp], _i32),
+    "mla_decode_lowbit_tc": ([ctypes.POINTER(Dims), _i32, _i32, _i32, _i32, _vp, _i32, _vp, _i32,
+                              _vp, _vp, _vp, _i64, _vp, _i32, _vp, _i32, _vp, _vp, _i32, _vp, _vp,
+                              _vp, _vp, _sz, _vp, _sz, _vp], _i32),
     "mla_decode_qknorm": ([ctypes.POINTER(Dims), _i32, _i32, _vp, _i32, _vp, _i32, _vp, _vp, _i64,
                            _vp, _i32, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
 }
@@ -225,3 +230,31 @@ def decode_lowbit(dims, bits_c, bits_r, B, s_q, q_abs, n_ver, head_ids, n_h, cac
         _p(cache), _p(scale_c), _p(scale_r), cache.shape[0], _p(block_table),
         block_table.shape[1], _p(segs), segs.shape[1], _p(gather_rows), _p(n_gather),
         max_gather, _p(q_pos), _p(o_lat), _p(lse), _s(stream)))
+
+
+def lowbit_dequant_bytes(dims, n_pages):
+    """mla_lowbit_dequant_bytes: bytes of a dequantised pool of n_pages pages."""
+    return lib().mla_lowbit_dequant_bytes(ctypes.byref(dims), n_pages)
+
+
+def dequant_rows(dims, bits_c, bits_r, packed, scale_c, scale_r, out, stream=None):
+    """mla_dequant_rows: packed codes [n, row bytes] -> out [n, d_c + d_r] (dtype)."""
+    _check("mla_dequant_rows", lib().mla_dequant_rows(ctypes.byref(dims), bits_c, bits_r,
+                                                      packed.shape[0], _p(packed), _p(scale_c),
+                                                      _p(scale_r), _p(out), _s(stream)))
+
+
+def decode_lowbit_tc(dims, bits_c, bits_r, B, s_q, q_abs, n_ver, head_ids, n_h, cache, scale_c,
+                     scale_r, block_table, segs, q_pos, o_lat, lse, dequant, workspace,
+                     gather_rows=None, n_gather=None, stream=None):
+    """mla_decode_lowbit_tc over a packed pool cache [n_pages, 64, row bytes]
+    (uint8), dequantising into ``dequant`` and decoding with ``workspace``."""
+    max_gather = gather_rows.shape[1] if gather_rows is not None else 0
+    dq_bytes = dequant.numel() * dequant.element_size()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("mla_decode_lowbit_tc", lib().mla_decode_lowbit_tc(
+        ctypes.byref(dims), bits_c, bits_r, B, s_q, _p(q_abs), n_ver, _p(head_ids), n_h,
+        _p(cache), _p(scale_c), _p(scale_r), cache.shape[0], _p(block_table),
+        block_table.shape[1], _p(segs), segs.shape[1], _p(gather_rows), _p(n_gather),
+        max_gather, _p(q_pos), _p(o_lat), _p(lse), _p(dequant), dq_bytes, _p(workspace),
+        ws_bytes, _s(stream)))

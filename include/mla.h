@@ -355,6 +355,45 @@ mla_status_t mla_decode_lowbit(const mla_dims_t* dims, int32_t bits_c, int32_t b
                                float* lse, mla_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Tensor-core route of the low-bit cache (same packed rows, same scales).
+ *
+ * mla_lowbit_dequant_bytes -- bytes of a pool of n_pages pages of dtype rows
+ *   (n_pages * page_size * (d_c + d_r) * sizeof(dtype)); 0 for bad dims.
+ * mla_dequant_rows -- out[i][k] = code_k(packed[i]) * scale_k, the product in
+ *   fp32, rounded to dims->dtype (round to nearest even for bf16).  packed
+ *   [n_rows, row bytes] 4-byte aligned; out [n_rows, d_c + d_r] 16-byte
+ *   aligned.  Bit pairs and dims as mla_pack_rows; UNSUPPORTED when
+ *   d_c + d_r > 8192.
+ * mla_decode_lowbit_tc -- the result of mla_decode_lowbit computed as
+ *   mla_dequant_rows over the whole packed pool (n_pages * page_size rows)
+ *   into the caller's scratch pool `dequant` (>= mla_lowbit_dequant_bytes,
+ *   256-byte aligned, else MLA_ERR_WORKSPACE / MLA_ERR_INVALID_ARG), then
+ *   mla_decode over that pool with the workspace (its rules and its errors;
+ *   the bf16 decode runs on the tensor cores).  The difference from
+ *   mla_decode_lowbit is where the scales act: here on each dequantised
+ *   element, rounded to dtype; there on the query and the output.  The
+ *   scratch pool's contents afterwards are the dequantised rows (or
+ *   unspecified when the decode refused the call).  Cost: one read of the
+ *   packed pool, one write of the dequantised pool, then the decode, which
+ *   reads the pool back from L2 when it fits there. */
+size_t mla_lowbit_dequant_bytes(const mla_dims_t* dims, int64_t n_pages);
+
+mla_status_t mla_dequant_rows(const mla_dims_t* dims, int32_t bits_c, int32_t bits_r,
+                              int64_t n_rows, const void* packed, const float* scale_c,
+                              const float* scale_r, void* out, mla_stream_t stream);
+
+mla_status_t mla_decode_lowbit_tc(const mla_dims_t* dims, int32_t bits_c, int32_t bits_r,
+                                  int32_t B, int32_t s_q, const void* q_abs, int32_t n_ver,
+                                  const int32_t* head_ids, int32_t n_h, const void* cache,
+                                  const float* scale_c, const float* scale_r, int64_t n_pages,
+                                  const int32_t* block_table, int32_t max_pages,
+                                  const mla_seg_t* segs, int32_t max_segs,
+                                  const int32_t* gather_rows, const int32_t* n_gather,
+                                  int32_t max_gather, const int32_t* q_pos, float* o_lat,
+                                  float* lse, void* dequant, size_t dequant_bytes,
+                                  void* workspace, size_t ws_bytes, mla_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * QK-normed MLA ("QK-Normed MLA" abstract): RMSNorm of the content query and
  * of each token's content keys after the key up-projection, with all heads
  * one group (statistics over H * d_n values).  In the absorbed form the

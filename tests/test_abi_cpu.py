@@ -169,6 +169,31 @@ def test_lowbit_calls_reject_bad_arguments(L):
     assert lb(cache=FAKE + 1) == 1 and lb(sc=None) == 1 and lb(n_h=129) == 1
 
 
+def test_lowbit_tc_calls_reject_bad_arguments(L):
+    f = mla.lib()
+    d = _dims()
+    # pool bytes: pages * 64 rows * 576 channels * 2 bytes (bf16 dims)
+    assert f.mla_lowbit_dequant_bytes(ctypes.byref(d), 3) == 3 * 64 * 576 * 2
+    assert f.mla_lowbit_dequant_bytes(ctypes.byref(d), -1) == 0
+    assert f.mla_lowbit_dequant_bytes(None, 3) == 0
+    dq = lambda bc=4, br=4, n=4, src=FAKE, sc=FAKE, out=FAKE: f.mla_dequant_rows(
+        ctypes.byref(d), bc, br, n, src, sc, FAKE, out, None)
+    assert dq(bc=3) == 2 and dq(br=2) == 2
+    assert dq(n=-1) == 1 and dq(sc=None) == 1
+    assert dq(src=FAKE + 2) == 1 and dq(out=FAKE + 8) == 1       # 4- and 16-byte alignment
+    assert dq(n=0, src=None, sc=None, out=None) == 0
+    big = 3 * 64 * 576 * 2
+    tc = lambda bc=4, n_h=128, q=FAKE, dqp=FAKE, dqb=big: f.mla_decode_lowbit_tc(
+        ctypes.byref(d), bc, 4, 1, 1, q, 1, None, n_h, FAKE, FAKE, FAKE, 3, FAKE, 4, FAKE, 1,
+        None, None, 0, FAKE, FAKE, FAKE, dqp, dqb, FAKE, 0, None)
+    assert tc(bc=8) == 2
+    assert tc(dqp=None) == 3 and tc(dqb=big - 1) == 3           # scratch pool too small
+    assert tc(n_h=129) == 1 and tc(q=None) == 1
+    assert tc(dqp=FAKE + 16) == 1                                 # pool not 256-byte aligned
+    # everything else valid: a zero-byte workspace is refused before any launch
+    assert tc() == 3
+
+
 def test_wait_probe_rejects_bad_arguments(L):
     f = mla.lib()
     assert f.mla_debug_wait_probe(10, FAKE, None) == 1             # below 1 us
