@@ -442,6 +442,49 @@ class Problem:
         torch.cuda.empty_cache()
         return out
 
+    def fold_gemm(self, reps=10):
+        """The folded output projection (W_UV folded into W_O, out = o_lat
+        [n_q, H d_c] x W_fold^T with W_fold [d_model, H d_c]) as a plain
+        cuBLAS bf16 GEMM, against this library's two-GEMM out_proj call on
+        the same rows.  Evidence for the design choice, not a product path:
+        the folded weights are H d_c / (H d_v) = 4x the bytes of W_O."""
+        import torch
+        p, wl = self.p, self.wl
+        try:
+            K = wl.H * wl.d_c
+            n_q = self.inp.n_q
+            g = torch.Generator(device=p.cache.device)
+            g.manual_seed(12)
+            a = torch.randn(n_q, K, generator=g, device=p.cache.device).to(torch.bfloat16)
+            w = torch.empty(wl.d_model, K, dtype=torch.bfloat16, device=p.cache.device)
+            w.normal_(0.0, 0.01, generator=g)
+            out = torch.empty(n_q, wl.d_model, dtype=torch.bfloat16, device=p.cache.device)
+            for _ in range(3):
+                torch.matmul(a, w.t(), out=out)
+            ts = []
+            for _ in range(reps):
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(self.stream)
+                torch.matmul(a, w.t(), out=out)
+                e1.record(self.stream)
+                ts.append((e0, e1))
+            torch.cuda.synchronize()
+            t_fold = float(np.median([x.elapsed_time(y) * 1e3 for x, y in ts]))
+            t_two = self._median_us([self.g_out], reps)
+            w_fold = w.numel() * 2
+            w_two = (p.w_uv.numel() + p.w_o.numel()) * 2
+            del a, w, out
+            torch.cuda.empty_cache()
+            return {"folded_gemm_us": round(t_fold, 2), "out_proj_us": round(t_two, 2),
+                    "folded_weight_bytes": w_fold, "two_gemm_weight_bytes": w_two,
+                    "folded_GB_s": round(w_fold / (t_fold * 1e-6) / 1e9, 1),
+                    "folded_gemm": "torch.matmul (cuBLAS) bf16, [n_q, H*d_c] x [H*d_c, d_model]",
+                    "repeats": reps}
+        except Exception as e:   # a measurement of an alternative; never fails the run
+            torch.cuda.empty_cache()
+            return {"error": f"{type(e).__name__}: {e}"[:200]}
+
     def release(self):
         import torch
         del self.g_abs, self.g_dec, self.g_out, self.caches, self.p
@@ -578,6 +621,7 @@ def run_gpu(args):
         if world == 1 and not args.no_workloads and args.workload == WORKLOAD:
             variants["qknorm"] = prob.qknorm_overhead()
             variants["lowbit"] = prob.lowbit()
+            variants["fold_value_into_output"] = prob.fold_gemm()
         prob.release()
 
         # --- the other configurations, decode only, on this GPU
