@@ -28,7 +28,6 @@
 namespace mla {
 namespace {
 
-
 // The codes of one word as exact floats.  XOR with the sign bit of every
 // field turns code c into c + 2^(B-1) in [0, 2^B); masking puts one field in
 // each byte; a byte permute then builds the float 2^23 + (c + 2^(B-1))
@@ -86,7 +85,7 @@ __device__ __forceinline__ void put8(float* dst, const float* v) {
 // 32 / B channels -- and their scales, held in registers -- never change.
 // A block reads R consecutive packed rows (consecutive threads, consecutive
 // words) and writes R consecutive output rows; kDqUnroll passes' loads are
-// issued before any is decoded.  Threads past R * row_words idle.
+// issued before any is decoded.
 constexpr int kDqUnroll = 4;
 
 template <typename T, int B>
@@ -161,7 +160,8 @@ cudaError_t launch(int bits_c, long long n_rows, const mla_dims_t* d, const void
       return cudaErrorUnknown;
   }
   // rows per pass: the fewest that fill whole warps (32 / gcd(row_words,
-  // 32)), repeated up to ~512 threads; a single row when that exceeds 1024
+  // 32)), repeated up to ~512 threads; when those rows need more than 1024
+  // threads, as many rows as 1024 threads hold (the last warp then partial)
   const int row_words = (d->d_c * bits_c + d->d_r * 4) / 32;
   int g = row_words, b = 32;
   while (b) { const int t = g % b; g = b; b = t; }
